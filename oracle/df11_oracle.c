@@ -1,0 +1,544 @@
+/*
+ * df11_oracle.c -- plain, slow, single-threaded CPU oracle for the DF11 codec.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the CPU
+ * baseline arm of bench.py may load this code.  It shares no source, header,
+ * table or helper with the CUDA library, and the library never calls it.
+ *
+ * Source of the method: the page "DFloat11: Nén suy luận GPU không mất dữ liệu,
+ * giảm LLM xuống còn 70% kích thước" (vi.news.hada.io/topic?id=20542).  Sections
+ * are cited by their headings:
+ *   [Exponent]  "Dư địa nén còn lại trong exponent của BFloat16"
+ *   [Format]    "Định dạng DFloat11"
+ *   [LUT]       "Giải mã dựa trên LUT phân cấp"
+ *   [Kernel]    "Kernel GPU hai giai đoạn và metadata bổ trợ"
+ *
+ * Everything is written as the definition, step by step and bit by bit: the
+ * encoder emits one bit at a time, both decoders consume one bit at a time,
+ * the Huffman builder searches the live node list for its two smallest nodes,
+ * and package-merge keeps explicit item lists with leaf multiplicities.
+ *
+ * Readings where the page is silent (each one is listed with its reason in the
+ * design notes of the repository):
+ *   R1 sign/mantissa byte: sign in bit 7, mantissa in bits 6..0.
+ *   R2 Huffman tie-break: leaves ordered by (count asc, symbol asc) get ids
+ *      0..m-1, internal nodes get ids m, m+1, ... in creation order, and each
+ *      merge takes the two live nodes with the smallest (weight, id).
+ *      One symbol -> length 1.
+ *   R3 length cap (32): if Huffman exceeds it, package-merge with leaves in the
+ *      same order, packages placed after equal-weight leaves, and the first
+ *      2(m-1) items of the last list selected.
+ *   R4 normalisation: the multiset of lengths is handed out again so that
+ *      symbols sorted by (count desc, symbol asc) get lengths in ascending
+ *      order.  Canonical codes follow the DEFLATE convention (RFC 1951 3.2.2).
+ *   R5 bit order: code bits are written most significant first; stream bit k
+ *      is bit (7 - k%8) of byte k/8; the stream is zero-padded to whole
+ *      64-bit chunks.
+ *   R6 gaps: gap[c] = (first code start >= 64c, or total_bits if none) - 64c,
+ *      packed 5 bits per chunk, most significant bit first.
+ *   R7 block positions: 256 chunks per block; pos[b] = number of codes that
+ *      start before bit 64*256*b; pos[B] = n; stored as uint32.
+ *
+ * Parity status: every function here is pinned by a test in
+ * tests/test_oracle_pins.py (closed forms, brute force, textbook identities,
+ * invariants).  The tie-break (R2), the package-merge item order (R3), the
+ * normalisation (R4) and the 256-chunk block (R7) are readings of the page,
+ * not facts printed on it: parity on those is parity with the reading.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_CHUNK_BITS 64u       /* [Kernel]: one thread owns n = 8 bytes   */
+#define OR_BLOCK_CHUNKS 256u    /* R7                                        */
+#define OR_GAP_BITS 5u          /* [Kernel]: gaps lie in [0,31], 5 bits      */
+#define OR_MAX_CAP 32           /* [Kernel]: longest code is 32 bits         */
+
+enum {
+  OR_OK = 0,
+  OR_ERR_ARG = 1,
+  OR_ERR_SYMBOL = 2,   /* a value to encode has no code                  */
+  OR_ERR_CORRUPT = 3,  /* the stream or its metadata is inconsistent     */
+};
+
+/* ------------------------------------------------------------------ */
+/* Step 1: split a BF16 word into its exponent and sign+mantissa byte. */
+/* [Exponent]: 1 sign bit, 8 exponent bits, 7 mantissa bits.           */
+/* [Format]: sign and mantissa are kept as they are, in a byte array.  */
+/* ------------------------------------------------------------------ */
+void oracle_split(const uint16_t *w, uint64_t n, uint8_t *exponent,
+                  uint8_t *sign_mantissa) {
+  for (uint64_t i = 0; i < n; i++) {
+    unsigned word = w[i];
+    unsigned sign = (word >> 15) & 1u;
+    unsigned expo = (word >> 7) & 0xFFu;
+    unsigned mant = word & 0x7Fu;
+    exponent[i] = (uint8_t)expo;
+    sign_mantissa[i] = (uint8_t)((sign << 7) | mant); /* R1 */
+  }
+}
+
+/* The inverse of oracle_split. */
+void oracle_merge(const uint8_t *exponent, const uint8_t *sign_mantissa,
+                  uint64_t n, uint16_t *w) {
+  for (uint64_t i = 0; i < n; i++) {
+    unsigned sign = (sign_mantissa[i] >> 7) & 1u;
+    unsigned mant = sign_mantissa[i] & 0x7Fu;
+    unsigned expo = exponent[i];
+    w[i] = (uint16_t)((sign << 15) | (expo << 7) | mant);
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 2: exponent histogram ([Exponent]: the exponent distribution). */
+/* ------------------------------------------------------------------ */
+void oracle_histogram(const uint8_t *exponent, uint64_t n, uint64_t hist[256]) {
+  for (int s = 0; s < 256; s++) hist[s] = 0;
+  for (uint64_t i = 0; i < n; i++) hist[exponent[i]] += 1;
+}
+
+/* Shannon entropy of the histogram in bits per symbol ([Exponent]). */
+double oracle_entropy(const uint64_t hist[256]) {
+  double total = 0.0, h = 0.0;
+  for (int s = 0; s < 256; s++) total += (double)hist[s];
+  if (total <= 0.0) return 0.0;
+  for (int s = 0; s < 256; s++) {
+    if (hist[s] == 0) continue;
+    double p = (double)hist[s] / total;
+    h -= p * log2(p);
+  }
+  return h;
+}
+
+/* Symbols with nonzero count, ordered by (count asc, symbol asc).
+ * Insertion sort: plain and obviously right for 256 items. */
+static int present_symbols_ascending(const uint64_t hist[256], int order[256]) {
+  int m = 0;
+  for (int s = 0; s < 256; s++) {
+    if (hist[s] == 0) continue;
+    int j = m;
+    while (j > 0) {
+      int prev = order[j - 1];
+      int prev_after = hist[prev] > hist[s] ||
+                       (hist[prev] == hist[s] && prev > s);
+      if (!prev_after) break;
+      order[j] = prev;
+      j--;
+    }
+    order[j] = s;
+    m++;
+  }
+  return m;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 3: Huffman code lengths ([Format]: a Huffman tree built from   */
+/* the exponent distribution; frequent values get short codes).  R2.  */
+/* Returns the longest length (0 when the histogram is empty).         */
+/* ------------------------------------------------------------------ */
+int oracle_huffman_lengths(const uint64_t hist[256], uint8_t len[256]) {
+  int order[256];
+  uint64_t weight[511];
+  int parent[511];
+  int alive[511];
+  for (int s = 0; s < 256; s++) len[s] = 0;
+  int m = present_symbols_ascending(hist, order);
+  if (m == 0) return 0;
+  if (m == 1) {
+    len[order[0]] = 1;
+    return 1;
+  }
+  int nodes = m;
+  for (int i = 0; i < m; i++) {
+    weight[i] = hist[order[i]];
+    parent[i] = -1;
+    alive[i] = 1;
+  }
+  for (int live = m; live > 1; live--) {
+    int pick[2];
+    for (int k = 0; k < 2; k++) {
+      int best = -1;
+      for (int id = 0; id < nodes; id++) {
+        if (!alive[id]) continue;
+        /* ids grow with creation order, so the first live node met with
+           the smallest weight is the one with the smallest (weight, id) */
+        if (best < 0 || weight[id] < weight[best]) best = id;
+      }
+      alive[best] = 0;
+      pick[k] = best;
+    }
+    weight[nodes] = weight[pick[0]] + weight[pick[1]];
+    parent[nodes] = -1;
+    alive[nodes] = 1;
+    parent[pick[0]] = nodes;
+    parent[pick[1]] = nodes;
+    nodes++;
+  }
+  int longest = 0;
+  for (int i = 0; i < m; i++) {
+    int depth = 0;
+    for (int id = i; parent[id] >= 0; id = parent[id]) depth++;
+    len[order[i]] = (uint8_t)depth;
+    if (depth > longest) longest = depth;
+  }
+  return longest;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 3b: optimal length-limited code by package-merge (Larmore and  */
+/* Hirschberg, 1990).  R3.  Every item carries how many times each     */
+/* leaf occurs inside it; a code length is the number of selected      */
+/* items a symbol occurs in.  Returns the longest length, or -1 if the */
+/* cap cannot hold m symbols.                                          */
+/* ------------------------------------------------------------------ */
+typedef struct {
+  uint64_t weight;
+  uint8_t mult[256]; /* multiplicity of each leaf (index into order[]) */
+} pm_item;
+
+int oracle_package_merge(const uint64_t hist[256], int cap, uint8_t len[256]) {
+  int order[256];
+  for (int s = 0; s < 256; s++) len[s] = 0;
+  int m = present_symbols_ascending(hist, order);
+  if (m == 0) return 0;
+  if (cap < 1 || cap > OR_MAX_CAP) return -1;
+  if (m == 1) {
+    len[order[0]] = 1;
+    return 1;
+  }
+  if (cap < 31 && ((uint64_t)1 << cap) < (uint64_t)m) return -1;
+
+  /* a list never holds more than m leaves plus m packages */
+  size_t list_cap = (size_t)2 * (size_t)m;
+  pm_item *prev = (pm_item *)calloc(list_cap, sizeof(pm_item));
+  pm_item *cur = (pm_item *)calloc(list_cap, sizeof(pm_item));
+  pm_item *pkg = (pm_item *)calloc(list_cap, sizeof(pm_item));
+  if (!prev || !cur || !pkg) {
+    free(prev);
+    free(cur);
+    free(pkg);
+    return -1;
+  }
+
+  /* the deepest list (denomination 2^-cap) holds the leaves only */
+  size_t prev_n = 0;
+  for (int i = 0; i < m; i++) {
+    memset(&prev[prev_n], 0, sizeof(pm_item));
+    prev[prev_n].weight = hist[order[i]];
+    prev[prev_n].mult[i] = 1;
+    prev_n++;
+  }
+  for (int level = cap - 1; level >= 1; level--) {
+    /* package consecutive pairs of the list one level deeper */
+    size_t pkg_n = 0;
+    for (size_t k = 0; k + 1 < prev_n; k += 2) {
+      pkg[pkg_n].weight = prev[k].weight + prev[k + 1].weight;
+      for (int i = 0; i < m; i++)
+        pkg[pkg_n].mult[i] = (uint8_t)(prev[k].mult[i] + prev[k + 1].mult[i]);
+      pkg_n++;
+    }
+    /* merge leaves and packages by weight; a leaf goes first on a tie */
+    size_t li = 0, pi = 0, cur_n = 0;
+    while (li < (size_t)m || pi < pkg_n) {
+      int take_leaf;
+      if (li >= (size_t)m) take_leaf = 0;
+      else if (pi >= pkg_n) take_leaf = 1;
+      else take_leaf = hist[order[li]] <= pkg[pi].weight;
+      if (take_leaf) {
+        memset(&cur[cur_n], 0, sizeof(pm_item));
+        cur[cur_n].weight = hist[order[li]];
+        cur[cur_n].mult[li] = 1;
+        li++;
+      } else {
+        cur[cur_n] = pkg[pi];
+        pi++;
+      }
+      cur_n++;
+    }
+    pm_item *t = prev;
+    prev = cur;
+    cur = t;
+    prev_n = cur_n;
+  }
+  /* select the 2(m-1) cheapest items of the shallowest list */
+  size_t take = (size_t)2 * (size_t)(m - 1);
+  int longest = 0;
+  unsigned count[256];
+  for (int i = 0; i < m; i++) count[i] = 0;
+  for (size_t k = 0; k < take && k < prev_n; k++)
+    for (int i = 0; i < m; i++) count[i] += prev[k].mult[i];
+  for (int i = 0; i < m; i++) {
+    len[order[i]] = (uint8_t)count[i];
+    if ((int)count[i] > longest) longest = (int)count[i];
+  }
+  free(prev);
+  free(cur);
+  free(pkg);
+  return longest;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 3c: normalisation (R4).                                        */
+/* ------------------------------------------------------------------ */
+void oracle_normalize_lengths(const uint64_t hist[256], uint8_t len[256]) {
+  int syms[256];
+  int lens[256];
+  int m = 0;
+  for (int s = 0; s < 256; s++)
+    if (len[s] > 0) syms[m++] = s;
+  /* lengths ascending */
+  for (int i = 0; i < m; i++) lens[i] = len[syms[i]];
+  for (int i = 1; i < m; i++)
+    for (int j = i; j > 0 && lens[j - 1] > lens[j]; j--) {
+      int t = lens[j];
+      lens[j] = lens[j - 1];
+      lens[j - 1] = t;
+    }
+  /* symbols by (count desc, symbol asc) */
+  for (int i = 1; i < m; i++)
+    for (int j = i; j > 0; j--) {
+      int a = syms[j - 1], b = syms[j];
+      int swap = hist[a] < hist[b] || (hist[a] == hist[b] && a > b);
+      if (!swap) break;
+      syms[j - 1] = b;
+      syms[j] = a;
+    }
+  for (int i = 0; i < m; i++) len[syms[i]] = (uint8_t)lens[i];
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 3d: canonical codes, DEFLATE convention (RFC 1951 3.2.2).      */
+/* ------------------------------------------------------------------ */
+void oracle_canonical_codes(const uint8_t len[256], uint32_t code[256]) {
+  uint64_t bl_count[OR_MAX_CAP + 1];
+  uint64_t next_code[OR_MAX_CAP + 2];
+  for (int b = 0; b <= OR_MAX_CAP; b++) bl_count[b] = 0;
+  for (int s = 0; s < 256; s++)
+    if (len[s] > 0) bl_count[len[s]]++;
+  uint64_t c = 0;
+  bl_count[0] = 0;
+  for (int bits = 1; bits <= OR_MAX_CAP; bits++) {
+    c = (c + bl_count[bits - 1]) << 1;
+    next_code[bits] = c;
+  }
+  for (int s = 0; s < 256; s++) {
+    code[s] = 0;
+    if (len[s] == 0) continue;
+    code[s] = (uint32_t)next_code[len[s]];
+    next_code[len[s]]++;
+  }
+}
+
+/* Whole codebook: Huffman, cap by package-merge when needed, normalise,
+ * canonical codes.  Returns the longest length, or -1 on a bad cap. */
+int oracle_codebook(const uint64_t hist[256], int cap, uint8_t len[256],
+                    uint32_t code[256]) {
+  int longest = oracle_huffman_lengths(hist, len);
+  if (longest > cap) longest = oracle_package_merge(hist, cap, len);
+  if (longest < 0) return -1;
+  oracle_normalize_lengths(hist, len);
+  oracle_canonical_codes(len, code);
+  return longest;
+}
+
+/* Total number of code bits for a sequence of exponents. */
+int oracle_total_bits(const uint8_t *exponent, uint64_t n, const uint8_t len[256],
+                      uint64_t *total_bits) {
+  uint64_t t = 0;
+  for (uint64_t i = 0; i < n; i++) {
+    if (len[exponent[i]] == 0) return OR_ERR_SYMBOL;
+    t += len[exponent[i]];
+  }
+  *total_bits = t;
+  return OR_OK;
+}
+
+static void put_bit(uint8_t *stream, uint64_t k, unsigned bit) {
+  if (bit) stream[k >> 3] |= (uint8_t)(0x80u >> (k & 7u)); /* R5 */
+}
+
+static unsigned get_bit(const uint8_t *stream, uint64_t k) {
+  return (stream[k >> 3] >> (7u - (unsigned)(k & 7u))) & 1u;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 4: bit-serial encoder.  [Format]: the exponent codes are packed */
+/* into the byte array EncodedExponent.  [Kernel]: per chunk the bit    */
+/* offset of its first code (gaps, R6) and per block the output index   */
+/* of its first code (R7).                                              */
+/* stream must hold 8*C zeroed bytes, gap C bytes, pos B+1 entries,     */
+/* where C = ceil(total_bits/64) and B = ceil(C/256).                   */
+/* ------------------------------------------------------------------ */
+int oracle_encode(const uint8_t *exponent, uint64_t n, const uint8_t len[256],
+                  const uint32_t code[256], uint64_t total_bits, uint8_t *stream,
+                  uint8_t *gap, uint32_t *pos) {
+  uint64_t chunks = (total_bits + OR_CHUNK_BITS - 1) / OR_CHUNK_BITS;
+  uint64_t blocks = (chunks + OR_BLOCK_CHUNKS - 1) / OR_BLOCK_CHUNKS;
+  uint64_t block_bits = (uint64_t)OR_CHUNK_BITS * OR_BLOCK_CHUNKS;
+  if (n > 0xFFFFFFFFull) return OR_ERR_ARG;
+  uint64_t bit = 0, next_chunk = 0, next_block = 0;
+  for (uint64_t i = 0; i < n; i++) {
+    unsigned s = exponent[i];
+    unsigned l = len[s];
+    if (l == 0) return OR_ERR_SYMBOL;
+    uint64_t start = bit;
+    while (next_chunk < chunks && next_chunk * OR_CHUNK_BITS <= start) {
+      gap[next_chunk] = (uint8_t)(start - next_chunk * OR_CHUNK_BITS);
+      next_chunk++;
+    }
+    while (next_block < blocks && next_block * block_bits <= start) {
+      pos[next_block] = (uint32_t)i;
+      next_block++;
+    }
+    for (int k = (int)l - 1; k >= 0; k--) {
+      put_bit(stream, bit, (code[s] >> k) & 1u);
+      bit++;
+    }
+  }
+  if (bit != total_bits) return OR_ERR_ARG;
+  while (next_chunk < chunks) {
+    gap[next_chunk] = (uint8_t)(total_bits - next_chunk * OR_CHUNK_BITS);
+    next_chunk++;
+  }
+  while (next_block < blocks) {
+    pos[next_block] = (uint32_t)n;
+    next_block++;
+  }
+  pos[blocks] = (uint32_t)n;
+  for (uint64_t c = 0; c < chunks; c++)
+    if (gap[c] > 31) return OR_ERR_CORRUPT;
+  return OR_OK;
+}
+
+/* Gaps packed as 5-bit fields, most significant bit first (R6).
+ * packed must hold ceil(5*C/8) zeroed bytes. */
+void oracle_pack_gaps(const uint8_t *gap, uint64_t chunks, uint8_t *packed) {
+  uint64_t k = 0;
+  for (uint64_t c = 0; c < chunks; c++)
+    for (int b = (int)OR_GAP_BITS - 1; b >= 0; b--) {
+      put_bit(packed, k, (gap[c] >> b) & 1u);
+      k++;
+    }
+}
+
+void oracle_unpack_gaps(const uint8_t *packed, uint64_t chunks, uint8_t *gap) {
+  uint64_t k = 0;
+  for (uint64_t c = 0; c < chunks; c++) {
+    unsigned g = 0;
+    for (unsigned b = 0; b < OR_GAP_BITS; b++) {
+      g = (g << 1) | get_bit(packed, k);
+      k++;
+    }
+    gap[c] = (uint8_t)g;
+  }
+}
+
+/* Canonical decoding tables: for every length, the first code, the number
+ * of codes, and where its symbols start in the (length, symbol) order. */
+typedef struct {
+  uint64_t first[OR_MAX_CAP + 1];
+  uint64_t count[OR_MAX_CAP + 1];
+  uint64_t offset[OR_MAX_CAP + 1];
+  int symbol[256];
+} canon_tables;
+
+static void build_canon(const uint8_t len[256], const uint32_t code[256],
+                        canon_tables *t) {
+  for (int l = 0; l <= OR_MAX_CAP; l++) {
+    t->first[l] = 0;
+    t->count[l] = 0;
+    t->offset[l] = 0;
+  }
+  int k = 0;
+  for (int l = 1; l <= OR_MAX_CAP; l++) {
+    t->offset[l] = (uint64_t)k;
+    int first_seen = 0;
+    for (int s = 0; s < 256; s++) {
+      if (len[s] != l) continue;
+      if (!first_seen) {
+        t->first[l] = code[s];
+        first_seen = 1;
+      }
+      t->symbol[k++] = s;
+      t->count[l]++;
+    }
+  }
+}
+
+/* Read one code bit by bit starting at bit p; returns its symbol and sets
+ * *used to its length, or returns -1 when no code matches within 32 bits
+ * or the stream ends first. */
+static int read_one_code(const uint8_t *stream, uint64_t stream_bits, uint64_t p,
+                         const canon_tables *t, unsigned *used) {
+  uint64_t value = 0;
+  for (unsigned l = 1; l <= OR_MAX_CAP; l++) {
+    if (p + l - 1 >= stream_bits) return -1;
+    value = (value << 1) | get_bit(stream, p + l - 1);
+    if (t->count[l] > 0 && value >= t->first[l] &&
+        value - t->first[l] < t->count[l]) {
+      *used = l;
+      return t->symbol[t->offset[l] + (value - t->first[l])];
+    }
+  }
+  return -1;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 5a: bit-serial decode from the start of the stream, n codes.   */
+/* ------------------------------------------------------------------ */
+int oracle_decode_serial(const uint8_t *stream, uint64_t total_bits, uint64_t n,
+                         const uint8_t len[256], const uint32_t code[256],
+                         uint8_t *exponent) {
+  canon_tables t;
+  build_canon(len, code, &t);
+  uint64_t p = 0;
+  for (uint64_t i = 0; i < n; i++) {
+    unsigned used = 0;
+    int s = read_one_code(stream, total_bits, p, &t, &used);
+    if (s < 0) return OR_ERR_CORRUPT;
+    exponent[i] = (uint8_t)s;
+    p += used;
+  }
+  return p == total_bits ? OR_OK : OR_ERR_CORRUPT;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 5b: decode driven by the metadata ([Kernel]): every chunk is    */
+/* started at its gap and decodes the codes that start inside it (a     */
+/* code that runs past the chunk end belongs to the chunk it starts in); */
+/* block b writes from output index pos[b] on.  stream must hold         */
+/* 8*C bytes; no code may run past total_bits.                          */
+/* ------------------------------------------------------------------ */
+int oracle_decode_chunked(const uint8_t *stream, const uint8_t *gap,
+                          const uint32_t *pos,
+                          uint64_t total_bits, uint64_t n, const uint8_t len[256],
+                          const uint32_t code[256], uint8_t *exponent) {
+  canon_tables t;
+  build_canon(len, code, &t);
+  uint64_t chunks = (total_bits + OR_CHUNK_BITS - 1) / OR_CHUNK_BITS;
+  uint64_t blocks = (chunks + OR_BLOCK_CHUNKS - 1) / OR_BLOCK_CHUNKS;
+  if (pos[0] != 0 || pos[blocks] != n) return OR_ERR_CORRUPT;
+  for (uint64_t b = 0; b < blocks; b++) {
+    uint64_t out = pos[b];
+    uint64_t end_chunk = (b + 1) * OR_BLOCK_CHUNKS;
+    if (end_chunk > chunks) end_chunk = chunks;
+    for (uint64_t c = b * OR_BLOCK_CHUNKS; c < end_chunk; c++) {
+      uint64_t chunk_start = c * OR_CHUNK_BITS;
+      uint64_t limit = chunk_start + OR_CHUNK_BITS;
+      if (limit > total_bits) limit = total_bits;
+      if (gap[c] > 31) return OR_ERR_CORRUPT;
+      uint64_t p = chunk_start + gap[c];
+      while (p < limit) {
+        unsigned used = 0;
+        int s = read_one_code(stream, total_bits, p, &t, &used);
+        if (s < 0) return OR_ERR_CORRUPT;
+        if (out >= pos[b + 1]) return OR_ERR_CORRUPT;
+        exponent[out++] = (uint8_t)s;
+        p += used;
+      }
+    }
+    if (out != pos[b + 1]) return OR_ERR_CORRUPT;
+  }
+  return OR_OK;
+}
