@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""DF11 decode benchmark on B200.
+
+One step = one decode launch (df11_decode_block_batch) of a whole
+transformer block: by default the seven matrices of the Llama-3-70B-shaped
+block (855,638,016 BF16 weights, per-matrix codebooks), compressed by this
+library from the seeded synthetic weights of ``workloads``.
+
+Prints ONE JSON line (rank 0).  ``value`` is decoded BF16 output in GB/s
+(2 bytes per weight, 1e9 bytes) summed over all ranks; each rank decodes its
+own replica of the block (independent work, no collective on the data path:
+weak scaling).  Extra keys: roofline of the decode kernel against the
+measured HBM copy bandwidth, compression ratio, the oracle's CPU decode rate
+on a bounded sample, an end-to-end figure through the C ABI with host
+buffers, clocks sampled during the timed region.
+
+``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "DF11 decode output BF16 GB/s & % of HBM roofline (bit-exact); ratio"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
+KERNEL_SOURCE = os.path.join(ROOT, "lossless_bf16_weight_df11_b200", "csrc", "df11_kernels.cu")
+ORACLE_SAMPLE = ("q", "o", "k", "v", "gate")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=5, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="df11", choices=["df11", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-verify", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(workload_name: str):
+    """DRAM bytes per decode launch from a committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    try:
+        kv = {}
+        for line in open(PROFILE_TRAFFIC):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("kernel_sha") != kernel_hash() or kv.get("workload") != workload_name:
+            return None
+        return int(float(kv["traffic_bytes_per_launch"]))
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_decode_rate(mats_np, names):
+    """The CPU oracle (bit-serial, one thread) decoding a bounded sample of the
+    workload: (GB/s of BF16 output, seconds, weights)."""
+    import oracle
+    encs = [oracle.encode(x) for x in mats_np]
+    t0 = time.perf_counter()
+    for x, enc in zip(mats_np, encs):
+        out = oracle.decode(enc)
+        assert np.array_equal(out, x.reshape(-1))
+    dt = time.perf_counter() - t0
+    n = sum(x.size for x in mats_np)
+    return 2 * n / dt / 1e9, dt, n
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    wid = args.workload
+    name = workloads.workload_name(wid)
+    mats = workloads.WORKLOADS[wid][1]
+    # each step: the oracle decodes the smallest matrix of the workload
+    idx = min(range(len(mats)), key=lambda i: int(np.prod(mats[i][1])))
+    x = workloads.matrix(wid, idx).reshape(-1)
+    enc = oracle.encode(x)
+    for _ in range(args.warmup):
+        oracle.decode(enc)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        out = oracle.decode(enc)
+    dt = time.perf_counter() - t0
+    assert np.array_equal(out, x)
+    gbs = 2 * x.size * args.steps / dt / 1e9
+    sample = f"matrix {mats[idx][0]} {mats[idx][1][0]}x{mats[idx][1][1] if len(mats[idx][1]) > 1 else ''} ({x.size} weights) of {name} per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "data": "synthetic",
+        "config": {"workload": name, "weights": int(x.size), "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_df11(args):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        dist = None
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import lossless_bf16_weight_df11_b200 as df11
+    from lossless_bf16_weight_df11_b200 import build as df11_build
+    if not os.path.exists(df11.library_path()):
+        df11_build.build()
+    import lossless_bf16_weight_df11_b200.codec as codec
+
+    wid = args.workload
+    name = workloads.workload_name(wid)
+    mats_def = workloads.WORKLOADS[wid][1]
+    xs = [workloads.matrix(wid, i) for i in range(len(mats_def))]
+    n_total = sum(x.size for x in xs)
+
+    # compress on the GPU (histogram -> codebook -> encode), and time it
+    comp_t0 = time.perf_counter()
+    ws = [torch.from_numpy(x.reshape(-1).view(np.int16)).to(dev) for x in xs]
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    cms = [codec.compress(w) for w in ws]
+    ev1.record()
+    torch.cuda.synchronize()
+    compress_ms = ev0.elapsed_time(ev1)
+    compress_wall = time.perf_counter() - comp_t0
+    read_bytes = sum(m.read_bytes for m in cms)
+    stored = sum(m.stored_bytes for m in cms)
+    ratio = stored / (2 * n_total)
+    algo_bytes = read_bytes + 2 * n_total  # compressed bytes read + BF16 written
+
+    outs = [torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in xs]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    abis = [m.abi() for m in cms]
+    out_ptrs = [o.data_ptr() for o in outs]
+    sh = int(stream.cuda_stream)
+
+    def step():
+        st = df11.df11_decode_block_batch(abis, out_ptrs, status.data_ptr(), sh)
+        if st:
+            raise df11.DF11Error(st, "df11_decode_block_batch")
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise df11.DF11Error(int(status.item()), "decode (device)")
+    bit_exact = None
+    if not args.no_verify:
+        bit_exact = all(torch.equal(o.reshape(-1).view(torch.int16), w) for o, w in zip(outs, ws))
+        if not bit_exact:
+            raise SystemExit("decode is not bit-exact")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            for i in range(args.steps):
+                starts[i].record(stream)
+                step()
+                ends[i].record(stream)
+            t_end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if dist:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    value = 2 * n_total * world * args.steps / (total_ms / 1e3) / 1e9
+    if int(status.item()) != 0:
+        raise df11.DF11Error(int(status.item()), "decode (device)")
+
+    # ---- end to end through the C ABI with host buffers (pinned)
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = end_to_end(torch, df11, codec, cms, xs, dev, args.e2e_steps, dist, world)
+
+    peak, peak_kind = measured_peak()
+    avg_launch_ms = statistics.mean(per_launch_ms)
+    achieved = algo_bytes / (avg_launch_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(name),
+                "peak_kind": peak_kind, "kernel": "decode_kernel",
+                "algorithmic_bytes_per_launch": algo_bytes,
+                "frac_of_8TBps": achieved / 8000.0,
+                "median_launch_ms": statistics.median(per_launch_ms)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = [xs[i] for i, (nm, _) in enumerate(mats_def) if nm in ORACLE_SAMPLE] or xs[:1]
+        gbs, dt, ns = oracle_decode_rate(sample, ORACLE_SAMPLE)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{'+'.join(nm for nm, _ in mats_def if nm in ORACLE_SAMPLE) or 'first matrix'}"
+                         f" of {name}: {ns} weights decoded bit-serially in {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": name, "matrices": len(xs), "weights_per_gpu": int(n_total),
+                       "codebooks": len(xs), "l2": "inputs (2.9 GB) larger than L2; no flush",
+                       "parallelism": f"replica per GPU x{world}"},
+            "weights_per_s": n_total * world * args.steps / (total_ms / 1e3),
+            "ratio": ratio, "bits_per_weight": 16 * ratio, "bit_exact": bit_exact,
+            "compress": {"gpu_ms": compress_ms, "wall_s": compress_wall,
+                         "input_GBps": 2 * n_total / (compress_ms / 1e3) / 1e9},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def end_to_end(torch, df11, codec, cms, xs, dev, steps, dist, world):
+    """Host-resident compressed block -> device (pinned H2D), one decode
+    launch, decoded BF16 -> host (D2H), every step, all timed."""
+    host_parts, dev_parts = [], []
+    h2d = 0
+    for m in cms:
+        for buf in (m.stream, m.gaps, m.block_pos, m.sign_mantissa, m.tables):
+            h = torch.empty(buf.shape, dtype=buf.dtype, pin_memory=True)
+            h.copy_(buf)
+            d = torch.empty_like(buf)
+            host_parts.append(h)
+            dev_parts.append(d)
+            h2d += buf.numel() * buf.element_size()
+    n_total = sum(x.size for x in xs)
+    outs = [torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in xs]
+    host_out = [torch.empty(x.shape, dtype=torch.bfloat16, pin_memory=True) for x in xs]
+    d2h = 2 * n_total
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    abis = []
+    k = 0
+    for m in cms:
+        d_stream, d_gaps, d_pos, d_sm, d_tab = dev_parts[k:k + 5]
+        k += 5
+        a = m.abi()
+        a.stream, a.gaps, a.block_pos = d_stream.data_ptr(), d_gaps.data_ptr(), d_pos.data_ptr()
+        a.sign_mantissa, a.tables = d_sm.data_ptr(), d_tab.data_ptr()
+        abis.append(a)
+    stream = torch.cuda.Stream(device=dev)
+    sh = int(stream.cuda_stream)
+
+    def step():
+        for h, d in zip(host_parts, dev_parts):
+            d.copy_(h, non_blocking=True)
+        st = df11.df11_decode_block_batch(abis, [o.data_ptr() for o in outs], status.data_ptr(), sh)
+        if st:
+            raise df11.DF11Error(st, "df11_decode_block_batch")
+        for o, h in zip(outs, host_out):
+            h.copy_(o, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if dist:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ok = all(torch.equal(h.view(torch.int16).reshape(-1), torch.from_numpy(x.reshape(-1).view(np.int16)))
+             for h, x in zip(host_out, xs))
+    if int(status.item()) != 0 or not ok:
+        raise SystemExit("end-to-end decode is not bit-exact")
+    return {"value": 2 * n_total * world * steps / (ms / 1e3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_df11(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,225 @@
+/*
+ * df11.h -- C ABI of the DF11 lossless BF16 weight codec for NVIDIA B200
+ * (sm_100a).
+ *
+ * The method: the page "DFloat11: Nén suy luận GPU không mất dữ liệu, giảm LLM
+ * xuống còn 70% kích thước" (vi.news.hada.io/topic?id=20542).  Citations below
+ * name its sections:
+ *   [Exponent] "Dư địa nén còn lại trong exponent của BFloat16"
+ *   [Format]   "Định dạng DFloat11"
+ *   [GPU]      "Giải nén tối ưu cho suy luận GPU"
+ *   [LUT]      "Giải mã dựa trên LUT phân cấp"
+ *   [Kernel]   "Kernel GPU hai giai đoạn và metadata bổ trợ"
+ *   [Block]    "Giải nén theo từng transformer block"
+ *
+ * A BF16 weight keeps its sign and 7 mantissa bits verbatim in one byte of the
+ * sign/mantissa plane; its 8-bit exponent is replaced by a canonical Huffman
+ * code built from the exponent histogram and capped at 32 bits.  The codes are
+ * packed into a bitstream read by the decoder in 64-bit chunks, with a 5-bit
+ * gap per chunk (offset of the first code that starts in it) and one 32-bit
+ * output position per block of 256 chunks.
+ *
+ * Format (all little-endian, byte arrays unless stated):
+ *   stream         8*C bytes; code bits most significant first, stream bit k
+ *                  is bit 7-(k%8) of byte k/8; zero padding after total_bits.
+ *                  C = ceil(total_bits/64) chunks.
+ *   gaps           ceil(5C/8) bytes; 5-bit fields, most significant bit first;
+ *                  gap[c] = (first code start >= 64c, else total_bits) - 64c.
+ *   block_pos      uint32[B+1], B = ceil(C/256); block_pos[b] = number of
+ *                  codes starting before bit 16384*b; block_pos[B] = n.
+ *   sign_mantissa  n bytes; (w >> 8 & 0x80) | (w & 0x7F).
+ *   code lengths   256 bytes (the codebook; canonical codes follow, RFC 1951).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers named d_* are device pointers; h_* and plain structs are host
+ *     memory.  The library never allocates device memory: the caller owns
+ *     every buffer (sizes come from df11_encoded_sizes).
+ *   - Device calls are asynchronous on the caller's stream (NULL = the legacy
+ *     default stream) and return a status for argument and launch errors
+ *     only.  Errors found in the data (a corrupt stream, a symbol without a
+ *     code) are written to the caller's device word *d_status (0 = OK; the
+ *     first error wins; the caller zeroes it).
+ *   - Host calls are synchronous and pure.
+ *   - A matrix holds at most DF11_MAX_N values (output positions are 32-bit,
+ *     [Kernel]); larger requests return DF11_ERR_TOO_LARGE.
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DF11_CHUNK_BITS 64u        /* [Kernel]: one thread per n = 8 bytes      */
+#define DF11_BLOCK_CHUNKS 256u     /* chunks (threads) per block of positions   */
+#define DF11_GAP_BITS 5u           /* [Kernel]: gaps in [0,31], 5 bits each      */
+#define DF11_MAX_CODE_LEN 32u      /* [Kernel]/[LUT]: longest code, 32 bits      */
+#define DF11_MAX_N 0xFFFFFFFFull   /* [Kernel]: 32-bit block output positions    */
+#define DF11_MAX_BATCH 32u         /* matrices per decode launch (more = split)  */
+
+/* A CUDA stream (cudaStream_t), passed as an opaque pointer. */
+typedef struct CUstream_st *df11_stream_t;
+
+typedef enum {
+  DF11_OK = 0,
+  DF11_ERR_INVALID_ARG = 1,            /* bad pointer, size, alignment or cap  */
+  DF11_ERR_TOO_LARGE = 2,              /* n > DF11_MAX_N                        */
+  DF11_ERR_CUDA = 3,                   /* a CUDA launch or query failed         */
+  DF11_ERR_CORRUPT = 4,                /* stream/metadata inconsistent          */
+  DF11_ERR_SYMBOL_NOT_IN_CODEBOOK = 5, /* a value to encode has no code         */
+  DF11_ERR_TIMEOUT = 6,                /* a bounded wait inside a kernel ran out */
+  DF11_ERR_NO_DEVICE = 7               /* no usable CUDA device                 */
+} df11_status;
+
+/* Canonical, length-limited code for the 256 exponent values. */
+typedef struct {
+  uint8_t len[256];    /* code length of each exponent value, 0 = no code      */
+  uint32_t code[256];  /* canonical code, right-aligned in len bits            */
+  uint32_t max_len;    /* longest length (<= cap)                              */
+  uint32_t min_len;    /* shortest nonzero length                              */
+  uint32_t n_symbols;  /* number of values with a code                         */
+  uint32_t cap;        /* the length cap the code was built under              */
+} df11_codebook;
+
+/* Byte counts for one matrix.  *_bytes: what the format stores (used for the
+ * compression ratio).  *_alloc: what the device buffers must hold, padded so
+ * the decoder can fetch whole blocks with 16-byte bulk copies. */
+typedef struct {
+  uint64_t n, total_bits, n_chunks, n_blocks;
+  uint64_t stream_bytes, gaps_bytes, block_pos_bytes, sign_mantissa_bytes;
+  uint64_t stored_bytes;       /* sum of the four above + 256 code lengths      */
+  uint64_t stream_alloc, gaps_alloc, block_pos_alloc, sign_mantissa_alloc;
+  uint64_t tables_bytes;       /* df11_build_tables output                      */
+  uint64_t workspace_bytes;    /* df11_encode scratch                           */
+} df11_sizes;
+
+/* One compressed matrix in device memory (non-owning).  Every pointer must be
+ * 16-byte aligned and its buffer at least the *_alloc size. */
+typedef struct {
+  uint64_t n;                  /* number of BF16 values                         */
+  uint64_t total_bits;         /* exponent code bits                            */
+  const uint8_t *stream;       /* EncodedExponent ([Format])                    */
+  const uint8_t *gaps;         /* packed 5-bit gaps ([Kernel])                  */
+  const uint32_t *block_pos;   /* per-block output positions ([Kernel])         */
+  const uint8_t *sign_mantissa;/* PackedSignMantissa ([Format])                 */
+  const void *tables;          /* device copy of df11_build_tables output       */
+  uint32_t min_len;            /* shortest code length (codebook.min_len)       */
+  uint32_t reserved;
+} df11_matrix;
+
+/* Encoder outputs in device memory (sizes from df11_encoded_sizes). */
+typedef struct {
+  uint8_t *stream;
+  uint8_t *gaps;
+  uint32_t *block_pos;
+  uint8_t *sign_mantissa;
+} df11_encoded;
+
+/* Human-readable name of a status code (static string). */
+const char *df11_status_string(df11_status s);
+
+/*
+ * df11_histogram -- 256-bin histogram of the exponent field of n BF16 words.
+ * [Exponent]: the codec starts from the exponent distribution of the weights.
+ *   d_w       n uint16 BF16 bit patterns, 16-byte aligned.
+ *   d_hist256 256 uint64 counts, overwritten.
+ * Two kernel launches (clear, count).  n == 0 writes zeros.
+ */
+df11_status df11_histogram(const uint16_t *d_w, uint64_t n, uint64_t *d_hist256,
+                           df11_stream_t stream);
+
+/*
+ * df11_build_codebook -- host.  [Format]: Huffman code from the exponent
+ * histogram, frequent values short.  [LUT]/[Kernel]: lengths capped at 32.
+ * Huffman with ties broken by (weight, creation order; leaves before internal
+ * nodes), package-merge when the longest code exceeds cap, lengths handed to
+ * symbols by (count desc, value asc), canonical codes (RFC 1951).
+ *   hist256   256 counts (host).   cap  1..32.
+ * Returns DF11_ERR_INVALID_ARG if cap cannot hold the alphabet.  An empty
+ * histogram gives an empty codebook (n_symbols 0).
+ */
+df11_status df11_build_codebook(const uint64_t hist256[256], uint32_t cap,
+                                df11_codebook *out);
+
+/*
+ * df11_encoded_sizes -- host.  Exact sizes of every buffer of a matrix with
+ * histogram hist256 coded by cb: total_bits = sum(hist[e] * len[e]).
+ * Returns DF11_ERR_SYMBOL_NOT_IN_CODEBOOK if a counted value has no code and
+ * DF11_ERR_TOO_LARGE if n > DF11_MAX_N.
+ */
+df11_status df11_encoded_sizes(const df11_codebook *cb, const uint64_t hist256[256],
+                               uint64_t n, df11_sizes *out);
+
+/* Bytes of the decode tables of one codebook (a constant). */
+size_t df11_tables_bytes(void);
+
+/*
+ * df11_build_tables -- host.  Decode tables for cb, written to h_tables
+ * (bytes >= df11_tables_bytes()); the caller copies them to device memory and
+ * points df11_matrix.tables at the copy.  [LUT]: table lookups replace the
+ * bit-serial tree walk; here one 4096-entry table maps the next 12 stream bits
+ * to up to three whole codes, and codes longer than 12 bits go through a
+ * canonical length search.
+ */
+df11_status df11_build_tables(const df11_codebook *cb, void *h_tables, size_t bytes);
+
+/*
+ * df11_encode -- compress n BF16 words.  [Format] + [Kernel].
+ *   d_w           n uint16, 16-byte aligned.
+ *   cb            host codebook (from df11_build_codebook).
+ *   total_bits    from df11_encoded_sizes (checked on the device).
+ *   out           device buffers of at least the *_alloc sizes; overwritten,
+ *                 padding included.
+ *   d_workspace   scratch of sizes.workspace_bytes bytes (16-byte aligned).
+ *   d_status      device word; DF11_ERR_SYMBOL_NOT_IN_CODEBOOK or
+ *                 DF11_ERR_CORRUPT (total_bits mismatch) on data errors.
+ * Three kernel launches: length sums per tile, their prefix sum, packing.
+ */
+df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_codebook *cb,
+                        uint64_t total_bits, const df11_encoded *out, void *d_workspace,
+                        size_t workspace_bytes, uint32_t *d_status, df11_stream_t stream);
+
+/*
+ * df11_decode -- decompress one matrix into BF16.  [GPU], [Kernel].
+ *   m      host struct describing device buffers.
+ *   d_out  n uint16 BF16 words, 16-byte aligned; written in full.
+ *   d_status  DF11_ERR_CORRUPT if a block's decoded count disagrees with its
+ *          stored positions or a code is invalid; DF11_ERR_TIMEOUT if a bulk
+ *          copy did not land within the kernel's wait limit.
+ * One kernel launch (the batch kernel with one matrix).
+ */
+df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32_t *d_status,
+                        df11_stream_t stream);
+
+/*
+ * df11_decode_block_batch -- decompress several matrices (e.g. the seven of a
+ * transformer block) in one launch.  [Block]: all matrices of a block are
+ * decompressed as one batch just before the block's forward pass.
+ *   ms      host array of count matrices, each with its own tables.
+ *   d_outs  host array of count device pointers (16-byte aligned).
+ * One launch per DF11_MAX_BATCH matrices.
+ */
+df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
+                                    uint16_t *const *d_outs, uint32_t *d_status,
+                                    df11_stream_t stream);
+
+/*
+ * df11_validate -- host.  Checks stored metadata before it is trusted:
+ * sizes derived from n and total_bits, every gap <= 31 and below its chunk's
+ * code limit, block positions from 0 to n, non-decreasing, and no block
+ * holding more codes than 256 chunks of codes of length >= min_len can start.
+ *   h_gaps       packed gaps (host copy), >= ceil(5C/8) bytes.
+ *   h_block_pos  B+1 positions (host copy).
+ */
+df11_status df11_validate(uint64_t n, uint64_t total_bits, uint32_t min_len,
+                          const uint8_t *h_gaps, uint64_t gaps_bytes,
+                          const uint32_t *h_block_pos, uint64_t block_pos_count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_H */

@@ -1,0 +1,187 @@
+"""Python binding of the DF11 C ABI (``include/df11.h``).
+
+Argument marshalling only: every entry point of ``libdf11_b200.so`` is exposed
+under its C name with the same arguments (device pointers and streams as
+integers, host structs as ctypes structures).  All codec work happens in the
+library's CUDA kernels and its C++ host code; there is no Python or CPU
+fallback, and loading fails loudly if the library has not been built.
+
+``lossless_bf16_weight_df11_b200.codec`` adds torch-tensor helpers that
+allocate the buffers with PyTorch and call these entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdf11_b200.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "df11.h")
+
+CHUNK_BITS = 64
+BLOCK_CHUNKS = 256
+GAP_BITS = 5
+MAX_CODE_LEN = 32
+MAX_N = 0xFFFFFFFF
+MAX_BATCH = 32
+
+DF11_OK = 0
+DF11_ERR_INVALID_ARG = 1
+DF11_ERR_TOO_LARGE = 2
+DF11_ERR_CUDA = 3
+DF11_ERR_CORRUPT = 4
+DF11_ERR_SYMBOL_NOT_IN_CODEBOOK = 5
+DF11_ERR_TIMEOUT = 6
+DF11_ERR_NO_DEVICE = 7
+
+
+class df11_codebook(ctypes.Structure):
+    _fields_ = [("len", ctypes.c_uint8 * 256), ("code", ctypes.c_uint32 * 256),
+                ("max_len", ctypes.c_uint32), ("min_len", ctypes.c_uint32),
+                ("n_symbols", ctypes.c_uint32), ("cap", ctypes.c_uint32)]
+
+
+class df11_sizes(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_uint64) for name in (
+        "n", "total_bits", "n_chunks", "n_blocks",
+        "stream_bytes", "gaps_bytes", "block_pos_bytes", "sign_mantissa_bytes",
+        "stored_bytes",
+        "stream_alloc", "gaps_alloc", "block_pos_alloc", "sign_mantissa_alloc",
+        "tables_bytes", "workspace_bytes")]
+
+
+class df11_matrix(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_uint64), ("total_bits", ctypes.c_uint64),
+                ("stream", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
+                ("block_pos", ctypes.c_void_p), ("sign_mantissa", ctypes.c_void_p),
+                ("tables", ctypes.c_void_p), ("min_len", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
+
+
+class df11_encoded(ctypes.Structure):
+    _fields_ = [("stream", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
+                ("block_pos", ctypes.c_void_p), ("sign_mantissa", ctypes.c_void_p)]
+
+
+class DF11Error(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {df11_status_string(status)} (status {status})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+_u64p = ctypes.POINTER(ctypes.c_uint64)
+_vp = ctypes.c_void_p
+_u64 = ctypes.c_uint64
+_u32 = ctypes.c_uint32
+
+
+def _declare(lib):
+    sig = {
+        "df11_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "df11_histogram": (ctypes.c_int, [_vp, _u64, _vp, _vp]),
+        "df11_build_codebook": (ctypes.c_int, [_u64p, _u32, ctypes.POINTER(df11_codebook)]),
+        "df11_encoded_sizes": (ctypes.c_int, [ctypes.POINTER(df11_codebook), _u64p, _u64,
+                                              ctypes.POINTER(df11_sizes)]),
+        "df11_tables_bytes": (ctypes.c_size_t, []),
+        "df11_build_tables": (ctypes.c_int, [ctypes.POINTER(df11_codebook), _vp, ctypes.c_size_t]),
+        "df11_encode": (ctypes.c_int, [_vp, _u64, ctypes.POINTER(df11_codebook), _u64,
+                                       ctypes.POINTER(df11_encoded), _vp, ctypes.c_size_t, _vp, _vp]),
+        "df11_decode": (ctypes.c_int, [ctypes.POINTER(df11_matrix), _vp, _vp, _vp]),
+        "df11_decode_block_batch": (ctypes.c_int, [ctypes.POINTER(df11_matrix), _u32,
+                                                   ctypes.POINTER(ctypes.c_void_p), _vp, _vp]),
+        "df11_validate": (ctypes.c_int, [_u64, _u64, _u32, _vp, _u64, _vp, _u64]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load():
+    """Load the built library; raise if it is missing (no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"DF11 CUDA library not built ({LIB_PATH}); run "
+                    "`python -m lossless_bf16_weight_df11_b200.build` or __graft_entry__.build()")
+            _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions declared in include/df11.h."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(df11_\w+)\s*\(", text, re.M)))
+
+
+# ------------------------------------------------------------- entry points
+
+
+def df11_status_string(status: int) -> str:
+    return load().df11_status_string(int(status)).decode()
+
+
+def check(status: int, where: str = "df11") -> None:
+    if status != DF11_OK:
+        raise DF11Error(status, where)
+
+
+def df11_histogram(d_w: int, n: int, d_hist256: int, stream: int = 0) -> int:
+    return load().df11_histogram(d_w, n, d_hist256, stream)
+
+
+def df11_build_codebook(hist256, cap: int = MAX_CODE_LEN):
+    """hist256: 256 counts (any sequence).  Returns (status, df11_codebook)."""
+    h = (ctypes.c_uint64 * 256)(*[int(x) for x in hist256])
+    cb = df11_codebook()
+    st = load().df11_build_codebook(h, cap, ctypes.byref(cb))
+    return st, cb
+
+
+def df11_encoded_sizes(cb: df11_codebook, hist256, n: int):
+    h = (ctypes.c_uint64 * 256)(*[int(x) for x in hist256])
+    out = df11_sizes()
+    st = load().df11_encoded_sizes(ctypes.byref(cb), h, n, ctypes.byref(out))
+    return st, out
+
+
+def df11_tables_bytes() -> int:
+    return int(load().df11_tables_bytes())
+
+
+def df11_build_tables(cb: df11_codebook, h_tables: int, nbytes: int) -> int:
+    return load().df11_build_tables(ctypes.byref(cb), h_tables, nbytes)
+
+
+def df11_encode(d_w: int, n: int, cb: df11_codebook, total_bits: int, out: df11_encoded,
+                d_workspace: int, workspace_bytes: int, d_status: int, stream: int = 0) -> int:
+    return load().df11_encode(d_w, n, ctypes.byref(cb), total_bits, ctypes.byref(out),
+                              d_workspace, workspace_bytes, d_status, stream)
+
+
+def df11_decode(m: df11_matrix, d_out: int, d_status: int, stream: int = 0) -> int:
+    return load().df11_decode(ctypes.byref(m), d_out, d_status, stream)
+
+
+def df11_decode_block_batch(ms, d_outs, d_status: int, stream: int = 0) -> int:
+    arr = (df11_matrix * len(ms))(*ms)
+    outs = (ctypes.c_void_p * len(d_outs))(*[int(p) for p in d_outs])
+    return load().df11_decode_block_batch(arr, len(ms), outs, d_status, stream)
+
+
+def df11_validate(n: int, total_bits: int, min_len: int, h_gaps: int, gaps_bytes: int,
+                  h_block_pos: int, block_pos_count: int) -> int:
+    return load().df11_validate(n, total_bits, min_len, h_gaps, gaps_bytes, h_block_pos,
+                                block_pos_count)

@@ -1,0 +1,233 @@
+"""Torch-tensor helpers over the DF11 C ABI.
+
+PyTorch provides device memory and streams; every step of compression and
+decompression runs in the library (``libdf11_b200.so``): histogram, encode and
+decode in its CUDA kernels, codebook and table construction in its C++ host
+code.  These helpers only allocate buffers, move the 256-entry histogram and
+the small decode tables between host and device, and marshal arguments.
+
+Page: "DFloat11: Nén suy luận GPU không mất dữ liệu, giảm LLM xuống còn 70% kích
+thước" (vi.news.hada.io/topic?id=20542), sections "Định dạng DFloat11" and
+"Giải nén theo từng transformer block".
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from . import (MAX_CODE_LEN, DF11Error, check, df11_build_codebook, df11_build_tables,
+               df11_codebook, df11_decode, df11_decode_block_batch, df11_encode, df11_encoded,
+               df11_encoded_sizes, df11_histogram, df11_matrix, df11_sizes, df11_tables_bytes)
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _as_u16(w: torch.Tensor) -> torch.Tensor:
+    if w.dtype == torch.bfloat16:
+        w = w.view(torch.int16)
+    elif w.dtype not in (torch.int16, torch.uint16):
+        raise TypeError(f"expected bfloat16 (or its 16-bit pattern), got {w.dtype}")
+    if not w.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    return w.contiguous().reshape(-1)
+
+
+@dataclass
+class DF11Matrix:
+    """One compressed matrix resident in device memory."""
+    shape: tuple
+    n: int
+    total_bits: int
+    codebook: df11_codebook
+    sizes: df11_sizes
+    stream: torch.Tensor         # uint8, sizes.stream_alloc
+    gaps: torch.Tensor           # uint8, sizes.gaps_alloc
+    block_pos: torch.Tensor      # int32 (uint32 bits), sizes.block_pos_alloc / 4
+    sign_mantissa: torch.Tensor  # uint8, sizes.sign_mantissa_alloc
+    tables: torch.Tensor         # uint8, df11_tables_bytes()
+    hist: np.ndarray = field(repr=False, default=None)
+
+    def abi(self) -> df11_matrix:
+        return df11_matrix(n=self.n, total_bits=self.total_bits, stream=self.stream.data_ptr(),
+                           gaps=self.gaps.data_ptr(), block_pos=self.block_pos.data_ptr(),
+                           sign_mantissa=self.sign_mantissa.data_ptr(),
+                           tables=self.tables.data_ptr(), min_len=max(1, self.codebook.min_len),
+                           reserved=0)
+
+    @property
+    def stored_bytes(self) -> int:
+        """Bytes the format stores (stream, gaps, positions, plane, lengths)."""
+        return int(self.sizes.stored_bytes)
+
+    @property
+    def ratio(self) -> float:
+        return self.stored_bytes / (2 * self.n) if self.n else 0.0
+
+    @property
+    def read_bytes(self) -> int:
+        """Compressed bytes one decode reads (everything but the lengths)."""
+        return int(self.sizes.stored_bytes) - 256
+
+    def host_arrays(self):
+        """Stored arrays copied to the host (for checks and serialisation)."""
+        s = self.sizes
+        return dict(
+            stream=self.stream[: s.stream_bytes].cpu().numpy(),
+            gaps=self.gaps[: s.gaps_bytes].cpu().numpy(),
+            block_pos=self.block_pos[: s.n_blocks + 1].cpu().numpy().view(np.uint32),
+            sign_mantissa=self.sign_mantissa[: s.sign_mantissa_bytes].cpu().numpy(),
+            lengths=np.frombuffer(bytes(self.codebook.len), np.uint8).copy(),
+        )
+
+
+def histogram(w: torch.Tensor, stream=None) -> torch.Tensor:
+    """256 exponent counts (int64 tensor holding uint64 values) on w's device."""
+    u = _as_u16(w)
+    h = torch.empty(256, dtype=torch.int64, device=u.device)
+    with torch.cuda.device(u.device):
+        check(df11_histogram(u.data_ptr(), u.numel(), h.data_ptr(), _stream_handle(stream)),
+              "df11_histogram")
+    return h
+
+
+def build_tables(cb: df11_codebook, device) -> torch.Tensor:
+    nb = df11_tables_bytes()
+    host = np.zeros(nb, np.uint8)
+    check(df11_build_tables(cb, host.ctypes.data, nb), "df11_build_tables")
+    return torch.from_numpy(host).to(device)
+
+
+def alloc_encoded(sizes: df11_sizes, device):
+    return dict(
+        stream=torch.empty(sizes.stream_alloc, dtype=torch.uint8, device=device),
+        gaps=torch.empty(sizes.gaps_alloc, dtype=torch.uint8, device=device),
+        block_pos=torch.empty(sizes.block_pos_alloc // 4, dtype=torch.int32, device=device),
+        sign_mantissa=torch.empty(sizes.sign_mantissa_alloc, dtype=torch.uint8, device=device),
+    )
+
+
+def compress(w: torch.Tensor, cap: int = MAX_CODE_LEN, codebook: df11_codebook | None = None,
+             stream=None, check_status: bool = True) -> DF11Matrix:
+    """BF16 tensor on a CUDA device -> DF11Matrix (GPU histogram, host
+    codebook, GPU encode)."""
+    u = _as_u16(w)
+    dev = u.device
+    sh = _stream_handle(stream)
+    h = histogram(u, stream)
+    hist = h.cpu().numpy().view(np.uint64).copy()
+    if codebook is None:
+        st, codebook = df11_build_codebook(hist, cap)
+        check(st, "df11_build_codebook")
+    st, sizes = df11_encoded_sizes(codebook, hist, u.numel())
+    check(st, "df11_encoded_sizes")
+    bufs = alloc_encoded(sizes, dev)
+    tables = build_tables(codebook, dev)
+    ws = torch.empty(max(16, sizes.workspace_bytes), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = df11_encoded(stream=bufs["stream"].data_ptr(), gaps=bufs["gaps"].data_ptr(),
+                       block_pos=bufs["block_pos"].data_ptr(),
+                       sign_mantissa=bufs["sign_mantissa"].data_ptr())
+    with torch.cuda.device(dev):
+        check(df11_encode(u.data_ptr(), u.numel(), codebook, sizes.total_bits, out,
+                          ws.data_ptr(), ws.numel(), status.data_ptr(), sh), "df11_encode")
+    if check_status:
+        s = int(status.item())
+        if s:
+            raise DF11Error(s, "df11_encode (device)")
+    return DF11Matrix(shape=tuple(w.shape), n=u.numel(), total_bits=int(sizes.total_bits),
+                      codebook=codebook, sizes=sizes, tables=tables, hist=hist, **bufs)
+
+
+def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    dev = m.stream.device
+    if out is None:
+        out = torch.empty(m.shape, dtype=torch.bfloat16, device=dev)
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        check(df11_decode(m.abi(), out.data_ptr(), status.data_ptr(), _stream_handle(stream)),
+              "df11_decode")
+    if own_status:
+        s = int(status.item())
+        if s:
+            raise DF11Error(s, "df11_decode (device)")
+    return out
+
+
+def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=None):
+    """Decode every matrix of a block in one launch."""
+    dev = ms[0].stream.device
+    if outs is None:
+        outs = [torch.empty(m.shape, dtype=torch.bfloat16, device=dev) for m in ms]
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        check(df11_decode_block_batch([m.abi() for m in ms], [o.data_ptr() for o in outs],
+                                      status.data_ptr(), _stream_handle(stream)),
+              "df11_decode_block_batch")
+    if own_status:
+        s = int(status.item())
+        if s:
+            raise DF11Error(s, "df11_decode_block_batch (device)")
+    return outs
+
+
+def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, stream, gaps,
+                     block_pos, sign_mantissa, device) -> DF11Matrix:
+    """Upload stored arrays (e.g. produced elsewhere) into padded device
+    buffers ready for decoding."""
+    hist = np.zeros(256, np.uint64)
+    # sizes only depend on n, total_bits and the code lengths' extremes
+    sizes = df11_sizes()
+    C = (total_bits + 63) // 64
+    B = (C + 255) // 256
+    sizes.n, sizes.total_bits, sizes.n_chunks, sizes.n_blocks = n, total_bits, C, B
+    sizes.stream_bytes, sizes.gaps_bytes = 8 * C, (5 * C + 7) // 8
+    sizes.block_pos_bytes, sizes.sign_mantissa_bytes = 4 * (B + 1), n
+    sizes.stored_bytes = sizes.stream_bytes + sizes.gaps_bytes + sizes.block_pos_bytes + n + 256
+    sizes.stream_alloc, sizes.gaps_alloc = 2048 * B + 16, 160 * B + 16
+    sizes.block_pos_alloc = ((4 * (B + 1) + 15) // 16) * 16
+    sizes.sign_mantissa_alloc = ((n + 15) // 16) * 16 + 16
+    sizes.tables_bytes = df11_tables_bytes()
+
+    def padded(a, size, dtype=np.uint8):
+        buf = np.zeros(size // np.dtype(dtype).itemsize, dtype)
+        a = np.asarray(a).view(dtype).reshape(-1)
+        buf[: a.size] = a
+        return torch.from_numpy(buf).to(device)
+
+    return DF11Matrix(shape=tuple(shape), n=n, total_bits=total_bits, codebook=codebook,
+                      sizes=sizes, stream=padded(stream, sizes.stream_alloc),
+                      gaps=padded(gaps, sizes.gaps_alloc),
+                      block_pos=padded(np.asarray(block_pos, np.uint32).view(np.int32),
+                                       sizes.block_pos_alloc, np.int32),
+                      sign_mantissa=padded(sign_mantissa, sizes.sign_mantissa_alloc),
+                      tables=build_tables(codebook, device), hist=hist)
+
+
+def codebook_from_lengths(lengths, codes) -> df11_codebook:
+    cb = df11_codebook()
+    ln = [int(x) for x in lengths]
+    for i in range(256):
+        cb.len[i] = ln[i]
+        cb.code[i] = int(codes[i])
+    nz = [x for x in ln if x]
+    cb.max_len = max(nz) if nz else 0
+    cb.min_len = min(nz) if nz else 0
+    cb.n_symbols = len(nz)
+    cb.cap = MAX_CODE_LEN
+    return cb
+
+
+__all__ = ["DF11Matrix", "histogram", "compress", "decompress", "decompress_block",
+           "build_tables", "alloc_encoded", "from_host_arrays", "codebook_from_lengths",
+           "ctypes"]

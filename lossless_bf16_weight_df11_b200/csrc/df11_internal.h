@@ -1,0 +1,47 @@
+// df11_internal.h -- layouts shared by the host code and the kernels of the
+// DF11 library (not part of the public ABI).
+#pragma once
+
+#include <stdint.h>
+
+namespace df11i {
+
+// Decode tables of one codebook, built on the host by df11_build_tables and
+// copied to shared memory by every decoding CTA.
+//
+// lut: indexed by the next kLutBits stream bits.  Each entry describes the
+// whole codes (at most three) that fit in those bits, decoded greedily:
+//   bits  0..3   bits consumed by those codes (1..12)
+//   bits  4..5   number of codes (1..3); 0 means the first code is longer
+//                than kLutBits bits (or invalid) and the length search below
+//                must be used
+//   bits  8..31  the decoded exponent values, first code in bits 8..15
+// limit/base/sym: canonical decoding of a long code from a 32-bit
+// left-justified window: its length L is the smallest with
+// window < limit[L], its value sym[(window >> (32-L)) + base[L]].
+constexpr int kLutBits = 12;
+constexpr int kLutSize = 1 << kLutBits;
+
+struct alignas(16) DecodeTables {
+  uint32_t lut[kLutSize];
+  uint64_t limit[33];
+  uint32_t base[33];
+  uint8_t codelen[256];
+  uint8_t sym[256];
+  uint32_t max_len;
+  uint32_t min_len;
+  uint32_t n_symbols;
+  uint32_t lut_bits;
+};
+
+static_assert(sizeof(DecodeTables) % 16 == 0, "tables are copied in 16-byte units");
+
+inline uint32_t lut_consumed(uint32_t e) { return e & 0xFu; }
+inline uint32_t lut_count(uint32_t e) { return (e >> 4) & 0x3u; }
+
+// Encoder tile: 256 threads x 16 values.
+constexpr int kEncThreads = 256;
+constexpr int kEncPerThread = 16;
+constexpr int kEncTile = kEncThreads * kEncPerThread;
+
+}  // namespace df11i
