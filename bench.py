@@ -39,6 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
 KERNEL_SOURCE = os.path.join(ROOT, "lossless_bf16_weight_df11_b200", "csrc", "df11_kernels.cu")
 ORACLE_SAMPLE = ("q", "o", "k", "v", "gate")
+CAP = 12  # code-length cap of the benchmarked codebooks (the decode table's reach)
 
 
 def parse():
@@ -51,6 +52,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-verify", action="store_true")
+    ap.add_argument("--cap32", type=int, default=1, help="also time the block coded with cap 32")
     return ap.parse_args()
 
 
@@ -149,7 +151,7 @@ def oracle_decode_rate(mats_np, names):
     """The CPU oracle (bit-serial, one thread) decoding a bounded sample of the
     workload: (GB/s of BF16 output, seconds, weights)."""
     import oracle
-    encs = [oracle.encode(x) for x in mats_np]
+    encs = [oracle.encode(x, cap=CAP) for x in mats_np]
     t0 = time.perf_counter()
     for x, enc in zip(mats_np, encs):
         out = oracle.decode(enc)
@@ -170,7 +172,7 @@ def run_reference(args):
     # each step: the oracle decodes the smallest matrix of the workload
     idx = min(range(len(mats)), key=lambda i: int(np.prod(mats[i][1])))
     x = workloads.matrix(wid, idx).reshape(-1)
-    enc = oracle.encode(x)
+    enc = oracle.encode(x, cap=CAP)
     for _ in range(args.warmup):
         oracle.decode(enc)
     t0 = time.perf_counter()
@@ -223,7 +225,7 @@ def run_df11(args):
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
-    cms = [codec.compress(w) for w in ws]
+    cms = [codec.compress(w, cap=CAP) for w in ws]
     ev1.record()
     torch.cuda.synchronize()
     compress_ms = ev0.elapsed_time(ev1)
@@ -290,6 +292,38 @@ def run_df11(args):
     if args.e2e_steps > 0:
         e2e = end_to_end(torch, df11, codec, cms, xs, dev, args.e2e_steps, dist, world)
 
+    # ---- the same block coded under the format's 32-bit cap (codes longer
+    # than the decode table take the length search): reported beside
+    cap32 = None
+    if args.cap32:
+        cms32 = [codec.compress(w, cap=32) for w in ws]
+        abis32 = [m.abi() for m in cms32]
+        algo32 = sum(m.read_bytes for m in cms32) + 2 * n_total
+
+        def step32():
+            st = df11.df11_decode_block_batch(abis32, out_ptrs, status.data_ptr(), sh)
+            if st:
+                raise df11.DF11Error(st, "df11_decode_block_batch")
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                step32()
+        torch.cuda.synchronize()
+        ok32 = all(torch.equal(o.reshape(-1).view(torch.int16), w) for o, w in zip(outs, ws))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step32()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms32 = e0.elapsed_time(e1) / args.steps
+        cap32 = {"ms_per_step": ms32, "value": 2 * n_total / (ms32 / 1e3) / 1e9, "unit": "GB/s",
+                 "ratio": sum(m.stored_bytes for m in cms32) / (2 * n_total),
+                 "roofline_achieved": algo32 / (ms32 / 1e3) / 1e9, "bit_exact": ok32,
+                 "max_code_len": max(int(m.codebook.max_len) for m in cms32)}
+        del cms32, abis32
+
     peak, peak_kind = measured_peak()
     avg_launch_ms = statistics.mean(per_launch_ms)
     achieved = algo_bytes / (avg_launch_ms / 1e3) / 1e9
@@ -320,7 +354,9 @@ def run_df11(args):
             "ratio": ratio, "bits_per_weight": 16 * ratio, "bit_exact": bit_exact,
             "compress": {"gpu_ms": compress_ms, "wall_s": compress_wall,
                          "input_GBps": 2 * n_total / (compress_ms / 1e3) / 1e9},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "code_len_cap": CAP,
+            "max_code_len": max(int(m.codebook.max_len) for m in cms),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "cap32": cap32,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

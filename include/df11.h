@@ -59,6 +59,10 @@ extern "C" {
 #define DF11_MAX_CODE_LEN 32u      /* [Kernel]/[LUT]: longest code, 32 bits      */
 #define DF11_MAX_N 0xFFFFFFFFull   /* [Kernel]: 32-bit block output positions    */
 #define DF11_MAX_BATCH 32u         /* matrices per decode launch (more = split)  */
+#define DF11_TABLE_BITS 12u        /* reach of the decode table: codebooks whose
+                                      codes are all this short decode on the
+                                      fast path; longer codes (up to 32) take a
+                                      length search.  The codec's default cap.  */
 
 /* A CUDA stream (cudaStream_t), passed as an opaque pointer. */
 typedef struct CUstream_st *df11_stream_t;

@@ -26,6 +26,7 @@ GAP_BITS = 5
 MAX_CODE_LEN = 32
 MAX_N = 0xFFFFFFFF
 MAX_BATCH = 32
+TABLE_BITS = 12  # decode-table reach; the codec's default length cap
 
 DF11_OK = 0
 DF11_ERR_INVALID_ARG = 1

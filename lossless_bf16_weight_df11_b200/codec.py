@@ -18,7 +18,7 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-from . import (MAX_CODE_LEN, DF11Error, check, df11_build_codebook, df11_build_tables,
+from . import (MAX_CODE_LEN, TABLE_BITS, DF11Error, check, df11_build_codebook, df11_build_tables,
                df11_codebook, df11_decode, df11_decode_block_batch, df11_encode, df11_encoded,
                df11_encoded_sizes, df11_histogram, df11_matrix, df11_sizes, df11_tables_bytes)
 
@@ -112,10 +112,19 @@ def alloc_encoded(sizes: df11_sizes, device):
     )
 
 
-def compress(w: torch.Tensor, cap: int = MAX_CODE_LEN, codebook: df11_codebook | None = None,
+DEFAULT_CAP = TABLE_BITS
+
+
+def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | None = None,
              stream=None, check_status: bool = True) -> DF11Matrix:
     """BF16 tensor on a CUDA device -> DF11Matrix (GPU histogram, host
-    codebook, GPU encode)."""
+    codebook, GPU encode).
+
+    cap is the code-length limit.  The default (12, the decode table's
+    reach) lets every code decode on the fast path; for the weight
+    distributions measured here it costs about 0.2% more exponent bits
+    (0.05% of the compressed size) than the 32-bit limit of the format,
+    which remains fully supported (cap=32)."""
     u = _as_u16(w)
     dev = u.device
     sh = _stream_handle(stream)

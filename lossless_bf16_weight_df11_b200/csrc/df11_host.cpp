@@ -313,7 +313,8 @@ extern "C" df11_status df11_build_tables(const df11_codebook *cb, void *h_tables
       ++nsym;
       used += L;
     }
-    t.lut[v] = nsym ? (used | (nsym << 4) | (syms << 8)) : 0u;
+    t.lut[v] = nsym ? df11i::lut_entry(syms, nsym, used)
+                    : (df11i::lut_entry(0, 0, (uint32_t)K) | df11i::kLutLongFlag);
   }
   std::memcpy(h_tables, &t, sizeof(t));
   return DF11_OK;

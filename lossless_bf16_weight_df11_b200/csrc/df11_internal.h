@@ -11,11 +11,15 @@ namespace df11i {
 //
 // lut: indexed by the next kLutBits stream bits.  Each entry describes the
 // whole codes (at most three) that fit in those bits, decoded greedily:
-//   bits  0..3   bits consumed by those codes (1..12)
-//   bits  4..5   number of codes (1..3); 0 means the first code is longer
-//                than kLutBits bits (or invalid) and the length search below
-//                must be used
-//   bits  8..31  the decoded exponent values, first code in bits 8..15
+//   bits  0..23  the decoded exponent values, first code in bits 0..7,
+//                zero beyond the last code
+//   bits 24..25  number of codes (1..3)
+//   bit  26      set when the first code is longer than kLutBits bits (or
+//                invalid); then the count is zero, bits 28..31 hold kLutBits,
+//                and the code must be decoded by the length search below
+//   bits 28..31  bits consumed by those codes (1..kLutBits)
+// (The fields sit where the decoder can read them with a multiply-high:
+// bits consumed = e >> 28, count = (e & 0x03000000) >> 24.)
 // limit/base/sym: canonical decoding of a long code from a 32-bit
 // left-justified window: its length L is the smallest with
 // window < limit[L], its value sym[(window >> (32-L)) + base[L]].
@@ -36,8 +40,11 @@ struct alignas(16) DecodeTables {
 
 static_assert(sizeof(DecodeTables) % 16 == 0, "tables are copied in 16-byte units");
 
-inline uint32_t lut_consumed(uint32_t e) { return e & 0xFu; }
-inline uint32_t lut_count(uint32_t e) { return (e >> 4) & 0x3u; }
+constexpr uint32_t kLutLongFlag = 1u << 26;
+constexpr uint32_t kLutCountMask = 3u << 24;
+inline constexpr uint32_t lut_entry(uint32_t syms, uint32_t count, uint32_t used) {
+  return syms | (count << 24) | (used << 28);
+}
 
 // Encoder tile: 256 threads x 16 values.
 constexpr int kEncThreads = 256;

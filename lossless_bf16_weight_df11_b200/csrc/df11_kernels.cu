@@ -29,6 +29,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <mutex>
 
 #include "df11.h"
@@ -39,7 +40,6 @@ using df11i::DecodeTables;
 namespace {
 
 constexpr int kT = DF11_BLOCK_CHUNKS;  // chunks per block = threads per decode CTA
-constexpr int kLutShift = 64 - df11i::kLutBits;
 constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls
 
 __device__ __forceinline__ void set_status(uint32_t *st, uint32_t code) {
@@ -48,10 +48,6 @@ __device__ __forceinline__ void set_status(uint32_t *st, uint32_t code) {
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
-__device__ __forceinline__ uint64_t bswap64(uint64_t x) {
-  uint32_t lo = (uint32_t)x, hi = (uint32_t)(x >> 32);
-  return ((uint64_t)bswap32(lo) << 32) | bswap32(hi);
-}
 
 // ============================================================ histogram
 
@@ -393,95 +389,141 @@ struct DecMat {
   const DecodeTables *tables;
   uint16_t *out;
   uint64_t n;
-  uint64_t total_bits;
-  uint64_t n_chunks;
+  uint32_t n_chunks;   // C = ceil(total_bits / 64) (< 2^31 for n < 2^32)
+  uint32_t tail_bits;  // code bits in the last chunk, 1..64
 };
 
 struct DecParams {
   DecMat m[DF11_MAX_BATCH];
   uint64_t block_start[DF11_MAX_BATCH + 1];  // prefix sums of blocks per matrix
   uint32_t count;
-  uint32_t stage_cap;  // bytes: max codes per block rounded up to 16
+  uint32_t stage_cap;     // bytes: max codes per block, rounded up to 16
+  uint32_t region_bytes;  // private decode region per thread (odd number of words)
+  uint32_t min_len;       // shortest code of the batch (regions are sized by it)
   uint32_t *status;
 };
 
 constexpr uint32_t kStreamStage = 8 * kT + 16;         // a block of chunks + the next one
 constexpr uint32_t kGapStage = DF11_GAP_BITS * kT / 8;  // 160 B
-constexpr uint32_t kGapStagePad = kGapStage + 16;
-
-struct StageLayout {
-  uint32_t stream, gaps, sm, size;
-};
-
-__host__ __device__ inline StageLayout stage_layout(uint32_t cap) {
-  StageLayout L;
-  L.stream = 0;
-  L.gaps = kStreamStage;
-  L.sm = L.gaps + kGapStagePad;
-  L.size = L.sm + cap + 32;
-  return L;
-}
+constexpr uint32_t kStageBytes = kStreamStage + kGapStage + 16;
 
 struct SmemLayout {
-  uint32_t tables, stage0, stage1, staging, bars, meta, warp, total;
+  uint32_t tables, stage0, stage1, sm, linear, priv, bars, meta, warp, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(uint32_t cap) {
+__host__ __device__ inline SmemLayout smem_layout(uint32_t cap, uint32_t region_bytes) {
   SmemLayout S;
-  StageLayout L = stage_layout(cap);
   S.tables = 0;
   S.stage0 = (uint32_t)sizeof(DecodeTables);
-  S.stage1 = S.stage0 + L.size;
-  S.staging = S.stage1 + L.size;
-  S.bars = S.staging + cap + 16;
-  S.meta = S.bars + 16;
+  S.stage1 = S.stage0 + kStageBytes;
+  S.sm = S.stage1 + kStageBytes;
+  S.linear = S.sm + cap + 32;
+  S.priv = S.linear + cap + 16 + 64;
+  S.bars = S.priv + kT * region_bytes;
+  S.meta = S.bars + 32;
   S.warp = S.meta + 2 * 16;
   S.total = S.warp + 16 * 4;
   return S;
 }
 
+// Per-thread private region: the codes that can start in a chunk
+// (ceil(64/min_len)), two codes of overshoot from the last table entry, and
+// the two spare bytes that entry's unconditional three-byte store may touch;
+// an odd number of 32-bit words so that word j of all 32 lanes of a warp
+// falls in 32 different banks.
+__host__ __device__ constexpr uint32_t region_bytes_for(uint32_t min_len) {
+  return 4 * (((64 + min_len - 1) / min_len + 4 + 3) / 4 +
+              ((((64 + min_len - 1) / min_len + 4 + 3) / 4) % 2 == 0 ? 1 : 0));
+}
+
+// ---- shared memory through 32-bit shared-window addresses
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts8(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void red_or32(uint32_t a, uint32_t v) {
+  asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+// predicated store: the compiler cannot predicate an asm statement itself,
+// so the predicate is passed in and applied inside (no branch)
+__device__ __forceinline__ void sts8_if(uint32_t a, uint32_t v, bool c) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q st.shared.u8 [%0], %1;\n}\n" ::"r"(a),
+               "r"(v), "r"((uint32_t)c)
+               : "memory");
+}
+// (a * b) >> 32 and ((a * b) >> 32) + c: field extraction on the multiply pipe
+__device__ __forceinline__ uint32_t mulhi(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t madhi(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
 
 // Bulk copy global -> shared (TMA, CTA-local, no multicast).  Both addresses
 // 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
 
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase) {
-  const uint32_t a = smem_addr(bar);
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
   for (uint32_t it = 0; it < kWaitLimit; ++it) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, "
         "p;\n}\n"
         : "=r"(done)
-        : "r"(a), "r"(phase)
+        : "r"(bar), "r"(phase)
         : "memory");
     if (done) return true;
   }
   return false;
 }
 
-// Stream bits [p, p+64) of the 128-bit pair (hi, lo), p in [0, 63].
-__device__ __forceinline__ uint64_t window64(uint64_t hi, uint64_t lo, uint32_t p) {
-  return (hi << p) | ((lo >> 1) >> (63 - p));
+// Stream bits [p, p+32) of the chunk words A (bits 0..31), B (32..63) and the
+// next chunk's first word C, p in [0, 63].
+__device__ __forceinline__ uint32_t window32(uint32_t A, uint32_t B, uint32_t C, uint32_t p) {
+  const bool up = p >= 32;
+  return __funnelshift_l(up ? C : B, up ? B : A, p);
 }
 
 // Length of a code longer than the table's reach: the smallest L with
@@ -494,55 +536,35 @@ __device__ __forceinline__ uint32_t long_code_len(uint32_t w32, const DecodeTabl
   return 0;
 }
 
-// Codes of one chunk: those that start in [p, lim).  WRITE = false counts
-// them; WRITE = true also stores their exponents to dst[0..count).
-template <bool WRITE>
-__device__ __forceinline__ uint32_t chunk_codes(uint64_t hi, uint64_t lo, uint32_t p, uint32_t lim,
-                                                const DecodeTables &tab, uint8_t *dst, bool &bad) {
-  uint32_t cnt = 0;
-  while (p < lim) {
-    const uint64_t w = window64(hi, lo, p);
-    const uint32_t e = tab.lut[(uint32_t)(w >> kLutShift)];
-    const uint32_t used = e & 0xFu, ns = (e >> 4) & 0x3u;
-    if (used == 0) {  // first code longer than the table's reach (or invalid)
-      const uint32_t w32 = (uint32_t)(w >> 32);
-      const uint32_t L = long_code_len(w32, tab);
-      if (L == 0) {
-        bad = true;
-        break;
-      }
-      if (WRITE) dst[cnt] = tab.sym[((w32 >> (32 - L)) + tab.base[L]) & 0xFFu];
-      ++cnt;
-      p += L;
-      continue;
-    }
-    if (p + used <= lim) {
-      if (WRITE) {
-        dst[cnt] = (uint8_t)(e >> 8);
-        if (ns > 1) dst[cnt + 1] = (uint8_t)(e >> 16);
-        if (ns > 2) dst[cnt + 2] = (uint8_t)(e >> 24);
-      }
-      cnt += ns;
-      p += used;
-      continue;
-    }
-    // the entry runs past the limit: keep the codes that start before it
-    if (WRITE) dst[cnt] = (uint8_t)(e >> 8);
-    ++cnt;
-    uint32_t q = p + tab.codelen[(e >> 8) & 0xFFu];
-    if (ns > 1 && q < lim) {
-      if (WRITE) dst[cnt] = (uint8_t)(e >> 16);
-      ++cnt;
-      q += tab.codelen[(e >> 16) & 0xFFu];
-      if (ns > 2 && q < lim) {
-        if (WRITE) dst[cnt] = (uint8_t)(e >> 24);
-        ++cnt;
-      }
-    }
-    break;
+// One table step of the fast decoder on window w.  A flagged entry (first
+// code longer than the table's reach) leaves the loop before anything is
+// stored; otherwise the entry's three exponent slots are stored at dst+d
+// (absent slots are zero), d advances by the number of codes and p by the
+// bits they use.
+#define DF11_FAST_STEP(w)                                                   \
+  e = lds32(lut_a + (mulhi((w), 1u << df11i::kLutBits) << 2));              \
+  if (e & df11i::kLutLongFlag) break;                                       \
+  {                                                                         \
+    const uint32_t at = priv_a + d;                                         \
+    sts8(at, e);                                                            \
+    sts8(at + 1, mulhi(e, 1u << 24));                                       \
+    sts8(at + 2, mulhi(e, 1u << 16));                                       \
+    d = madhi(e & df11i::kLutCountMask, 1u << 8, d);                        \
+    p = madhi(e, 1u << 4, p);                                               \
   }
-  return cnt;
-}
+
+// The same step for tables whose codes all fit in kLutBits bits: no flag
+// test, nothing but the loop's exit branches.
+#define DF11_FAST_STEP_NOFLAG(w)                                            \
+  {                                                                         \
+    e = lds32(lut_a + (mulhi((w), 1u << df11i::kLutBits) << 2));            \
+    const uint32_t at = priv_a + d;                                         \
+    sts8(at, e);                                                            \
+    sts8(at + 1, mulhi(e, 1u << 24));                                       \
+    sts8(at + 2, mulhi(e, 1u << 16));                                       \
+    d = madhi(e & df11i::kLutCountMask, 1u << 8, d);                        \
+    p = madhi(e, 1u << 4, p);                                               \
+  }
 
 // 4 exponents + 4 sign/mantissa bytes -> 4 BF16 words (two 32-bit halves).
 __device__ __forceinline__ void merge4(uint32_t e4, uint32_t s4, uint32_t &w01, uint32_t &w23) {
@@ -563,17 +585,73 @@ __device__ __forceinline__ BlockRef locate(const DecParams &P, uint64_t g, uint3
   return BlockRef{m, g - P.block_start[m]};
 }
 
-__global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ DecParams P) {
+// A decoded block waiting for its merge: positions, output, staging.
+struct Pending {
+  uint32_t P0, P1;
+  uint16_t *out;
+  bool ok;
+};
+
+// Merge a decoded block: exponents in the linear row, sign/mantissa bytes in
+// the sm stage.  Thread t takes the whole 8-output groups t, t+256, ...; each
+// is one 16-byte store.  The ragged first and last groups are written
+// element by element by threads 0 and 1.  The row is cleared behind the
+// reads.
+__device__ __forceinline__ void merge_group(uint32_t lin_a, uint32_t smb, uint32_t k, uint4 &r) {
+  const uint2 e8 = lds64(lin_a + 8 * k);
+  sts64(lin_a + 8 * k, 0u, 0u);
+  const uint2 s8 = lds64(smb + 8 * k);
+  merge4(e8.x, s8.x, r.x, r.y);
+  merge4(e8.y, s8.y, r.z, r.w);
+}
+
+__device__ __forceinline__ void merge_block(const Pending &q, uint32_t lin_a, uint32_t sm_a, int t) {
+  const uint32_t base8 = q.P0 & ~7u;
+  const uint32_t smb = sm_a + (base8 - (q.P0 & ~15u));
+  const uint32_t head = q.P0 & 7u;         // outputs of group 0 before the block
+  const uint32_t span8 = q.P1 - base8;     // outputs from base8 to the block's end
+  const uint32_t full0 = head ? 1u : 0u;
+  const uint32_t full1 = span8 >> 3;
+  uint4 *out4 = reinterpret_cast<uint4 *>(q.out + base8);
+  for (uint32_t k = full0 + t; k < full1; k += kT) {
+    uint4 r;
+    merge_group(lin_a, smb, k, r);
+    out4[k] = r;
+  }
+  // ragged first group (thread 0) and last group (thread 1, unless it is
+  // the first one); element j of group k is output base8 + 8k + j
+  const bool last_edge = (span8 & 7u) != 0 && !(head && full1 == 0);
+  if ((t == 0 && head) || (t == 1 && last_edge)) {
+    const uint32_t k = t == 0 ? 0u : full1;
+    const uint32_t lo = t == 0 ? head : 0u;
+    const uint32_t hi = min(8u, span8 - 8 * k);
+    uint4 r;
+    merge_group(lin_a, smb, k, r);
+    const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
+    uint16_t *o = q.out + base8 + 8 * k;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if ((uint32_t)j >= lo && (uint32_t)j < hi) o[j] = (uint16_t)(wv[j >> 1] >> (16 * (j & 1)));
+  }
+}
+
+// MAXW: 32-bit words of a thread's private region.
+template <int MAXW>
+__global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ DecParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t cap = P.stage_cap;
-  const SmemLayout S = smem_layout(cap);
-  const StageLayout L = stage_layout(cap);
-  DecodeTables &tab = *reinterpret_cast<DecodeTables *>(smem + S.tables);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S.bars);
-  uint32_t *meta = reinterpret_cast<uint32_t *>(smem + S.meta);  // [stage][P0, P1, m, -]
+  const SmemLayout S = smem_layout(cap, 4 * MAXW);
+  const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem + S.tables);
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t lut_a = sbase + S.tables;  // lut is the first member
+  const uint32_t codelen_a = sbase + S.tables + (uint32_t)offsetof(DecodeTables, codelen);
+  const uint32_t bar_stage = sbase + S.bars, bar_sm = sbase + S.bars + 16;
+  uint32_t *meta = reinterpret_cast<uint32_t *>(smem + S.meta);  // [stage][P0, P1, m, b]
   uint32_t *warp_tot = reinterpret_cast<uint32_t *>(smem + S.warp);
-  uint8_t *staging = smem + S.staging;
+  const uint32_t lin_a = sbase + S.linear;
+  const uint32_t sm_a = sbase + S.sm;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const uint32_t priv_a = sbase + S.priv + t * (4 * MAXW);
 
   const uint64_t total = P.block_start[P.count];
   const uint64_t g0 = (uint64_t)blockIdx.x * total / gridDim.x;
@@ -583,24 +661,18 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
   // thread 0 fetches the block after next's positions one iteration early
   uint32_t nxt_p0 = 0, nxt_p1 = 0, nxt_m = 0;
   uint32_t hint = 0;
-  auto issue = [&](uint64_t g, uint32_t stage, uint32_t p0, uint32_t p1, uint32_t m) {
+  auto issue_stream = [&](uint64_t g, uint32_t stage, uint32_t p0, uint32_t p1, uint32_t m) {
     const DecMat &M = P.m[m];
     const uint64_t b = g - P.block_start[m];
-    uint8_t *st = smem + (stage ? S.stage1 : S.stage0);
-    // positions are trusted only as far as they stay inside the matrix and
-    // the stage; anything else is flagged as corrupt after the count
-    const bool sane = p1 >= p0 && p1 <= M.n && p1 - p0 <= P.stage_cap;
-    const uint32_t sm_lo = p0 & ~15u;
-    const uint32_t sm_bytes = sane ? (uint32_t)((((uint64_t)p1 + 15u) & ~15ull) - sm_lo) : 0u;
+    const uint32_t st = sbase + (stage ? S.stage1 : S.stage0);
     meta[stage * 4 + 0] = p0;
     meta[stage * 4 + 1] = p1;
     meta[stage * 4 + 2] = m;
     meta[stage * 4 + 3] = (uint32_t)b;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(&bars[stage], kStreamStage + kGapStage + sm_bytes);
-    bulk_g2s(st + L.stream, M.stream + b * (8 * kT), kStreamStage, &bars[stage]);
-    bulk_g2s(st + L.gaps, M.gaps + b * kGapStage, kGapStage, &bars[stage]);
-    if (sm_bytes) bulk_g2s(st + L.sm, M.sm + sm_lo, sm_bytes, &bars[stage]);
+    mbar_expect_tx(bar_stage + 8 * stage, kStreamStage + kGapStage);
+    bulk_g2s(st, M.stream + b * (8 * kT), kStreamStage, bar_stage + 8 * stage);
+    bulk_g2s(st + kStreamStage, M.gaps + b * kGapStage, kGapStage, bar_stage + 8 * stage);
   };
   auto fetch_pos = [&](uint64_t g) {
     BlockRef r = locate(P, g, hint);
@@ -610,117 +682,228 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
     nxt_p1 = __ldg(P.m[r.m].pos + r.b + 1);
   };
 
+  // the linear row and the private regions start zeroed (the row's words are
+  // OR-ed into; a region holds zeros beyond its codes)
+  for (uint32_t k = t; k < (cap + 16) / 4; k += kT) sts32(lin_a + 4 * k, 0u);
+#pragma unroll
+  for (int k = 0; k < MAXW; ++k) sts32(priv_a + 4 * k, 0u);
   if (t == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    mbar_init(bar_stage, 1);
+    mbar_init(bar_stage + 8, 1);
+    mbar_init(bar_sm, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fetch_pos(g0);
-    issue(g0, 0, nxt_p0, nxt_p1, nxt_m);
+    issue_stream(g0, 0, nxt_p0, nxt_p1, nxt_m);
     if (g0 + 1 < g1) fetch_pos(g0 + 1);
   }
   __syncthreads();
 
   uint32_t cur_m = 0xFFFFFFFFu;
+  bool table_ok = false, table_short = false;
+  Pending prev{0, 0, nullptr, false};
   for (uint64_t g = g0, it = 0; g < g1; ++g, ++it) {
     const uint32_t s = (uint32_t)(it & 1);
-    const bool ok_wait = mbar_wait(&bars[s], (uint32_t)((it >> 1) & 1));
-    if (__syncthreads_or(!ok_wait)) {
-      // the only copy in flight is the one just waited for (the next block's
-      // copy is issued after this wait), so the CTA can leave
-      if (t == 0) set_status(P.status, DF11_ERR_TIMEOUT);
-      return;
-    }
+    // [A] the previous block is relocated into the linear row
+    if (it) __syncthreads();
+    const uint32_t *mt = meta + s * 4;
+    const uint32_t P0 = mt[0], P1 = mt[1], m = mt[2], b = mt[3];
+    const DecMat &M = P.m[m];
+    // positions are trusted only as far as they stay inside the matrix and
+    // the staging row; anything else is flagged as corrupt after the count
+    const bool sane = P1 >= P0 && P1 <= M.n && P1 - P0 <= cap;
     if (t == 0 && g + 1 < g1) {
-      issue(g + 1, s ^ 1, nxt_p0, nxt_p1, nxt_m);
+      issue_stream(g + 1, s ^ 1, nxt_p0, nxt_p1, nxt_m);
       if (g + 2 < g1) fetch_pos(g + 2);
     }
-    const uint32_t *mt = meta + s * 4;
-    const uint32_t P0 = mt[0], P1 = mt[1], m = mt[2];
-    const uint64_t b = mt[3];
     if (m != cur_m) {
       // new matrix: its decode tables into shared memory
-      const uint4 *src = reinterpret_cast<const uint4 *>(P.m[m].tables);
-      uint4 *dst = reinterpret_cast<uint4 *>(&tab);
+      const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
+      uint4 *dst = reinterpret_cast<uint4 *>(smem + S.tables);
       for (uint32_t k = t; k < sizeof(DecodeTables) / 16; k += kT) dst[k] = __ldg(src + k);
       cur_m = m;
       __syncthreads();
+      // every table entry must spend at least min_len bits per code, so that
+      // no chunk can produce more codes than its private region holds
+      bool tbad = false;
+      for (uint32_t k = t; k < (uint32_t)df11i::kLutSize; k += kT) {
+        const uint32_t e = tab.lut[k], used = e >> 28, ns = (e >> 24) & 0x3u;
+        tbad |= used == 0 || used < ns * P.min_len;
+      }
+      table_ok = !__syncthreads_or(tbad);
+      // every code fits the table: the decode loop needs no long-code test
+      table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
     }
-    const DecMat &M = P.m[m];
-    const uint8_t *st = smem + (s ? S.stage1 : S.stage0);
+    const uint32_t st = sbase + (s ? S.stage1 : S.stage0);
+    bool timed_out = !mbar_wait(bar_stage + 8 * s, (uint32_t)((it >> 1) & 1));
 
-    // ---- this thread's chunk
-    const uint64_t c = b * kT + t;
-    uint64_t hi = 0, lo = 0;
-    uint32_t p = 0, lim = 0;
-    if (c < M.n_chunks) {
-      const uint64_t *s64 = reinterpret_cast<const uint64_t *>(st + L.stream);
-      hi = bswap64(s64[t]);
-      lo = bswap64(s64[t + 1]);
-      const uint64_t rem = M.total_bits - c * 64;
-      lim = rem < 64 ? (uint32_t)rem : 64u;
-      const uint8_t *gp = st + L.gaps;
-      const uint32_t q = 5u * t;
-      const uint32_t two = ((uint32_t)gp[q >> 3] << 8) | gp[(q >> 3) + 1];
-      p = (two >> (11 - (q & 7u))) & 31u;
-    }
-    // ---- phase 1: count the codes that start in the chunk
+    // ---- this thread's chunk: decode once into the private region
+    const uint32_t c = b * kT + t;
+    uint32_t cnt = 0;
     bool bad = false;
-    const uint32_t cnt = chunk_codes<false>(hi, lo, p, lim, tab, nullptr, bad);
-    // ---- CTA prefix sum of the counts
-    uint32_t incl = cnt;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += o;
-    }
-    const bool warp_bad = __any_sync(0xffffffffu, bad);
-    if (lane == 31) warp_tot[warp] = incl | (warp_bad ? 0x80000000u : 0u);
-    __syncthreads();
-    uint32_t wpre = 0, tot = 0;
-    bool any_bad = false;
-#pragma unroll
-    for (int i = 0; i < kT / 32; ++i) {
-      const uint32_t x = warp_tot[i];
-      any_bad |= (x >> 31) != 0;
-      const uint32_t v = x & 0x7FFFFFFFu;
-      tot += v;
-      if (i < warp) wpre += v;
-    }
-    const bool ok = !any_bad && P1 >= P0 && P1 <= M.n && tot == P1 - P0 && tot <= cap;
-    if (!ok && t == 0) set_status(P.status, DF11_ERR_CORRUPT);
-    // ---- phase 2: decode into the staging row at this thread's offset
-    if (ok) chunk_codes<true>(hi, lo, p, lim, tab, staging + (P0 & 7u) + wpre + incl - cnt, bad);
-    __syncthreads();
-    // ---- merge with the sign/mantissa bytes; 16-byte BF16 stores
-    if (ok) {
-      const uint32_t base8 = P0 & ~7u;
-      const uint32_t sm_lo = P0 & ~15u;
-      const uint32_t ng = (P1 - base8 + 7) >> 3;
-      const uint8_t *smst = st + L.sm;
-      uint16_t *out = M.out;
-      for (uint32_t k = t; k < ng; k += kT) {
-        const uint64_t o = (uint64_t)base8 + 8ull * k;
-        const uint2 e8 = *reinterpret_cast<const uint2 *>(staging + 8 * k);
-        const uint2 s8 = *reinterpret_cast<const uint2 *>(smst + (uint32_t)(o - sm_lo));
-        uint4 r;
-        merge4(e8.x, s8.x, r.x, r.y);
-        merge4(e8.y, s8.y, r.z, r.w);
-        if (o >= P0 && o + 8 <= P1) {
-          *reinterpret_cast<uint4 *>(out + o) = r;
-        } else {
-          const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint64_t oj = o + j;
-            if (oj >= P0 && oj < P1) out[oj] = (uint16_t)(wv[j >> 1] >> (16 * (j & 1)));
+    if (table_ok && c < M.n_chunks) {
+      const uint2 ab = lds64(st + 8 * t);
+      const uint32_t C = bswap32(lds32(st + 8 * t + 8));
+      const uint32_t A = bswap32(ab.x), B = bswap32(ab.y);
+      const uint32_t lim = c + 1 < M.n_chunks ? 64u : M.tail_bits;
+      const uint32_t q = 5u * t;
+      const uint32_t ga = st + kStreamStage + (q >> 3);
+      const uint32_t two = (lds8(ga) << 8) | lds8(ga + 1);
+      const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
+      uint32_t p = gap, d = 0, e = 0;
+      // codes starting in the chunk's first word, then in its second (each
+      // loop's window needs no select).  With codes longer than the table's
+      // reach, a flagged entry leaves the loops, the code is decoded by the
+      // length search, and the loops resume after it
+      const uint32_t lim1 = min(lim, 32u);
+      if (table_short) {
+#pragma unroll 1
+        while (p < lim1) {
+          const uint32_t w = __funnelshift_l(B, A, p);
+          DF11_FAST_STEP_NOFLAG(w)
+        }
+#pragma unroll 1
+        while (p < lim) {
+          const uint32_t w = __funnelshift_l(C, B, p);  // the shift is p - 32
+          DF11_FAST_STEP_NOFLAG(w)
+        }
+      } else {
+#pragma unroll 1
+        for (;;) {
+#pragma unroll 1
+          while (p < lim1) {
+            const uint32_t w = __funnelshift_l(B, A, p);
+            DF11_FAST_STEP(w)
           }
+          if (p >= lim1) {
+#pragma unroll 1
+            while (p < lim) {
+              const uint32_t w = __funnelshift_l(C, B, p);  // the shift is p - 32
+              DF11_FAST_STEP(w)
+            }
+            if (p >= lim) break;
+          }
+          const uint32_t w = window32(A, B, C, p);
+          const uint32_t L = long_code_len(w, tab);
+          if (L == 0) {
+            bad = true;
+            break;
+          }
+          sts8(priv_a + d, tab.sym[((w >> (32 - L)) + tab.base[L]) & 0xFFu]);
+          d += 1;
+          p += L;
+          e = 1u << 24;  // one code: nothing to trim below
         }
       }
+      if (d && p > lim) {
+        // the last entry ran past the chunk's end: keep its codes that start
+        // before lim, clear the others
+        const uint32_t ns = (e >> 24) & 0x3u;
+        const uint32_t q1 = p - (e >> 28) + lds8(codelen_a + (e & 0xFFu));
+        const uint32_t q2 = q1 + lds8(codelen_a + ((e >> 8) & 0xFFu));
+        const bool drop2 = ns >= 2 && q1 >= lim;
+        const bool drop3 = ns == 3 && q2 >= lim;
+        sts8_if(priv_a + d - ns + 1, 0u, drop2);
+        sts8_if(priv_a + d - 1, 0u, drop3);
+        d -= (uint32_t)drop2 + (uint32_t)drop3;
+      }
+      cnt = d;
     }
+    // ---- the previous block's merge (between decode and the count barrier);
+    // its sign/mantissa phase is waited for even if the block was rejected,
+    // so that the barrier is never re-armed with a copy in flight
+    if (it) {
+      if (!mbar_wait(bar_sm, (uint32_t)((it - 1) & 1))) timed_out = true;
+      else if (prev.ok) merge_block(prev, lin_a, sm_a, t);
+    }
+    // ---- [B] CTA prefix sum of the counts
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int dd = 1; dd < 32; dd <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, dd);
+      if (lane >= dd) incl += o;
+    }
+    const uint32_t wflags = __ballot_sync(0xffffffffu, bad) ? 0x80000000u : 0u;
+    const uint32_t wtime = __ballot_sync(0xffffffffu, timed_out) ? 0x40000000u : 0u;
+    if (lane == 31) warp_tot[warp] = incl | wflags | wtime;
+    __syncthreads();
+    uint32_t wpre = 0, tot = 0, flagbits = 0;
+    {
+      const uint4 lo4 = reinterpret_cast<const uint4 *>(warp_tot)[0];
+      const uint4 hi4 = reinterpret_cast<const uint4 *>(warp_tot)[1];
+      const uint32_t x[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
+#pragma unroll
+      for (int i = 0; i < kT / 32; ++i) {
+        flagbits |= x[i];
+        const uint32_t v = x[i] & 0x3FFFFFFFu;
+        tot += v;
+        wpre += i < warp ? v : 0u;
+      }
+    }
+    if (flagbits & 0x40000000u) {
+      // a bounded wait ran out: leave (uniformly) with the status set, after
+      // a bounded wait for the next block's copy issued at the top
+      if (t == 0) {
+        set_status(P.status, DF11_ERR_TIMEOUT);
+        if (g + 1 < g1) mbar_wait(bar_stage + 8 * (s ^ 1), (uint32_t)(((it + 1) >> 1) & 1));
+      }
+      return;
+    }
+    const bool ok = table_ok && sane && !(flagbits >> 31) && tot == P1 - P0;
+    if (t == 0) {
+      if (!ok) set_status(P.status, DF11_ERR_CORRUPT);
+      // this block's sign/mantissa bytes (the previous block's merge is done),
+      // rounded out to 16 B
+      const uint32_t sm_lo = P0 & ~15u;
+      const uint32_t sm_bytes = sane ? (uint32_t)((((uint64_t)P1 + 15u) & ~15ull) - sm_lo) : 0u;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(bar_sm, sm_bytes);
+      if (sm_bytes) bulk_g2s(sm_a, M.sm + sm_lo, sm_bytes, bar_sm);
+    }
+    // ---- move this thread's exponents to its place in the linear row:
+    // 32-bit words realigned with funnel shifts and OR-ed in (the edge words
+    // are shared with the neighbouring threads); the region is cleared
+    // behind the reads
+    if (cnt) {
+      if (ok) {
+        const uint32_t D = (P0 & 7u) + wpre + incl - cnt;
+        const uint32_t sh = (D & 3u) * 8;
+        const uint32_t la = lin_a + (D & ~3u);
+        uint32_t prevw = 0;
+        // words past the thread's last target word OR in zeros (the bytes
+        // beyond its codes are zero) and stay inside the row's slack
+#pragma unroll
+        for (int j = 0; j <= MAXW; ++j) {
+          const uint32_t cur = j < MAXW ? lds32(priv_a + 4 * j) : 0u;
+          if (j < MAXW) sts32(priv_a + 4 * j, 0u);
+          red_or32(la + 4 * j, __funnelshift_l(prevw, cur, sh));
+          prevw = cur;
+        }
+      } else {
+        // a rejected block still leaves the private region cleared
+#pragma unroll
+        for (int k = 0; k < MAXW; ++k) sts32(priv_a + 4 * k, 0u);
+      }
+    }
+    prev = Pending{P0, P1, M.out, ok};
+  }
+  // the last block's merge
+  __syncthreads();
+  if (!mbar_wait(bar_sm, (uint32_t)((g1 - g0 - 1) & 1))) {
+    if (lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
+  } else if (prev.ok) {
+    merge_block(prev, lin_a, sm_a, t);
   }
 }
 
+#undef DF11_FAST_STEP
+
 // ============================================================ launch helpers
+
+// decode_kernel instantiations: regions of codes >= 2 bits and >= 1 bit
+constexpr int kMaxWords2 = 9;   // region_bytes_for(2) / 4
+constexpr int kMaxWords1 = 17;  // region_bytes_for(1) / 4
+static_assert(region_bytes_for(2) == 4 * kMaxWords2 && region_bytes_for(1) == 4 * kMaxWords1,
+              "private region sizes");
 
 struct DeviceInfo {
   int sms = 0;
@@ -744,8 +927,11 @@ df11_status device_info(int *dev, int *sms) {
     if (cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kHistSmem) != cudaSuccess)
       return DF11_ERR_CUDA;
-    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_layout(16384 + 16).total) != cudaSuccess)
+    const int max_smem = (int)smem_layout(16384, region_bytes_for(1)).total;
+    if (cudaFuncSetAttribute(decode_kernel<kMaxWords2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_kernel<kMaxWords1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess)
       return DF11_ERR_CUDA;
     d.configured = true;
   }
@@ -853,11 +1039,13 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
       if (!aligned16(m.stream) || !aligned16(m.gaps) || !aligned16(m.sign_mantissa) ||
           !aligned16(m.tables) || !aligned16(d_outs[first + i]) || ((uintptr_t)m.block_pos & 3u))
         return DF11_ERR_INVALID_ARG;
-      if (m.min_len < 1 || m.min_len > DF11_MAX_CODE_LEN) return DF11_ERR_INVALID_ARG;
+      // a complete code over at most 256 values has a code of at most 8 bits
+      if (m.min_len < 1 || m.min_len > 8) return DF11_ERR_INVALID_ARG;
       if (m.total_bits < m.n * (uint64_t)m.min_len || m.total_bits > m.n * 32ull)
         return DF11_ERR_INVALID_ARG;
       const uint64_t C = cdiv(m.total_bits, 64);
       const uint64_t B = cdiv(C, kT);
+      if (C >= (1ull << 31)) return DF11_ERR_TOO_LARGE;
       DecMat &d = P.m[P.count];
       d.stream = m.stream;
       d.gaps = m.gaps;
@@ -866,8 +1054,8 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
       d.tables = reinterpret_cast<const DecodeTables *>(m.tables);
       d.out = d_outs[first + i];
       d.n = m.n;
-      d.total_bits = m.total_bits;
-      d.n_chunks = C;
+      d.n_chunks = (uint32_t)C;
+      d.tail_bits = (uint32_t)(m.total_bits - 64 * (C - 1));
       P.block_start[P.count + 1] = P.block_start[P.count] + B;
       min_len = std::min(min_len, m.min_len);
       ++P.count;
@@ -877,14 +1065,17 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
     // at most ceil(64/min_len) codes start in a chunk
     const uint32_t per_block = (uint32_t)cdiv(64, min_len) * kT;
     P.stage_cap = (per_block + 15u) & ~15u;
-    const uint32_t smem = smem_layout(P.stage_cap).total;
+    P.region_bytes = 4u * (min_len >= 2 ? kMaxWords2 : kMaxWords1);
+    P.min_len = min_len;
+    const uint32_t smem = smem_layout(P.stage_cap, P.region_bytes).total;
+    auto kern = min_len >= 2 ? decode_kernel<kMaxWords2> : decode_kernel<kMaxWords1>;
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel, kT, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kT, smem) != cudaSuccess)
       return DF11_ERR_CUDA;
     if (occ < 1) return DF11_ERR_CUDA;
     const uint64_t blocks = P.block_start[P.count];
     const uint64_t grid = std::min<uint64_t>(blocks, (uint64_t)sms * occ);
-    decode_kernel<<<(unsigned)grid, kT, smem, s>>>(P);
+    kern<<<(unsigned)grid, kT, smem, s>>>(P);
     st = launch_status();
     if (st != DF11_OK) return st;
   }

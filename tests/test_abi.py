@@ -181,10 +181,11 @@ def test_decode_table_against_oracle_codes(lib, which):
         syms, used = greedy_window(codes_by_str, format(v, "012b"))
         e = int(lut[v])
         if not syms:
-            assert e == 0, (v, hex(e))
+            assert e == (12 << 28) | (1 << 26), (v, hex(e))  # long-code flag, 12 bits skipped
             continue
-        assert e & 0xF == used and (e >> 4) & 3 == len(syms)
-        assert [(e >> (8 + 8 * i)) & 0xFF for i in range(len(syms))] == syms
+        assert e >> 28 == used and (e >> 24) & 3 == len(syms) and not e & (1 << 26)
+        assert [(e >> (8 * i)) & 0xFF for i in range(len(syms))] == syms
+        assert e & 0xFFFFFF == sum(s << (8 * i) for i, s in enumerate(syms))
 
 
 def test_validate_accepts_oracle_metadata_and_rejects_corruption(lib):

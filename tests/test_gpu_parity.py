@@ -5,7 +5,12 @@ five workloads at full size, in the launch configuration bench.py times.
 
 Expected values come from the oracle only.  Where the expected decode output
 is the input itself, that is the oracle's own result: its round trip is the
-identity (pinned in test_oracle_pins.py) and small cases call it explicitly."""
+identity (pinned in test_oracle_pins.py) and small cases call it explicitly.
+
+Every case runs under two code-length caps: 12 (the codec default, the decode
+table's reach: the fast path) and 32 (the format's limit: codes longer than
+the table take the length search).  The oracle builds its codebook with the
+same cap."""
 import numpy as np
 import pytest
 import torch
@@ -42,13 +47,16 @@ def assert_encoded_equal(m, enc):
     assert np.array_equal(h["sign_mantissa"], enc.sign_mantissa), "sign/mantissa differ"
 
 
-def full_check(codec, x: np.ndarray, call_oracle_decode: bool = True):
+CAPS = [12, 32]
+
+
+def full_check(codec, x: np.ndarray, cap: int, call_oracle_decode: bool = True):
     x = np.ascontiguousarray(x, np.uint16).reshape(-1)
-    enc = oracle.encode(x)
+    enc = oracle.encode(x, cap=cap)
     w = to_dev(x)
     hist = codec.histogram(w).cpu().numpy().view(np.uint64)
     assert np.array_equal(hist, enc.hist), "histogram differs"
-    m = codec.compress(w)
+    m = codec.compress(w, cap=cap)
     assert_encoded_equal(m, enc)
     expected = oracle.decode(enc, chunked=True) if call_oracle_decode else x
     out = codec.decompress(m)
@@ -62,37 +70,43 @@ def full_check(codec, x: np.ndarray, call_oracle_decode: bool = True):
     return m, enc
 
 
+@pytest.mark.parametrize("cap", CAPS)
 @pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 15, 16, 17, 4097, 65_537, 1_000_003])
-def test_sizes_and_ragged_tails(codec, n):
-    full_check(codec, workloads.random_bf16(n, seed=1000 + n))
+def test_sizes_and_ragged_tails(codec, n, cap):
+    full_check(codec, workloads.random_bf16(n, seed=1000 + n), cap)
 
 
-def test_every_bit_pattern(codec):
-    m, enc = full_check(codec, workloads.all_patterns())
+@pytest.mark.parametrize("cap", CAPS)
+def test_every_bit_pattern(codec, cap):
+    m, enc = full_check(codec, workloads.all_patterns(), cap)
     assert np.array_equal(m.host_arrays()["stream"], oracle.split(workloads.all_patterns())[0])
 
 
-def test_every_bit_pattern_shuffled(codec):
-    full_check(codec, workloads.shuffled_patterns(4))
+@pytest.mark.parametrize("cap", CAPS)
+def test_every_bit_pattern_shuffled(codec, cap):
+    full_check(codec, workloads.shuffled_patterns(4), cap)
 
 
+@pytest.mark.parametrize("cap", CAPS)
 @pytest.mark.parametrize("n", [1, 64, 65, 16_384, 16_385, 1_000_000])
-def test_single_symbol(codec, n):
-    full_check(codec, workloads.constant(n, 0xBC00))
+def test_single_symbol(codec, n, cap):
+    full_check(codec, workloads.constant(n, 0xBC00), cap)
 
 
-def test_two_symbols_and_all_equal_words(codec):
+@pytest.mark.parametrize("cap", CAPS)
+def test_two_symbols_and_all_equal_words(codec, cap):
     g = np.random.default_rng(3)
     x = np.where(g.random(300_000) < 0.7, 0x3F80, 0xC000).astype(np.uint16)
-    full_check(codec, x)
-    full_check(codec, workloads.constant(123_457, 0x0000))
+    full_check(codec, x, cap)
+    full_check(codec, workloads.constant(123_457, 0x0000), cap)
 
 
-def test_worked_example(codec):
+@pytest.mark.parametrize("cap", CAPS)
+def test_worked_example(codec, cap):
     import json, os
     gd = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_tiny.json")))
     x = np.array([int(v, 16) for v in gd["weights_hex"]], np.uint16)
-    m, _ = full_check(codec, x)
+    m, _ = full_check(codec, x, cap)
     h = m.host_arrays()
     assert h["gaps"].tolist() == gd["gaps_packed"] and h["block_pos"].tolist() == gd["block_pos"]
 
@@ -101,27 +115,35 @@ def test_fibonacci_length_cap(codec):
     """14,930,351 values whose exponent counts are Fibonacci numbers: the code
     needs the 32-bit cap, so 20 of the codes are longer than the 12-bit
     decode table and take the length-search path."""
-    m, enc = full_check(codec, workloads.fibonacci_exponents(34), call_oracle_decode=False)
+    m, enc = full_check(codec, workloads.fibonacci_exponents(34), 32, call_oracle_decode=False)
     assert int(enc.lengths.max()) == 32
 
 
+def test_fibonacci_at_table_cap(codec):
+    """The same input under the 12-bit cap: package-merge shortens every code
+    to the table's reach."""
+    m, enc = full_check(codec, workloads.fibonacci_exponents(34), 12, call_oracle_decode=False)
+    assert int(enc.lengths.max()) == 12
+
+
+@pytest.mark.parametrize("cap", CAPS)
 @pytest.mark.parametrize("wid", [1, 2, 4])
-def test_workload_single_matrix(codec, wid):
+def test_workload_single_matrix(codec, wid, cap):
     x = workloads.matrix(wid, 0)
-    m, enc = full_check(codec, x, call_oracle_decode=(wid == 1))
+    m, enc = full_check(codec, x, cap, call_oracle_decode=(wid == 1))
     assert m.stored_bytes == oracle.stored_bytes(enc)
 
 
-@pytest.mark.parametrize("wid", [3, 5])
-def test_workload_block_batched(codec, wid):
+@pytest.mark.parametrize("wid,cap", [(3, 12), (3, 32), (5, 12), (5, 32)])
+def test_workload_block_batched(codec, wid, cap):
     """A whole transformer block: per-matrix codebooks, one decode launch
-    (the bench configuration)."""
+    (the bench configuration, cap 12; and cap 32)."""
     names = [nm for nm, _ in workloads.WORKLOADS[wid][1]]
     mats, xs = [], []
     for i, _ in enumerate(names):
         x = workloads.matrix(wid, i).reshape(-1)
-        enc = oracle.encode(x)
-        m = codec.compress(to_dev(x))
+        enc = oracle.encode(x, cap=cap)
+        m = codec.compress(to_dev(x), cap=cap)
         assert_encoded_equal(m, enc)
         mats.append(m)
         xs.append(x)
@@ -131,9 +153,10 @@ def test_workload_block_batched(codec, wid):
         assert np.array_equal(bits_of(o), x)
 
 
-def test_decode_reports_corrupt_positions_without_fault(codec):
+@pytest.mark.parametrize("cap", CAPS)
+def test_decode_reports_corrupt_positions_without_fault(codec, cap):
     x = workloads.random_bf16(2_000_000, seed=9)
-    m = codec.compress(to_dev(x))
+    m = codec.compress(to_dev(x), cap=cap)
     pos = m.block_pos.clone()
     m.block_pos[3] += 5
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
