@@ -187,6 +187,29 @@ df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_codebook *cb
                         size_t workspace_bytes, uint32_t *d_status, df11_stream_t stream);
 
 /*
+ * df11_encode_static_ws -- df11_encode for callers that cannot allocate
+ * device memory where they call the codec: for instance code running inside
+ * another framework's execution callback without access to its allocator,
+ * or a process that reserved all device memory up front.  The page has no
+ * counterpart to this entry point; it exists for such callers only.
+ * Arguments and results are those of df11_encode, without the workspace: the
+ * scratch (per-tile bit offsets) lives in a fixed array in the library's own
+ * device memory, which every GPU that loads the library holds (512 KiB) until
+ * the process exits.  Nothing is allocated.
+ *   n <= DF11_STATIC_WS_MAX_N, else DF11_ERR_TOO_LARGE (nothing launched).
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array: calls whose work overlaps on the GPU (other
+ * streams, other host threads) race on it and must be serialised by the
+ * caller.  Each call rewrites every entry it reads, so nothing needs clearing
+ * between calls.
+ */
+#define DF11_STATIC_WS_MAX_N 268431360ull /* 65535 tiles of 4096 values */
+df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n, const df11_codebook *cb,
+                                  uint64_t total_bits, const df11_encoded *out,
+                                  uint32_t *d_status, df11_stream_t stream);
+
+/*
  * df11_decode -- decompress one matrix into BF16.  [GPU], [Kernel].
  *   m      host struct describing device buffers.
  *   d_out  n uint16 BF16 words, 16-byte aligned; written in full.

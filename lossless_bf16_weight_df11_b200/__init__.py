@@ -96,6 +96,8 @@ def _declare(lib):
         "df11_decode_block_batch": (ctypes.c_int, [ctypes.POINTER(df11_matrix), _u32,
                                                    ctypes.POINTER(ctypes.c_void_p), _vp, _vp]),
         "df11_validate": (ctypes.c_int, [_u64, _u64, _u32, _vp, _u64, _vp, _u64]),
+        "df11_encode_static_ws": (ctypes.c_int, [_vp, _u64, ctypes.POINTER(df11_codebook), _u64,
+                                                 ctypes.POINTER(df11_encoded), _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -186,3 +188,14 @@ def df11_validate(n: int, total_bits: int, min_len: int, h_gaps: int, gaps_bytes
                   h_block_pos: int, block_pos_count: int) -> int:
     return load().df11_validate(n, total_bits, min_len, h_gaps, gaps_bytes, h_block_pos,
                                 block_pos_count)
+
+
+STATIC_WS_MAX_N = 268431360  # DF11_STATIC_WS_MAX_N
+
+
+def df11_encode_static_ws(d_w: int, n: int, cb: df11_codebook, total_bits: int, out: df11_encoded,
+                          d_status: int, stream: int = 0) -> int:
+    """df11_encode without a caller-provided workspace, for callers that cannot
+    allocate device memory at the call site; see include/df11.h."""
+    return load().df11_encode_static_ws(d_w, n, ctypes.byref(cb), total_bits, ctypes.byref(out),
+                                        d_status, stream)

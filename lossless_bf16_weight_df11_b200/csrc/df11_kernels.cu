@@ -1087,3 +1087,93 @@ extern "C" df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32
   if (!m) return DF11_ERR_INVALID_ARG;
   return df11_decode_block_batch(m, 1, &d_out, d_status, stream);
 }
+
+// ============================================================ encode without allocation
+//
+// df11_encode needs a scratch buffer from its caller (the per-tile bit
+// offsets).  Some callers cannot hand one over: code running inside another
+// framework's execution callback with no access to that framework's device
+// allocator, or a process that has reserved all device memory up front and
+// may not allocate afterwards.  For them this variant keeps its scratch in a
+// fixed array in the library's own device memory, so a call allocates
+// nothing.  Its cost: every GPU that loads the library holds the array
+// (kStaticTiles * 8 bytes, 512 KiB) until the process exits, and matrices are
+// limited to DF11_STATIC_WS_MAX_N values.
+
+namespace {
+
+constexpr uint64_t kStaticTiles = 1ull << 16;  // tile offsets the array holds (incl. the total)
+static_assert((kStaticTiles - 1) * df11i::kEncTile == DF11_STATIC_WS_MAX_N,
+              "header limit and array size agree");
+
+// The scratch itself.  Host code must not pass this name to a kernel (on the
+// host it names a stand-in, not device memory); it uses the device address
+// obtained with cudaGetSymbolAddress below.
+static __device__ __align__(256) uint64_t g_static_tile_offsets[kStaticTiles];
+
+std::mutex g_static_mu;
+uint64_t *g_static_ptr[64] = {nullptr};
+
+// Device address of the array on the current device, looked up once per device.
+df11_status static_scratch(int dev, uint64_t **ptr) {
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_tile_offsets) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return DF11_ERR_CUDA;
+    }
+    g_static_ptr[dev] = reinterpret_cast<uint64_t *>(p);
+  }
+  *ptr = g_static_ptr[dev];
+  return DF11_OK;
+}
+
+}  // namespace
+
+extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
+                                             const df11_codebook *cb, uint64_t total_bits,
+                                             const df11_encoded *out, uint32_t *d_status,
+                                             df11_stream_t stream) {
+  if (!cb || !out || !d_status) return DF11_ERR_INVALID_ARG;
+  if (n > DF11_STATIC_WS_MAX_N) return DF11_ERR_TOO_LARGE;
+  if ((n && (!d_w || !aligned16(d_w))) || !out->stream || !out->gaps || !out->block_pos ||
+      !out->sign_mantissa)
+    return DF11_ERR_INVALID_ARG;
+  if (!aligned16(out->stream) || !aligned16(out->gaps) || !aligned16(out->block_pos) ||
+      !aligned16(out->sign_mantissa))
+    return DF11_ERR_INVALID_ARG;
+  if (total_bits > n * (uint64_t)DF11_MAX_CODE_LEN || (n && total_bits < n))
+    return DF11_ERR_INVALID_ARG;
+  const uint64_t n_tiles = cdiv(n, df11i::kEncTile);
+  if (n_tiles + 1 > kStaticTiles) return DF11_ERR_TOO_LARGE;
+  int dev, sms;
+  df11_status st = device_info(&dev, &sms);
+  if (st != DF11_OK) return st;
+  uint64_t *ws = nullptr;
+  st = static_scratch(dev, &ws);
+  if (st != DF11_OK) return st;
+  EncCodebook ecb;
+  for (int i = 0; i < 256; ++i) {
+    ecb.code[i] = cb->code[i];
+    ecb.len[i] = cb->len[i];
+  }
+  const uint64_t C = cdiv(total_bits, 64);
+  const uint64_t B = cdiv(C, kT);
+  const uint64_t stream_alloc = 8 * kT * B + 16;
+  const uint64_t gaps_alloc = kGapStage * B + 16;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // nothing in the array needs clearing: every tile offset a call reads is
+  // written earlier in the same call
+  const uint64_t grid1 = std::max<uint64_t>(n_tiles, 1);
+  enc_sum_kernel<<<(unsigned)grid1, df11i::kEncThreads, 0, s>>>(
+      d_w, n, ecb, ws, n_tiles, reinterpret_cast<uint4 *>(out->stream), stream_alloc / 16,
+      reinterpret_cast<uint4 *>(out->gaps), gaps_alloc / 16, d_status);
+  enc_scan_kernel<<<1, kScanThreads, 0, s>>>(ws, n_tiles, total_bits, out->block_pos, B, n,
+                                            d_status);
+  if (n_tiles)
+    enc_pack_kernel<<<(unsigned)n_tiles, df11i::kEncThreads, 0, s>>>(
+        d_w, n, ecb, ws, total_bits, out->stream, stream_alloc, out->gaps, gaps_alloc,
+        out->block_pos, B, out->sign_mantissa);
+  return launch_status();
+}
