@@ -111,7 +111,11 @@ typedef struct {
   const uint8_t *sign_mantissa;/* PackedSignMantissa ([Format])                 */
   const void *tables;          /* device copy of df11_build_tables output       */
   uint32_t min_len;            /* shortest code length (codebook.min_len)       */
-  uint32_t reserved;
+  uint32_t max_block_codes;    /* most codes starting in one block of 256
+                                  chunks (df11_encoded.block_max), or 0 to
+                                  assume the most that min_len allows; sizes
+                                  the decoder's staging (a block exceeding it
+                                  is reported as corrupt)                       */
 } df11_matrix;
 
 /* Encoder outputs in device memory (sizes from df11_encoded_sizes). */
@@ -120,6 +124,8 @@ typedef struct {
   uint8_t *gaps;
   uint32_t *block_pos;
   uint8_t *sign_mantissa;
+  uint32_t *block_max;         /* optional device word (may be NULL): receives
+                                  the most codes starting in any one block     */
 } df11_encoded;
 
 /* Human-readable name of a status code (static string). */

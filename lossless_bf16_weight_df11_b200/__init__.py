@@ -58,12 +58,13 @@ class df11_matrix(ctypes.Structure):
                 ("stream", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
                 ("block_pos", ctypes.c_void_p), ("sign_mantissa", ctypes.c_void_p),
                 ("tables", ctypes.c_void_p), ("min_len", ctypes.c_uint32),
-                ("reserved", ctypes.c_uint32)]
+                ("max_block_codes", ctypes.c_uint32)]
 
 
 class df11_encoded(ctypes.Structure):
     _fields_ = [("stream", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
-                ("block_pos", ctypes.c_void_p), ("sign_mantissa", ctypes.c_void_p)]
+                ("block_pos", ctypes.c_void_p), ("sign_mantissa", ctypes.c_void_p),
+                ("block_max", ctypes.c_void_p)]
 
 
 class DF11Error(RuntimeError):

@@ -52,13 +52,14 @@ class DF11Matrix:
     sign_mantissa: torch.Tensor  # uint8, sizes.sign_mantissa_alloc
     tables: torch.Tensor         # uint8, df11_tables_bytes()
     hist: np.ndarray = field(repr=False, default=None)
+    max_block_codes: int = 0     # most codes in one block (0 = unknown)
 
     def abi(self) -> df11_matrix:
         return df11_matrix(n=self.n, total_bits=self.total_bits, stream=self.stream.data_ptr(),
                            gaps=self.gaps.data_ptr(), block_pos=self.block_pos.data_ptr(),
                            sign_mantissa=self.sign_mantissa.data_ptr(),
                            tables=self.tables.data_ptr(), min_len=max(1, self.codebook.min_len),
-                           reserved=0)
+                           max_block_codes=self.max_block_codes)
 
     @property
     def stored_bytes(self) -> int:
@@ -138,19 +139,20 @@ def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | 
     bufs = alloc_encoded(sizes, dev)
     tables = build_tables(codebook, dev)
     ws = torch.empty(max(16, sizes.workspace_bytes), dtype=torch.uint8, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    status = torch.zeros(2, dtype=torch.int32, device=dev)  # [status, most codes per block]
     out = df11_encoded(stream=bufs["stream"].data_ptr(), gaps=bufs["gaps"].data_ptr(),
                        block_pos=bufs["block_pos"].data_ptr(),
-                       sign_mantissa=bufs["sign_mantissa"].data_ptr())
+                       sign_mantissa=bufs["sign_mantissa"].data_ptr(),
+                       block_max=status.data_ptr() + 4)
     with torch.cuda.device(dev):
         check(df11_encode(u.data_ptr(), u.numel(), codebook, sizes.total_bits, out,
                           ws.data_ptr(), ws.numel(), status.data_ptr(), sh), "df11_encode")
-    if check_status:
-        s = int(status.item())
-        if s:
-            raise DF11Error(s, "df11_encode (device)")
+    st_host = status.cpu().numpy()
+    if check_status and int(st_host[0]):
+        raise DF11Error(int(st_host[0]), "df11_encode (device)")
     return DF11Matrix(shape=tuple(w.shape), n=u.numel(), total_bits=int(sizes.total_bits),
-                      codebook=codebook, sizes=sizes, tables=tables, hist=hist, **bufs)
+                      codebook=codebook, sizes=sizes, tables=tables, hist=hist,
+                      max_block_codes=int(st_host[1]), **bufs)
 
 
 def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Tensor | None = None,

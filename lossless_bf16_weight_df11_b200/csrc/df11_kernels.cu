@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_sum_kernel(
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) enc_scan_kernel(
     uint64_t *__restrict__ tile_sum, uint64_t n_tiles, uint64_t total_bits, uint32_t *block_pos,
-    uint64_t n_blocks, uint64_t n, uint32_t *status) {
+    uint64_t n_blocks, uint64_t n, uint32_t *status, uint32_t *block_max) {
   __shared__ uint64_t s_warp[kScanThreads / 32];
   __shared__ uint64_t s_total;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -246,6 +246,7 @@ __global__ void __launch_bounds__(kScanThreads) enc_scan_kernel(
     tile_sum[n_tiles] = carry;
     if (carry != total_bits) set_status(status, DF11_ERR_CORRUPT);
     block_pos[n_blocks] = (uint32_t)n;
+    if (block_max) *block_max = 0u;
   }
 }
 
@@ -377,6 +378,18 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     if (k == 0 || k + 1 == nwords) atomicOr(&stream32[gw], val);
     else stream32[gw] = val;
   }
+}
+
+// Most codes starting in any one block: max over b of pos[b+1] - pos[b].
+__global__ void __launch_bounds__(256) enc_block_max_kernel(const uint32_t *__restrict__ pos,
+                                                            uint64_t n_blocks, uint32_t *out) {
+  uint32_t best = 0;
+  for (uint64_t b = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks;
+       b += (uint64_t)gridDim.x * blockDim.x)
+    best = max(best, pos[b + 1] - pos[b]);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) best = max(best, __shfl_down_sync(0xffffffffu, best, d));
+  if ((threadIdx.x & 31) == 0 && best) atomicMax(out, best);
 }
 
 // ============================================================ decode
@@ -1005,11 +1018,14 @@ extern "C" df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_c
       d_w, n, ecb, ws, n_tiles, reinterpret_cast<uint4 *>(out->stream), stream_alloc / 16,
       reinterpret_cast<uint4 *>(out->gaps), gaps_alloc / 16, d_status);
   enc_scan_kernel<<<1, kScanThreads, 0, s>>>(ws, n_tiles, total_bits, out->block_pos, B, n,
-                                            d_status);
+                                            d_status, out->block_max);
   if (n_tiles)
     enc_pack_kernel<<<(unsigned)n_tiles, df11i::kEncThreads, 0, s>>>(
         d_w, n, ecb, ws, total_bits, out->stream, stream_alloc, out->gaps, gaps_alloc,
         out->block_pos, B, out->sign_mantissa);
+  if (out->block_max && B)
+    enc_block_max_kernel<<<(unsigned)std::min<uint64_t>(cdiv(B, 256), 1024), 256, 0, s>>>(
+        out->block_pos, B, out->block_max);
   return launch_status();
 }
 
@@ -1029,6 +1045,7 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
     P.status = d_status;
     P.block_start[0] = 0;
     uint32_t min_len = DF11_MAX_CODE_LEN;
+    uint32_t block_codes = 0;  // staging size: most codes in one block of the batch
     for (uint32_t i = 0; i < k; ++i) {
       const df11_matrix &m = ms[first + i];
       if (m.n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
@@ -1043,6 +1060,9 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
       if (m.min_len < 1 || m.min_len > 8) return DF11_ERR_INVALID_ARG;
       if (m.total_bits < m.n * (uint64_t)m.min_len || m.total_bits > m.n * 32ull)
         return DF11_ERR_INVALID_ARG;
+      const uint32_t worst = (uint32_t)cdiv(64, m.min_len) * kT;
+      if (m.max_block_codes > worst) return DF11_ERR_INVALID_ARG;
+      block_codes = std::max(block_codes, m.max_block_codes ? m.max_block_codes : worst);
       const uint64_t C = cdiv(m.total_bits, 64);
       const uint64_t B = cdiv(C, kT);
       if (C >= (1ull << 31)) return DF11_ERR_TOO_LARGE;
@@ -1062,9 +1082,7 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
     }
     if (P.count == 0) continue;
     for (uint32_t i = P.count + 1; i <= DF11_MAX_BATCH; ++i) P.block_start[i] = P.block_start[P.count];
-    // at most ceil(64/min_len) codes start in a chunk
-    const uint32_t per_block = (uint32_t)cdiv(64, min_len) * kT;
-    P.stage_cap = (per_block + 15u) & ~15u;
+    P.stage_cap = (block_codes + 15u) & ~15u;
     P.region_bytes = 4u * (min_len >= 2 ? kMaxWords2 : kMaxWords1);
     P.min_len = min_len;
     const uint32_t smem = smem_layout(P.stage_cap, P.region_bytes).total;
@@ -1170,10 +1188,13 @@ extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
       d_w, n, ecb, ws, n_tiles, reinterpret_cast<uint4 *>(out->stream), stream_alloc / 16,
       reinterpret_cast<uint4 *>(out->gaps), gaps_alloc / 16, d_status);
   enc_scan_kernel<<<1, kScanThreads, 0, s>>>(ws, n_tiles, total_bits, out->block_pos, B, n,
-                                            d_status);
+                                            d_status, out->block_max);
   if (n_tiles)
     enc_pack_kernel<<<(unsigned)n_tiles, df11i::kEncThreads, 0, s>>>(
         d_w, n, ecb, ws, total_bits, out->stream, stream_alloc, out->gaps, gaps_alloc,
         out->block_pos, B, out->sign_mantissa);
+  if (out->block_max && B)
+    enc_block_max_kernel<<<(unsigned)std::min<uint64_t>(cdiv(B, 256), 1024), 256, 0, s>>>(
+        out->block_pos, B, out->block_max);
   return launch_status();
 }
