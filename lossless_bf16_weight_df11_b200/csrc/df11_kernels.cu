@@ -39,7 +39,7 @@ using df11i::DecodeTables;
 
 namespace {
 
-constexpr int kT = DF11_BLOCK_CHUNKS;  // chunks per block = threads per decode CTA
+constexpr int kT = 256;  // threads per decode CTA
 constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls
 
 __device__ __forceinline__ void set_status(uint32_t *st, uint32_t code) {
@@ -54,7 +54,9 @@ __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 
 constexpr int kHistWarps = 4;
 constexpr int kHistThreads = kHistWarps * 32;
 constexpr size_t kHistSmem = (size_t)kHistWarps * 128 * 32 * 4;  // 64 KiB
-constexpr uint32_t kHistFlushEvery = 8000;  // < 65535 / 8 increments per lane
+constexpr int kHistUnroll = 8;              // 16-byte vectors per lane per step
+constexpr uint32_t kHistFlushEvery = 8000;  // vectors per lane: < 65535 / 8 increments
+static_assert(kHistFlushEvery % kHistUnroll == 0, "flush exactly at the limit");
 
 __global__ void hist_clear_kernel(unsigned long long *hist) { hist[threadIdx.x] = 0ull; }
 
@@ -93,26 +95,37 @@ __global__ void __launch_bounds__(kHistThreads) hist_kernel(const uint16_t *__re
     mine[(e0 >> 1) * 32] += 1u << ((e0 & 1u) * 16);
     mine[(e1 >> 1) * 32] += 1u << ((e1 & 1u) * 16);
   };
-  uint32_t since = 0;
-  // warp-uniform loop: each step a warp reads 4 x 32 consecutive 16-byte vectors
-  for (uint64_t base = gwarp * 128; base < nvec; base += warps_total * 128) {
-    uint4 q[4];
+  // warp-uniform loop: each step a warp reads kHistUnroll x 32 consecutive
+  // 16-byte vectors; the next step's vectors are requested before this
+  // step's counting (its chain of shared-memory read-modify-writes) starts
+  const uint64_t step = warps_total * (kHistUnroll * 32);
+  uint64_t base = gwarp * (kHistUnroll * 32);
+  uint4 q[kHistUnroll];
+  auto load = [&](uint64_t b) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      uint64_t i = base + u * 32 + lane;
+    for (int u = 0; u < kHistUnroll; ++u) {
+      const uint64_t i = b + u * 32 + lane;
       q[u] = i < nvec ? __ldg(wv + i) : make_uint4(0, 0, 0, 0);
     }
+  };
+  if (base < nvec) load(base);
+  uint32_t since = 0;
+  for (; base < nvec; base += step) {
+    uint4 cur[kHistUnroll];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      uint64_t i = base + u * 32 + lane;
+    for (int u = 0; u < kHistUnroll; ++u) cur[u] = q[u];
+    if (base + step < nvec) load(base + step);
+#pragma unroll
+    for (int u = 0; u < kHistUnroll; ++u) {
+      const uint64_t i = base + u * 32 + lane;
       if (i < nvec) {
-        add2(q[u].x);
-        add2(q[u].y);
-        add2(q[u].z);
-        add2(q[u].w);
+        add2(cur[u].x);
+        add2(cur[u].y);
+        add2(cur[u].z);
+        add2(cur[u].w);
       }
     }
-    since += 4;
+    since += kHistUnroll;
     if (since >= kHistFlushEvery) {
       hist_flush(warp_base, lane, hist);
       for (int j = 0; j < 128; ++j) mine[j * 32] = 0u;
@@ -250,13 +263,25 @@ __global__ void __launch_bounds__(kScanThreads) enc_scan_kernel(
   }
 }
 
-// Pack the codes of one tile.  Codes are OR-ed into a shared big-endian bit
-// buffer covering the tile's bit range, then written out as 32-bit words
-// (byte-swapped to the MSB-first byte order); the two edge words are shared
-// with the neighbouring tiles and are OR-ed atomically into the cleared
-// stream.  The thread that owns the first code starting in a chunk writes
-// that chunk's 5-bit gap; the one that owns the first code starting in a
-// block of 256 chunks writes the block's output position.
+// Pack the codes of one tile.  Each thread appends its 16 codes to a 64-bit
+// register accumulator (most significant bit first) and writes every 32-bit
+// word it completes to a shared bit buffer covering the tile's bit range: a
+// thread's interior words hold its bits alone and are plain stores; its first
+// and last words may hold a neighbouring thread's bits and are OR-ed in.  The
+// buffer is then written out as 32-bit words (byte-swapped to the MSB-first
+// byte order); the two edge words are shared with the neighbouring tiles and
+// are OR-ed atomically into the cleared stream.  The thread that owns the
+// first code starting in a chunk writes that chunk's 5-bit gap; the one that
+// owns the first code starting in a block of 256 chunks writes the block's
+// output position.
+__device__ __forceinline__ void or_gap(uint32_t *gaps32, uint64_t gap_words, uint64_t c, uint32_t g) {
+  const uint64_t q = 5 * c;
+  const uint64_t gw = q >> 5;
+  const uint64_t y = (uint64_t)g << (59 - (uint32_t)(q & 31u));
+  if (gw < gap_words) atomicOr(&gaps32[gw], bswap32((uint32_t)(y >> 32)));
+  if ((uint32_t)y && gw + 1 < gap_words) atomicOr(&gaps32[gw + 1], bswap32((uint32_t)y));
+}
+
 __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     const uint16_t *__restrict__ w, uint64_t n, EncCodebook cb,
     const uint64_t *__restrict__ tile_start, uint64_t total_bits, uint8_t *__restrict__ stream,
@@ -264,12 +289,10 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     uint32_t *__restrict__ block_pos, uint64_t n_blocks, uint8_t *__restrict__ sign_mantissa) {
   constexpr int kWords = df11i::kEncTile * DF11_MAX_CODE_LEN / 32 + 2;
   __shared__ uint32_t s_bits[kWords];
-  __shared__ uint32_t s_code[256];
-  __shared__ uint8_t s_len[256];
+  __shared__ uint2 s_lc[256];  // {length, code}
   __shared__ uint32_t s_warp[df11i::kEncThreads / 32];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  s_code[t] = cb.code[t];
-  s_len[t] = cb.len[t];
+  s_lc[t] = make_uint2(cb.len[t], cb.code[t]);
   const uint64_t tile = blockIdx.x;
   const uint64_t S = tile_start[tile], E = tile_start[tile + 1];
   const uint64_t S0 = S & ~31ull;
@@ -280,13 +303,9 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
   uint16_t v[16];
   const uint64_t i0 = tile * df11i::kEncTile + (uint64_t)t * df11i::kEncPerThread;
   load_tile_values(w, n, i0, v);
-  uint32_t lens[16];
   uint32_t sum = 0;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    lens[k] = (i0 + k < n) ? s_len[(v[k] >> 7) & 0xFFu] : 0u;
-    sum += lens[k];
-  }
+  for (int k = 0; k < 16; ++k) sum += (i0 + k < n) ? s_lc[(v[k] >> 7) & 0xFFu].x : 0u;
   uint32_t incl = sum;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -297,58 +316,57 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
   __syncthreads();
   uint32_t wpre = 0;
   for (int i = 0; i < warp; ++i) wpre += s_warp[i];
-  uint32_t rel = (uint32_t)(S - S0) + wpre + incl - sum;  // bit offset in s_bits
-  uint64_t start = S + wpre + incl - sum;                 // absolute bit offset
+  const uint32_t rel = (uint32_t)(S - S0) + wpre + incl - sum;  // bit offset in s_bits
+  uint64_t start = S + wpre + incl - sum;                       // absolute bit offset
   // length of the value before this thread's first one
   uint32_t prev_len = 0;
-  if (i0 > 0 && i0 < n) prev_len = s_len[(w[i0 - 1] >> 7) & 0xFFu];
+  if (i0 > 0 && i0 < n) prev_len = s_lc[(w[i0 - 1] >> 7) & 0xFFu].x;
   const uint64_t C = (total_bits + 63) >> 6;
   uint32_t *gaps32 = reinterpret_cast<uint32_t *>(gaps);
   const uint64_t gap_words = gaps_alloc >> 2;
+  // accumulator: bit 63 is bit (wi * 32) of the buffer; nb bits are filled
+  uint64_t acc = 0;
+  uint32_t nb = rel & 31u, wi = rel >> 5;
+  bool first_word = true;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     const uint64_t i = i0 + k;
     if (i >= n) break;
-    const uint32_t L = lens[k];
-    if (L == 0) continue;
-    const uint32_t code = s_code[(v[k] >> 7) & 0xFFu];
-    // code bits [rel, rel+L) of the big-endian buffer
-    const uint32_t wi = rel >> 5, off = rel & 31u;
-    const uint64_t placed = ((uint64_t)code << (64 - L)) >> off;
-    if (wi < (uint32_t)kWords) atomicOr(&s_bits[wi], (uint32_t)(placed >> 32));
-    if ((uint32_t)placed && wi + 1 < (uint32_t)kWords) atomicOr(&s_bits[wi + 1], (uint32_t)placed);
-    const uint64_t prev = start - prev_len;
-    if (i == 0 || (prev >> 6) != (start >> 6)) {
-      // first code starting in chunk start/64 -> gap
-      const uint64_t c = start >> 6;
-      const uint32_t g = (uint32_t)(start & 63u);
-      const uint64_t q = 5 * c;
-      const uint64_t gw = q >> 5;
-      const uint64_t y = (uint64_t)g << (59 - (uint32_t)(q & 31u));
-      if (gw < gap_words) atomicOr(&gaps32[gw], bswap32((uint32_t)(y >> 32)));
-      if ((uint32_t)y && gw + 1 < gap_words) atomicOr(&gaps32[gw + 1], bswap32((uint32_t)y));
+    const uint2 lc = s_lc[(v[k] >> 7) & 0xFFu];
+    const uint32_t L = lc.x;
+    // nb < 32 and L <= 32; a value without a code (L = 0, reported by the
+    // length-sum kernel) adds nothing
+    acc |= L ? ((uint64_t)lc.y << (64 - L)) >> nb : 0ull;
+    nb += L;
+    if (nb >= 32) {
+      const uint32_t word = (uint32_t)(acc >> 32);
+      if (wi < (uint32_t)kWords) {
+        if (first_word) atomicOr(&s_bits[wi], word);
+        else s_bits[wi] = word;
+      }
+      first_word = false;
+      ++wi;
+      acc <<= 32;
+      nb -= 32;
     }
-    if (i == 0 || (prev >> 14) != (start >> 14)) {
-      const uint64_t b = start >> 14;
-      if (b < n_blocks) block_pos[b] = (uint32_t)i;
+    // the code starts a new chunk (block) when its offset in that chunk
+    // (block) is below the previous code's length
+    if (i == 0 || (uint32_t)(start & 63u) < prev_len) {
+      or_gap(gaps32, gap_words, start >> 6, (uint32_t)(start & 63u));
+      if (i == 0 || (uint32_t)(start & 16383u) < prev_len) {
+        const uint64_t b = start >> 14;
+        if (b < n_blocks) block_pos[b] = (uint32_t)i;
+      }
     }
     if (i + 1 == n) {
       // the last chunk / block may begin inside the final code
-      if (C > 0 && (start >> 6) < C - 1) {
-        const uint64_t c = C - 1;
-        const uint32_t g = (uint32_t)(total_bits - 64 * c);
-        const uint64_t q = 5 * c;
-        const uint64_t gw = q >> 5;
-        const uint64_t y = (uint64_t)g << (59 - (uint32_t)(q & 31u));
-        if (gw < gap_words) atomicOr(&gaps32[gw], bswap32((uint32_t)(y >> 32)));
-        if ((uint32_t)y && gw + 1 < gap_words) atomicOr(&gaps32[gw + 1], bswap32((uint32_t)y));
-      }
+      if (C > 0 && (start >> 6) < C - 1) or_gap(gaps32, gap_words, C - 1, (uint32_t)(total_bits - 64 * (C - 1)));
       if (n_blocks > 0 && (start >> 14) < n_blocks - 1) block_pos[n_blocks - 1] = (uint32_t)n;
     }
     prev_len = L;
-    rel += L;
     start += L;
   }
+  if (nb && wi < (uint32_t)kWords) atomicOr(&s_bits[wi], (uint32_t)(acc >> 32));
   // sign/mantissa plane ([Format]: kept verbatim, one byte per value)
   if (i0 + 16 <= n) {
     uint32_t pk[4];
@@ -364,8 +382,9 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     }
     *reinterpret_cast<uint4 *>(sign_mantissa + i0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   } else {
-    for (int k = 0; k < 16 && i0 + k < n; ++k)
-      sign_mantissa[i0 + k] = (uint8_t)(((v[k] >> 8) & 0x80u) | (v[k] & 0x7Fu));
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (i0 + k < n) sign_mantissa[i0 + k] = (uint8_t)(((v[k] >> 8) & 0x80u) | (v[k] & 0x7Fu));
   }
   __syncthreads();
   uint32_t *stream32 = reinterpret_cast<uint32_t *>(stream);
@@ -393,6 +412,23 @@ __global__ void __launch_bounds__(256) enc_block_max_kernel(const uint32_t *__re
 }
 
 // ============================================================ decode
+//
+// Work unit: kUnitChunks = 512 consecutive chunks of one matrix (two of the
+// format's 256-chunk blocks; the last unit of a matrix may hold one).  A CTA
+// of 256 threads decodes a unit, each thread two consecutive chunks: it
+// starts at the first chunk's gap and decodes straight on through the second,
+// because the first code starting in the second chunk begins exactly where
+// the last code starting in the first one ends.  The unit's first output is
+// pos[2u] and its outputs end at pos[min(2u + 2, B)].
+
+constexpr int kCPT = 2;                                       // chunks per thread
+constexpr uint32_t kUnitChunks = kT * kCPT;                   // 512
+constexpr uint32_t kUnitBlocks = kUnitChunks / DF11_BLOCK_CHUNKS;  // 2
+constexpr uint32_t kBlockStreamBytes = 8 * DF11_BLOCK_CHUNKS;      // 2048
+constexpr uint32_t kBlockGapBytes = DF11_GAP_BITS * DF11_BLOCK_CHUNKS / 8;  // 160
+static_assert(kUnitBlocks == 2, "a unit is two blocks (its middle position is checked)");
+// warps whose threads decode the unit's first block
+constexpr int kFirstBlockWarps = DF11_BLOCK_CHUNKS / kCPT / 32;  // 4
 
 struct DecMat {
   const uint8_t *stream;
@@ -402,51 +438,68 @@ struct DecMat {
   const DecodeTables *tables;
   uint16_t *out;
   uint64_t n;
-  uint32_t n_chunks;   // C = ceil(total_bits / 64) (< 2^31 for n < 2^32)
-  uint32_t tail_bits;  // code bits in the last chunk, 1..64
+  uint64_t total_bits;
+  uint32_t n_chunks;  // C = ceil(total_bits / 64) (< 2^31 for n < 2^32)
+  uint32_t n_blocks;  // B = ceil(C / 256); pos holds B + 1 entries
 };
 
 struct DecParams {
   DecMat m[DF11_MAX_BATCH];
-  uint64_t block_start[DF11_MAX_BATCH + 1];  // prefix sums of blocks per matrix
+  uint64_t unit_start[DF11_MAX_BATCH + 1];  // prefix sums of units per matrix
   uint32_t count;
-  uint32_t stage_cap;     // bytes: max codes per block, rounded up to 16
+  uint32_t stage_cap;     // bytes: max codes per unit, rounded up to 16
   uint32_t region_bytes;  // private decode region per thread (odd number of words)
   uint32_t min_len;       // shortest code of the batch (regions are sized by it)
   uint32_t *status;
 };
 
-constexpr uint32_t kStreamStage = 8 * kT + 16;         // a block of chunks + the next one
-constexpr uint32_t kGapStage = DF11_GAP_BITS * kT / 8;  // 160 B
+constexpr uint32_t kStreamStage = 8 * kUnitChunks + 16;         // a unit of chunks + the next word
+constexpr uint32_t kGapStage = DF11_GAP_BITS * kUnitChunks / 8;  // 320 B
 constexpr uint32_t kStageBytes = kStreamStage + kGapStage + 16;
+static_assert(kStageBytes % 16 == 0 && sizeof(DecodeTables) % 16 == 0, "stage alignment");
 
 struct SmemLayout {
   uint32_t tables, stage0, stage1, sm, linear, priv, bars, meta, warp, total;
 };
 
+// The linear row holds the unit's exponents from byte P0 % 8 on; the
+// relocation of the thread with the last codes ORs region_bytes + 4 bytes
+// from a 4-byte boundary at most 7 + cap bytes in, so the row carries that
+// much slack.
+// Every section starts on a 16-byte boundary: bulk-copy destinations and
+// 16-byte reads (stages, sign/mantissa row, warp totals), 8-byte reads and
+// writes (linear row), mbarriers (8 bytes).
+__host__ __device__ constexpr uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
+
 __host__ __device__ inline SmemLayout smem_layout(uint32_t cap, uint32_t region_bytes) {
   SmemLayout S;
   S.tables = 0;
-  S.stage0 = (uint32_t)sizeof(DecodeTables);
-  S.stage1 = S.stage0 + kStageBytes;
-  S.sm = S.stage1 + kStageBytes;
-  S.linear = S.sm + cap + 32;
-  S.priv = S.linear + cap + 16 + 64;
-  S.bars = S.priv + kT * region_bytes;
-  S.meta = S.bars + 32;
-  S.warp = S.meta + 2 * 16;
-  S.total = S.warp + 16 * 4;
+  S.stage0 = round16((uint32_t)sizeof(DecodeTables));
+  S.stage1 = round16(S.stage0 + kStageBytes);
+  S.sm = round16(S.stage1 + kStageBytes);
+  S.linear = round16(S.sm + cap + 32);
+  S.priv = round16(S.linear + cap + region_bytes + 32);
+  S.bars = round16(S.priv + kT * region_bytes);
+  S.meta = round16(S.bars + 32);
+  S.warp = round16(S.meta + 2 * 32);
+  S.total = round16(S.warp + 16 * 4);
   return S;
 }
 
-// Per-thread private region: the codes that can start in a chunk
-// (ceil(64/min_len)), two codes of overshoot from the last table entry, and
-// the two spare bytes that entry's unconditional three-byte store may touch;
-// an odd number of 32-bit words so that word j of all 32 lanes of a warp
-// falls in 32 different banks.
+inline bool smem_layout_aligned(const SmemLayout &S) {
+  return ((S.stage0 | S.stage1 | S.sm | S.linear | S.priv | S.bars | S.meta | S.warp) & 15u) == 0;
+}
+
+// Per-thread private region: the codes that can start in a thread's two
+// chunks (ceil(128/min_len)), two codes of overshoot from the last table
+// entry, and the two spare bytes that entry's unconditional three-byte store
+// may touch; an odd number of 32-bit words so that word j of all 32 lanes of
+// a warp falls in 32 different banks.
+__host__ __device__ constexpr uint32_t region_words_even(uint32_t min_len) {
+  return ((64 * kCPT + min_len - 1) / min_len + 4 + 3) / 4;
+}
 __host__ __device__ constexpr uint32_t region_bytes_for(uint32_t min_len) {
-  return 4 * (((64 + min_len - 1) / min_len + 4 + 3) / 4 +
-              ((((64 + min_len - 1) / min_len + 4 + 3) / 4) % 2 == 0 ? 1 : 0));
+  return 4 * (region_words_even(min_len) + (region_words_even(min_len) % 2 == 0 ? 1 : 0));
 }
 
 // ---- shared memory through 32-bit shared-window addresses
@@ -466,6 +519,14 @@ __device__ __forceinline__ uint32_t lds8(uint32_t a) {
 __device__ __forceinline__ uint2 lds64(uint32_t a) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
+               : "memory");
   return v;
 }
 __device__ __forceinline__ void sts8(uint32_t a, uint32_t v) {
@@ -532,13 +593,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
   return false;
 }
 
-// Stream bits [p, p+32) of the chunk words A (bits 0..31), B (32..63) and the
-// next chunk's first word C, p in [0, 63].
-__device__ __forceinline__ uint32_t window32(uint32_t A, uint32_t B, uint32_t C, uint32_t p) {
-  const bool up = p >= 32;
-  return __funnelshift_l(up ? C : B, up ? B : A, p);
-}
-
 // Length of a code longer than the table's reach: the smallest L with
 // window < limit[L] (canonical codes are ordered by length when
 // left-justified); 0 if none (invalid code).
@@ -549,14 +603,17 @@ __device__ __forceinline__ uint32_t long_code_len(uint32_t w32, const DecodeTabl
   return 0;
 }
 
-// One table step of the fast decoder on window w.  A flagged entry (first
-// code longer than the table's reach) leaves the loop before anything is
-// stored; otherwise the entry's three exponent slots are stored at dst+d
+// One table step of the decoder on window w.  A flagged entry (first code
+// longer than the table's reach) sets f and leaves the loop before anything
+// is stored; otherwise the entry's three exponent slots are stored at dst+d
 // (absent slots are zero), d advances by the number of codes and p by the
 // bits they use.
-#define DF11_FAST_STEP(w)                                                   \
+#define DF11_FAST_STEP_FLAG(w, f)                                           \
   e = lds32(lut_a + (mulhi((w), 1u << df11i::kLutBits) << 2));              \
-  if (e & df11i::kLutLongFlag) break;                                       \
+  if (e & df11i::kLutLongFlag) {                                            \
+    f = true;                                                               \
+    break;                                                                  \
+  }                                                                         \
   {                                                                         \
     const uint32_t at = priv_a + d;                                         \
     sts8(at, e);                                                            \
@@ -587,15 +644,15 @@ __device__ __forceinline__ void merge4(uint32_t e4, uint32_t s4, uint32_t &w01, 
   w23 = __byte_perm(lo4, hi4, 0x7362);
 }
 
-struct BlockRef {
-  uint32_t m;
-  uint64_t b;
+struct UnitRef {
+  uint32_t m;  // matrix of the batch
+  uint32_t u;  // unit within the matrix
 };
 
-__device__ __forceinline__ BlockRef locate(const DecParams &P, uint64_t g, uint32_t hint) {
+__device__ __forceinline__ UnitRef locate(const DecParams &P, uint64_t g, uint32_t hint) {
   uint32_t m = hint;
-  while (m + 1 < P.count && g >= P.block_start[m + 1]) ++m;
-  return BlockRef{m, g - P.block_start[m]};
+  while (m + 1 < P.count && g >= P.unit_start[m + 1]) ++m;
+  return UnitRef{m, (uint32_t)(g - P.unit_start[m])};
 }
 
 // A decoded block waiting for its merge: positions, output, staging.
@@ -650,7 +707,7 @@ __device__ __forceinline__ void merge_block(const Pending &q, uint32_t lin_a, ui
 
 // MAXW: 32-bit words of a thread's private region.
 template <int MAXW>
-__global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ DecParams P) {
+__global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ DecParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t cap = P.stage_cap;
   const SmemLayout S = smem_layout(cap, 4 * MAXW);
@@ -659,45 +716,56 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
   const uint32_t lut_a = sbase + S.tables;  // lut is the first member
   const uint32_t codelen_a = sbase + S.tables + (uint32_t)offsetof(DecodeTables, codelen);
   const uint32_t bar_stage = sbase + S.bars, bar_sm = sbase + S.bars + 16;
-  uint32_t *meta = reinterpret_cast<uint32_t *>(smem + S.meta);  // [stage][P0, P1, m, b]
+  uint32_t *meta = reinterpret_cast<uint32_t *>(smem + S.meta);  // [stage][P0, P1, m, u, PM]
   uint32_t *warp_tot = reinterpret_cast<uint32_t *>(smem + S.warp);
   const uint32_t lin_a = sbase + S.linear;
   const uint32_t sm_a = sbase + S.sm;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const uint32_t priv_a = sbase + S.priv + t * (4 * MAXW);
 
-  const uint64_t total = P.block_start[P.count];
+  const uint64_t total = P.unit_start[P.count];
   const uint64_t g0 = (uint64_t)blockIdx.x * total / gridDim.x;
   const uint64_t g1 = (uint64_t)(blockIdx.x + 1) * total / gridDim.x;
   if (g0 >= g1) return;
 
-  // thread 0 fetches the block after next's positions one iteration early
-  uint32_t nxt_p0 = 0, nxt_p1 = 0, nxt_m = 0;
+  // thread 0 fetches the unit after next's positions one iteration early:
+  // its first output P0, the first output of its second block PM (P1 if it
+  // has one block) and the end of its outputs P1
+  uint32_t nxt_p0 = 0, nxt_p1 = 0, nxt_pm = 0, nxt_m = 0;
   uint32_t hint = 0;
-  auto issue_stream = [&](uint64_t g, uint32_t stage, uint32_t p0, uint32_t p1, uint32_t m) {
+  auto issue_stream = [&](uint64_t g, uint32_t stage, uint32_t p0, uint32_t p1, uint32_t pm,
+                          uint32_t m) {
     const DecMat &M = P.m[m];
-    const uint64_t b = g - P.block_start[m];
+    const uint32_t u = (uint32_t)(g - P.unit_start[m]);
+    // the unit's blocks (the last unit of a matrix may hold one) and the
+    // 16 bytes after them; nothing beyond the stream's and gaps' allocations
+    const uint32_t nb = min(kUnitBlocks, M.n_blocks - kUnitBlocks * u);
+    const uint32_t sbytes = nb * kBlockStreamBytes + 16, gbytes = nb * kBlockGapBytes;
     const uint32_t st = sbase + (stage ? S.stage1 : S.stage0);
-    meta[stage * 4 + 0] = p0;
-    meta[stage * 4 + 1] = p1;
-    meta[stage * 4 + 2] = m;
-    meta[stage * 4 + 3] = (uint32_t)b;
+    meta[stage * 8 + 0] = p0;
+    meta[stage * 8 + 1] = p1;
+    meta[stage * 8 + 2] = m;
+    meta[stage * 8 + 3] = u;
+    meta[stage * 8 + 4] = pm;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(bar_stage + 8 * stage, kStreamStage + kGapStage);
-    bulk_g2s(st, M.stream + b * (8 * kT), kStreamStage, bar_stage + 8 * stage);
-    bulk_g2s(st + kStreamStage, M.gaps + b * kGapStage, kGapStage, bar_stage + 8 * stage);
+    mbar_expect_tx(bar_stage + 8 * stage, sbytes + gbytes);
+    bulk_g2s(st, M.stream + (uint64_t)u * (8 * kUnitChunks), sbytes, bar_stage + 8 * stage);
+    bulk_g2s(st + kStreamStage, M.gaps + (uint64_t)u * kGapStage, gbytes, bar_stage + 8 * stage);
   };
   auto fetch_pos = [&](uint64_t g) {
-    BlockRef r = locate(P, g, hint);
+    UnitRef r = locate(P, g, hint);
     hint = r.m;
     nxt_m = r.m;
-    nxt_p0 = __ldg(P.m[r.m].pos + r.b);
-    nxt_p1 = __ldg(P.m[r.m].pos + r.b + 1);
+    const DecMat &M = P.m[r.m];
+    const uint32_t b0 = kUnitBlocks * r.u;
+    nxt_p0 = __ldg(M.pos + b0);
+    nxt_p1 = __ldg(M.pos + min(b0 + kUnitBlocks, M.n_blocks));
+    nxt_pm = b0 + 1 < M.n_blocks ? __ldg(M.pos + b0 + 1) : nxt_p1;
   };
 
   // the linear row and the private regions start zeroed (the row's words are
   // OR-ed into; a region holds zeros beyond its codes)
-  for (uint32_t k = t; k < (cap + 16) / 4; k += kT) sts32(lin_a + 4 * k, 0u);
+  for (uint32_t k = t; k < (S.priv - S.linear) / 4; k += kT) sts32(lin_a + 4 * k, 0u);
 #pragma unroll
   for (int k = 0; k < MAXW; ++k) sts32(priv_a + 4 * k, 0u);
   if (t == 0) {
@@ -706,7 +774,7 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
     mbar_init(bar_sm, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fetch_pos(g0);
-    issue_stream(g0, 0, nxt_p0, nxt_p1, nxt_m);
+    issue_stream(g0, 0, nxt_p0, nxt_p1, nxt_pm, nxt_m);
     if (g0 + 1 < g1) fetch_pos(g0 + 1);
   }
   __syncthreads();
@@ -716,16 +784,16 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
   Pending prev{0, 0, nullptr, false};
   for (uint64_t g = g0, it = 0; g < g1; ++g, ++it) {
     const uint32_t s = (uint32_t)(it & 1);
-    // [A] the previous block is relocated into the linear row
+    // [A] the previous unit is relocated into the linear row
     if (it) __syncthreads();
-    const uint32_t *mt = meta + s * 4;
-    const uint32_t P0 = mt[0], P1 = mt[1], m = mt[2], b = mt[3];
+    const uint32_t *mt = meta + s * 8;
+    const uint32_t P0 = mt[0], P1 = mt[1], m = mt[2], u = mt[3], PM = mt[4];
     const DecMat &M = P.m[m];
     // positions are trusted only as far as they stay inside the matrix and
     // the staging row; anything else is flagged as corrupt after the count
     const bool sane = P1 >= P0 && P1 <= M.n && P1 - P0 <= cap;
     if (t == 0 && g + 1 < g1) {
-      issue_stream(g + 1, s ^ 1, nxt_p0, nxt_p1, nxt_m);
+      issue_stream(g + 1, s ^ 1, nxt_p0, nxt_p1, nxt_pm, nxt_m);
       if (g + 2 < g1) fetch_pos(g + 2);
     }
     if (m != cur_m) {
@@ -736,7 +804,7 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
       cur_m = m;
       __syncthreads();
       // every table entry must spend at least min_len bits per code, so that
-      // no chunk can produce more codes than its private region holds
+      // no thread can produce more codes than its private region holds
       bool tbad = false;
       for (uint32_t k = t; k < (uint32_t)df11i::kLutSize; k += kT) {
         const uint32_t e = tab.lut[k], used = e >> 28, ns = (e >> 24) & 0x3u;
@@ -749,53 +817,65 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
     const uint32_t st = sbase + (s ? S.stage1 : S.stage0);
     bool timed_out = !mbar_wait(bar_stage + 8 * s, (uint32_t)((it >> 1) & 1));
 
-    // ---- this thread's chunk: decode once into the private region
-    const uint32_t c = b * kT + t;
+    // ---- this thread's two chunks: decoded once into the private region
+    const uint32_t c0 = u * kUnitChunks + kCPT * t;
     uint32_t cnt = 0;
     bool bad = false;
-    if (table_ok && c < M.n_chunks) {
-      const uint2 ab = lds64(st + 8 * t);
-      const uint32_t C = bswap32(lds32(st + 8 * t + 8));
-      const uint32_t A = bswap32(ab.x), B = bswap32(ab.y);
-      const uint32_t lim = c + 1 < M.n_chunks ? 64u : M.tail_bits;
-      const uint32_t q = 5u * t;
+    if (table_ok && c0 < M.n_chunks) {
+      // stream words W0..W3 of the two chunks and the next chunk's first, W4
+      const uint4 a4 = lds128(st + 16 * t);
+      const uint32_t W0 = bswap32(a4.x), W1 = bswap32(a4.y), W2 = bswap32(a4.z),
+                     W3 = bswap32(a4.w), W4 = bswap32(lds32(st + 16 * t + 16));
+      const uint64_t avail = M.total_bits - 64ull * c0;
+      const uint32_t lim = avail < 64u * kCPT ? (uint32_t)avail : 64u * kCPT;
+      // the first chunk's 5-bit gap
+      const uint32_t q = DF11_GAP_BITS * kCPT * t;
       const uint32_t ga = st + kStreamStage + (q >> 3);
       const uint32_t two = (lds8(ga) << 8) | lds8(ga + 1);
       const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
       uint32_t p = gap, d = 0, e = 0;
-      // codes starting in the chunk's first word, then in its second (each
-      // loop's window needs no select).  With codes longer than the table's
-      // reach, a flagged entry leaves the loops, the code is decoded by the
-      // length search, and the loops resume after it
-      const uint32_t lim1 = min(lim, 32u);
       if (table_short) {
+        // one loop per 32-bit word in which codes start (each loop's window
+        // needs no select): while p < 32(k+1) the window is Wk:Wk+1 << p % 32
+        const uint32_t l1 = min(lim, 32u), l2 = min(lim, 64u), l3 = min(lim, 96u);
 #pragma unroll 1
-        while (p < lim1) {
-          const uint32_t w = __funnelshift_l(B, A, p);
+        while (p < l1) {
+          const uint32_t w = __funnelshift_l(W1, W0, p);
+          DF11_FAST_STEP_NOFLAG(w)
+        }
+#pragma unroll 1
+        while (p < l2) {
+          const uint32_t w = __funnelshift_l(W2, W1, p);
+          DF11_FAST_STEP_NOFLAG(w)
+        }
+#pragma unroll 1
+        while (p < l3) {
+          const uint32_t w = __funnelshift_l(W3, W2, p);
           DF11_FAST_STEP_NOFLAG(w)
         }
 #pragma unroll 1
         while (p < lim) {
-          const uint32_t w = __funnelshift_l(C, B, p);  // the shift is p - 32
+          const uint32_t w = __funnelshift_l(W4, W3, p);
           DF11_FAST_STEP_NOFLAG(w)
         }
       } else {
+        // codes longer than the table's reach: per word a table loop; a
+        // flagged entry leaves it, the code is decoded by the length search
+        // (its 32-bit window lies inside Wk:Wk+1 too), and the loop resumes
 #pragma unroll 1
-        for (;;) {
+        while (p < lim) {
+          const uint32_t k = p >> 5;
+          const uint32_t hi = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
+          const uint32_t lo = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
+          const uint32_t seg = min(lim, 32u * (k + 1));
+          bool flagged = false;
 #pragma unroll 1
-          while (p < lim1) {
-            const uint32_t w = __funnelshift_l(B, A, p);
-            DF11_FAST_STEP(w)
+          while (p < seg) {
+            const uint32_t w = __funnelshift_l(lo, hi, p);
+            DF11_FAST_STEP_FLAG(w, flagged)
           }
-          if (p >= lim1) {
-#pragma unroll 1
-            while (p < lim) {
-              const uint32_t w = __funnelshift_l(C, B, p);  // the shift is p - 32
-              DF11_FAST_STEP(w)
-            }
-            if (p >= lim) break;
-          }
-          const uint32_t w = window32(A, B, C, p);
+          if (!flagged) continue;
+          const uint32_t w = __funnelshift_l(lo, hi, p);
           const uint32_t L = long_code_len(w, tab);
           if (L == 0) {
             bad = true;
@@ -808,8 +888,8 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
         }
       }
       if (d && p > lim) {
-        // the last entry ran past the chunk's end: keep its codes that start
-        // before lim, clear the others
+        // the last entry ran past the end of the thread's chunks: keep its
+        // codes that start before lim, clear the others
         const uint32_t ns = (e >> 24) & 0x3u;
         const uint32_t q1 = p - (e >> 28) + lds8(codelen_a + (e & 0xFFu));
         const uint32_t q2 = q1 + lds8(codelen_a + ((e >> 8) & 0xFFu));
@@ -821,8 +901,8 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
       }
       cnt = d;
     }
-    // ---- the previous block's merge (between decode and the count barrier);
-    // its sign/mantissa phase is waited for even if the block was rejected,
+    // ---- the previous unit's merge (between decode and the count barrier);
+    // its sign/mantissa phase is waited for even if the unit was rejected,
     // so that the barrier is never re-armed with a copy in flight
     if (it) {
       if (!mbar_wait(bar_sm, (uint32_t)((it - 1) & 1))) timed_out = true;
@@ -839,7 +919,7 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
     const uint32_t wtime = __ballot_sync(0xffffffffu, timed_out) ? 0x40000000u : 0u;
     if (lane == 31) warp_tot[warp] = incl | wflags | wtime;
     __syncthreads();
-    uint32_t wpre = 0, tot = 0, flagbits = 0;
+    uint32_t wpre = 0, tot = 0, tot_first = 0, flagbits = 0;
     {
       const uint4 lo4 = reinterpret_cast<const uint4 *>(warp_tot)[0];
       const uint4 hi4 = reinterpret_cast<const uint4 *>(warp_tot)[1];
@@ -850,21 +930,25 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
         const uint32_t v = x[i] & 0x3FFFFFFFu;
         tot += v;
         wpre += i < warp ? v : 0u;
+        tot_first += i < kFirstBlockWarps ? v : 0u;
       }
     }
     if (flagbits & 0x40000000u) {
       // a bounded wait ran out: leave (uniformly) with the status set, after
-      // a bounded wait for the next block's copy issued at the top
+      // a bounded wait for the next unit's copy issued at the top
       if (t == 0) {
         set_status(P.status, DF11_ERR_TIMEOUT);
         if (g + 1 < g1) mbar_wait(bar_stage + 8 * (s ^ 1), (uint32_t)(((it + 1) >> 1) & 1));
       }
       return;
     }
-    const bool ok = table_ok && sane && !(flagbits >> 31) && tot == P1 - P0;
+    // the codes of the whole unit and of its first block must match the
+    // block positions (every stored position is checked)
+    const bool ok =
+        table_ok && sane && !(flagbits >> 31) && tot == P1 - P0 && tot_first == PM - P0;
     if (t == 0) {
       if (!ok) set_status(P.status, DF11_ERR_CORRUPT);
-      // this block's sign/mantissa bytes (the previous block's merge is done),
+      // this unit's sign/mantissa bytes (the previous unit's merge is done),
       // rounded out to 16 B
       const uint32_t sm_lo = P0 & ~15u;
       const uint32_t sm_bytes = sane ? (uint32_t)((((uint64_t)P1 + 15u) & ~15ull) - sm_lo) : 0u;
@@ -892,14 +976,14 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
           prevw = cur;
         }
       } else {
-        // a rejected block still leaves the private region cleared
+        // a rejected unit still leaves the private region cleared
 #pragma unroll
         for (int k = 0; k < MAXW; ++k) sts32(priv_a + 4 * k, 0u);
       }
     }
     prev = Pending{P0, P1, M.out, ok};
   }
-  // the last block's merge
+  // the last unit's merge
   __syncthreads();
   if (!mbar_wait(bar_sm, (uint32_t)((g1 - g0 - 1) & 1))) {
     if (lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
@@ -908,13 +992,14 @@ __global__ void __launch_bounds__(kT, 4) decode_kernel(const __grid_constant__ D
   }
 }
 
-#undef DF11_FAST_STEP
+#undef DF11_FAST_STEP_FLAG
+#undef DF11_FAST_STEP_NOFLAG
 
 // ============================================================ launch helpers
 
 // decode_kernel instantiations: regions of codes >= 2 bits and >= 1 bit
-constexpr int kMaxWords2 = 9;   // region_bytes_for(2) / 4
-constexpr int kMaxWords1 = 17;  // region_bytes_for(1) / 4
+constexpr int kMaxWords2 = 17;  // region_bytes_for(2) / 4
+constexpr int kMaxWords1 = 33;  // region_bytes_for(1) / 4
 static_assert(region_bytes_for(2) == 4 * kMaxWords2 && region_bytes_for(1) == 4 * kMaxWords1,
               "private region sizes");
 
@@ -940,7 +1025,8 @@ df11_status device_info(int *dev, int *sms) {
     if (cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kHistSmem) != cudaSuccess)
       return DF11_ERR_CUDA;
-    const int max_smem = (int)smem_layout(16384, region_bytes_for(1)).total;
+    // the largest staging: a unit of codes of one bit
+    const int max_smem = (int)smem_layout(64 * kCPT * kT, region_bytes_for(1)).total;
     if (cudaFuncSetAttribute(decode_kernel<kMaxWords2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess ||
         cudaFuncSetAttribute(decode_kernel<kMaxWords1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -974,7 +1060,7 @@ extern "C" df11_status df11_histogram(const uint16_t *d_w, uint64_t n, uint64_t 
   auto *h = reinterpret_cast<unsigned long long *>(d_hist256);
   hist_clear_kernel<<<1, 256, 0, s>>>(h);
   if (n) {
-    const uint64_t vec_warps = cdiv(n >> 3, 128);
+    const uint64_t vec_warps = cdiv(n >> 3, kHistUnroll * 32);
     uint64_t grid = (uint64_t)sms * 3;
     grid = vec_warps ? std::min<uint64_t>(grid, cdiv(vec_warps, kHistWarps)) : 1;
     if (grid < 1) grid = 1;
@@ -1008,9 +1094,10 @@ extern "C" df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_c
     ecb.len[i] = cb->len[i];
   }
   const uint64_t C = cdiv(total_bits, 64);
-  const uint64_t B = cdiv(C, kT);
-  const uint64_t stream_alloc = 8 * kT * B + 16;
-  const uint64_t gaps_alloc = kGapStage * B + 16;
+  const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
+  // the stream and gap allocations of the format (df11_encoded_sizes)
+  const uint64_t stream_alloc = (uint64_t)kBlockStreamBytes * B + 16;
+  const uint64_t gaps_alloc = (uint64_t)kBlockGapBytes * B + 16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   auto *ws = reinterpret_cast<uint64_t *>(d_workspace);
   const uint64_t grid1 = std::max<uint64_t>(n_tiles, 1);
@@ -1043,9 +1130,9 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
     DecParams P;
     P.count = 0;
     P.status = d_status;
-    P.block_start[0] = 0;
+    P.unit_start[0] = 0;
     uint32_t min_len = DF11_MAX_CODE_LEN;
-    uint32_t block_codes = 0;  // staging size: most codes in one block of the batch
+    uint32_t unit_codes = 0;  // staging size: most codes in one unit of the batch
     for (uint32_t i = 0; i < k; ++i) {
       const df11_matrix &m = ms[first + i];
       if (m.n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
@@ -1060,11 +1147,15 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
       if (m.min_len < 1 || m.min_len > 8) return DF11_ERR_INVALID_ARG;
       if (m.total_bits < m.n * (uint64_t)m.min_len || m.total_bits > m.n * 32ull)
         return DF11_ERR_INVALID_ARG;
-      const uint32_t worst = (uint32_t)cdiv(64, m.min_len) * kT;
-      if (m.max_block_codes > worst) return DF11_ERR_INVALID_ARG;
-      block_codes = std::max(block_codes, m.max_block_codes ? m.max_block_codes : worst);
+      // codes that can start in one block / one unit
+      const uint32_t worst_block = (uint32_t)cdiv(64, m.min_len) * DF11_BLOCK_CHUNKS;
+      const uint32_t worst_unit = (uint32_t)cdiv(64 * kCPT, m.min_len) * kT;
+      if (m.max_block_codes > worst_block) return DF11_ERR_INVALID_ARG;
+      unit_codes = std::max(unit_codes, m.max_block_codes
+                                            ? std::min(kUnitBlocks * m.max_block_codes, worst_unit)
+                                            : worst_unit);
       const uint64_t C = cdiv(m.total_bits, 64);
-      const uint64_t B = cdiv(C, kT);
+      const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
       if (C >= (1ull << 31)) return DF11_ERR_TOO_LARGE;
       DecMat &d = P.m[P.count];
       d.stream = m.stream;
@@ -1074,25 +1165,28 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
       d.tables = reinterpret_cast<const DecodeTables *>(m.tables);
       d.out = d_outs[first + i];
       d.n = m.n;
+      d.total_bits = m.total_bits;
       d.n_chunks = (uint32_t)C;
-      d.tail_bits = (uint32_t)(m.total_bits - 64 * (C - 1));
-      P.block_start[P.count + 1] = P.block_start[P.count] + B;
+      d.n_blocks = (uint32_t)B;
+      P.unit_start[P.count + 1] = P.unit_start[P.count] + cdiv(B, kUnitBlocks);
       min_len = std::min(min_len, m.min_len);
       ++P.count;
     }
     if (P.count == 0) continue;
-    for (uint32_t i = P.count + 1; i <= DF11_MAX_BATCH; ++i) P.block_start[i] = P.block_start[P.count];
-    P.stage_cap = (block_codes + 15u) & ~15u;
+    for (uint32_t i = P.count + 1; i <= DF11_MAX_BATCH; ++i) P.unit_start[i] = P.unit_start[P.count];
+    P.stage_cap = (unit_codes + 15u) & ~15u;
     P.region_bytes = 4u * (min_len >= 2 ? kMaxWords2 : kMaxWords1);
     P.min_len = min_len;
-    const uint32_t smem = smem_layout(P.stage_cap, P.region_bytes).total;
+    const SmemLayout L = smem_layout(P.stage_cap, P.region_bytes);
+    if (!smem_layout_aligned(L)) return DF11_ERR_INVALID_ARG;
+    const uint32_t smem = L.total;
     auto kern = min_len >= 2 ? decode_kernel<kMaxWords2> : decode_kernel<kMaxWords1>;
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kT, smem) != cudaSuccess)
       return DF11_ERR_CUDA;
     if (occ < 1) return DF11_ERR_CUDA;
-    const uint64_t blocks = P.block_start[P.count];
-    const uint64_t grid = std::min<uint64_t>(blocks, (uint64_t)sms * occ);
+    const uint64_t units = P.unit_start[P.count];
+    const uint64_t grid = std::min<uint64_t>(units, (uint64_t)sms * occ);
     kern<<<(unsigned)grid, kT, smem, s>>>(P);
     st = launch_status();
     if (st != DF11_OK) return st;
@@ -1177,9 +1271,10 @@ extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
     ecb.len[i] = cb->len[i];
   }
   const uint64_t C = cdiv(total_bits, 64);
-  const uint64_t B = cdiv(C, kT);
-  const uint64_t stream_alloc = 8 * kT * B + 16;
-  const uint64_t gaps_alloc = kGapStage * B + 16;
+  const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
+  // the stream and gap allocations of the format (df11_encoded_sizes)
+  const uint64_t stream_alloc = (uint64_t)kBlockStreamBytes * B + 16;
+  const uint64_t gaps_alloc = (uint64_t)kBlockGapBytes * B + 16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // nothing in the array needs clearing: every tile offset a call reads is
   // written earlier in the same call

@@ -158,11 +158,13 @@ def test_decode_reports_corrupt_positions_without_fault(codec, cap):
     x = workloads.random_bf16(2_000_000, seed=9)
     m = codec.compress(to_dev(x), cap=cap)
     pos = m.block_pos.clone()
-    m.block_pos[3] += 5
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    codec.decompress(m, status=status)
-    assert int(status.item()) == 4  # DF11_ERR_CORRUPT
-    m.block_pos.copy_(pos)
+    for b in (3, 4):  # a position inside a decode unit and one between two units
+        m.block_pos[b] += 5
+        status.zero_()
+        codec.decompress(m, status=status)
+        assert int(status.item()) == 4  # DF11_ERR_CORRUPT
+        m.block_pos.copy_(pos)
     m.block_pos[5] = int(m.n) + 100  # beyond the matrix: must not be dereferenced
     status.zero_()
     codec.decompress(m, status=status)
