@@ -529,9 +529,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                : "memory");
   return v;
 }
-__device__ __forceinline__ void sts8(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
@@ -603,36 +600,43 @@ __device__ __forceinline__ uint32_t long_code_len(uint32_t w32, const DecodeTabl
   return 0;
 }
 
-// One table step of the decoder on window w.  A flagged entry (first code
-// longer than the table's reach) sets f and leaves the loop before anything
-// is stored; otherwise the entry's three exponent slots are stored at dst+d
-// (absent slots are zero), d advances by the number of codes and p by the
-// bits they use.
-#define DF11_FAST_STEP_FLAG(w, f)                                           \
+// Appending decoded exponents to a thread's private bytes.  The private
+// regions of a warp are interleaved by 32-bit word: word j of lane l is
+// shared word 32 j + l of the warp's region, so any access in which every
+// lane touches one word of its own falls in 32 different banks.  The word
+// being filled is kept in a register (cur) and written through on every
+// step with one 32-bit store at row_a; nb counts the bits appended (8 per
+// exponent).  x holds the step's exponents from the low byte up (absent
+// slots zero), cm its count in bits 24-25.
+#define DF11_APPEND(x, cm)                                                  \
+  {                                                                         \
+    const uint32_t xs = (x);                                                \
+    const uint32_t lo = cur | __funnelshift_l(0u, xs, nb);                  \
+    const uint32_t hi = __funnelshift_l(xs, 0u, nb);                        \
+    sts32(row_a, lo);                                                       \
+    const uint32_t nb2 = madhi((cm), 1u << 11, nb);                         \
+    row_a = col_a + ((nb2 >> 5) << 7);                                      \
+    cur = __funnelshift_rc(lo, hi, (nb ^ nb2) & 32u);                       \
+    nb = nb2;                                                               \
+  }
+
+// One table step of the decoder on window w: the entry's exponents are
+// appended and p advances by the bits they use.  In the flagged form an
+// entry whose first code is longer than the table's reach sets f and leaves
+// the loop before anything is appended.
+#define DF11_STEP_FLAG(w, f)                                                \
   e = lds32(lut_a + (mulhi((w), 1u << df11i::kLutBits) << 2));              \
   if (e & df11i::kLutLongFlag) {                                            \
     f = true;                                                               \
     break;                                                                  \
   }                                                                         \
-  {                                                                         \
-    const uint32_t at = priv_a + d;                                         \
-    sts8(at, e);                                                            \
-    sts8(at + 1, mulhi(e, 1u << 24));                                       \
-    sts8(at + 2, mulhi(e, 1u << 16));                                       \
-    d = madhi(e & df11i::kLutCountMask, 1u << 8, d);                        \
-    p = madhi(e, 1u << 4, p);                                               \
-  }
+  DF11_APPEND(e & 0x00FFFFFFu, e & df11i::kLutCountMask)                    \
+  p = madhi(e, 1u << 4, p);
 
-// The same step for tables whose codes all fit in kLutBits bits: no flag
-// test, nothing but the loop's exit branches.
-#define DF11_FAST_STEP_NOFLAG(w)                                            \
+#define DF11_STEP(w)                                                        \
   {                                                                         \
     e = lds32(lut_a + (mulhi((w), 1u << df11i::kLutBits) << 2));            \
-    const uint32_t at = priv_a + d;                                         \
-    sts8(at, e);                                                            \
-    sts8(at + 1, mulhi(e, 1u << 24));                                       \
-    sts8(at + 2, mulhi(e, 1u << 16));                                       \
-    d = madhi(e & df11i::kLutCountMask, 1u << 8, d);                        \
+    DF11_APPEND(e & 0x00FFFFFFu, e & df11i::kLutCountMask)                  \
     p = madhi(e, 1u << 4, p);                                               \
   }
 
@@ -721,7 +725,8 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
   const uint32_t lin_a = sbase + S.linear;
   const uint32_t sm_a = sbase + S.sm;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const uint32_t priv_a = sbase + S.priv + t * (4 * MAXW);
+  // this lane's column of its warp's interleaved private region
+  const uint32_t col_a = sbase + S.priv + (uint32_t)warp * (MAXW * 128u) + 4u * lane;
 
   const uint64_t total = P.unit_start[P.count];
   const uint64_t g0 = (uint64_t)blockIdx.x * total / gridDim.x;
@@ -767,7 +772,7 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
   // OR-ed into; a region holds zeros beyond its codes)
   for (uint32_t k = t; k < (S.priv - S.linear) / 4; k += kT) sts32(lin_a + 4 * k, 0u);
 #pragma unroll
-  for (int k = 0; k < MAXW; ++k) sts32(priv_a + 4 * k, 0u);
+  for (int k = 0; k < MAXW; ++k) sts32(col_a + 128 * k, 0u);
   if (t == 0) {
     mbar_init(bar_stage, 1);
     mbar_init(bar_stage + 8, 1);
@@ -833,7 +838,7 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
       const uint32_t ga = st + kStreamStage + (q >> 3);
       const uint32_t two = (lds8(ga) << 8) | lds8(ga + 1);
       const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
-      uint32_t p = gap, d = 0, e = 0;
+      uint32_t p = gap, e = 0, nb = 0, cur = 0, row_a = col_a;
       if (table_short) {
         // one loop per 32-bit word in which codes start (each loop's window
         // needs no select): while p < 32(k+1) the window is Wk:Wk+1 << p % 32
@@ -841,22 +846,22 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
 #pragma unroll 1
         while (p < l1) {
           const uint32_t w = __funnelshift_l(W1, W0, p);
-          DF11_FAST_STEP_NOFLAG(w)
+          DF11_STEP(w)
         }
 #pragma unroll 1
         while (p < l2) {
           const uint32_t w = __funnelshift_l(W2, W1, p);
-          DF11_FAST_STEP_NOFLAG(w)
+          DF11_STEP(w)
         }
 #pragma unroll 1
         while (p < l3) {
           const uint32_t w = __funnelshift_l(W3, W2, p);
-          DF11_FAST_STEP_NOFLAG(w)
+          DF11_STEP(w)
         }
 #pragma unroll 1
         while (p < lim) {
           const uint32_t w = __funnelshift_l(W4, W3, p);
-          DF11_FAST_STEP_NOFLAG(w)
+          DF11_STEP(w)
         }
       } else {
         // codes longer than the table's reach: per word a table loop; a
@@ -872,7 +877,7 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
 #pragma unroll 1
           while (p < seg) {
             const uint32_t w = __funnelshift_l(lo, hi, p);
-            DF11_FAST_STEP_FLAG(w, flagged)
+            DF11_STEP_FLAG(w, flagged)
           }
           if (!flagged) continue;
           const uint32_t w = __funnelshift_l(lo, hi, p);
@@ -881,22 +886,25 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
             bad = true;
             break;
           }
-          sts8(priv_a + d, tab.sym[((w >> (32 - L)) + tab.base[L]) & 0xFFu]);
-          d += 1;
+          DF11_APPEND(tab.sym[((w >> (32 - L)) + tab.base[L]) & 0xFFu], 1u << 24)
           p += L;
           e = 1u << 24;  // one code: nothing to trim below
         }
       }
+      sts32(row_a, cur);  // the word being filled (it may have just begun)
+      uint32_t d = nb >> 3;
       if (d && p > lim) {
         // the last entry ran past the end of the thread's chunks: keep its
-        // codes that start before lim, clear the others
+        // codes that start before lim, clear the others (byte k of the lane
+        // is byte k % 4 of its word k / 4)
         const uint32_t ns = (e >> 24) & 0x3u;
         const uint32_t q1 = p - (e >> 28) + lds8(codelen_a + (e & 0xFFu));
         const uint32_t q2 = q1 + lds8(codelen_a + ((e >> 8) & 0xFFu));
         const bool drop2 = ns >= 2 && q1 >= lim;
         const bool drop3 = ns == 3 && q2 >= lim;
-        sts8_if(priv_a + d - ns + 1, 0u, drop2);
-        sts8_if(priv_a + d - 1, 0u, drop3);
+        const uint32_t k2 = d - ns + 1, k3 = d - 1;
+        sts8_if(col_a + ((k2 >> 2) << 7) + (k2 & 3u), 0u, drop2);
+        sts8_if(col_a + ((k3 >> 2) << 7) + (k3 & 3u), 0u, drop3);
         d -= (uint32_t)drop2 + (uint32_t)drop3;
       }
       cnt = d;
@@ -970,15 +978,15 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
         // beyond its codes are zero) and stay inside the row's slack
 #pragma unroll
         for (int j = 0; j <= MAXW; ++j) {
-          const uint32_t cur = j < MAXW ? lds32(priv_a + 4 * j) : 0u;
-          if (j < MAXW) sts32(priv_a + 4 * j, 0u);
+          const uint32_t cur = j < MAXW ? lds32(col_a + 128 * j) : 0u;
+          if (j < MAXW) sts32(col_a + 128 * j, 0u);
           red_or32(la + 4 * j, __funnelshift_l(prevw, cur, sh));
           prevw = cur;
         }
       } else {
         // a rejected unit still leaves the private region cleared
 #pragma unroll
-        for (int k = 0; k < MAXW; ++k) sts32(priv_a + 4 * k, 0u);
+        for (int k = 0; k < MAXW; ++k) sts32(col_a + 128 * k, 0u);
       }
     }
     prev = Pending{P0, P1, M.out, ok};
@@ -992,8 +1000,9 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
   }
 }
 
-#undef DF11_FAST_STEP_FLAG
-#undef DF11_FAST_STEP_NOFLAG
+#undef DF11_APPEND
+#undef DF11_STEP_FLAG
+#undef DF11_STEP
 
 // ============================================================ launch helpers
 
