@@ -84,9 +84,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+DECODE_BEGIN = "// ============================================================ decode"
+DECODE_END = "// ============================================================ launch helpers"
+
+
 def kernel_hash() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Fingerprint of the decode kernel's source (the decode section of
+    df11_kernels.cu), so that a stored traffic figure is used only for the
+    kernel it was measured on."""
+    with open(KERNEL_SOURCE, encoding="utf-8") as f:
+        src = f.read()
+    a, b = src.find(DECODE_BEGIN), src.find(DECODE_END)
+    section = src[a:b] if 0 <= a < b else src
+    return hashlib.sha256(section.encode()).hexdigest()[:16]
 
 
 def profiled_traffic(workload_name: str):

@@ -263,23 +263,23 @@ __global__ void __launch_bounds__(kScanThreads) enc_scan_kernel(
   }
 }
 
-// Pack the codes of one tile.  Each thread appends its 16 codes to a 64-bit
-// register accumulator (most significant bit first) and writes every 32-bit
-// word it completes to a shared bit buffer covering the tile's bit range: a
-// thread's interior words hold its bits alone and are plain stores; its first
-// and last words may hold a neighbouring thread's bits and are OR-ed in.  The
-// buffer is then written out as 32-bit words (byte-swapped to the MSB-first
-// byte order); the two edge words are shared with the neighbouring tiles and
-// are OR-ed atomically into the cleared stream.  The thread that owns the
-// first code starting in a chunk writes that chunk's 5-bit gap; the one that
-// owns the first code starting in a block of 256 chunks writes the block's
-// output position.
-__device__ __forceinline__ void or_gap(uint32_t *gaps32, uint64_t gap_words, uint64_t c, uint32_t g) {
-  const uint64_t q = 5 * c;
-  const uint64_t gw = q >> 5;
-  const uint64_t y = (uint64_t)g << (59 - (uint32_t)(q & 31u));
-  if (gw < gap_words) atomicOr(&gaps32[gw], bswap32((uint32_t)(y >> 32)));
-  if ((uint32_t)y && gw + 1 < gap_words) atomicOr(&gaps32[gw + 1], bswap32((uint32_t)y));
+// Pack the codes of one tile.  Each thread appends its 16 codes to a pair of
+// 32-bit registers (the word being filled and the next, most significant bit
+// first) and ORs every word it completes into a shared bit buffer covering
+// the tile's bit range (a thread's first and last words may hold a
+// neighbouring thread's bits).  The thread that owns the first code starting
+// in a chunk records that chunk's gap in a shared byte per chunk; the one
+// that owns the first code starting in a block of 256 chunks writes the
+// block's output position.  The buffer is then written out as 32-bit words
+// (byte-swapped to the MSB-first byte order), and the tile's gaps as packed
+// 5-bit fields; words shared with the neighbouring tiles are OR-ed
+// atomically into the cleared stream and gap buffers.  Codes arrive
+// left-justified (code << (32 - length)).
+__device__ __forceinline__ void red_or_shared_if(uint32_t *p, uint32_t v, bool c) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q red.shared.or.b32 [%0], %1;\n}\n" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(p)),
+               "r"(v), "r"((uint32_t)c)
+               : "memory");
 }
 
 __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
@@ -289,84 +289,102 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     uint32_t *__restrict__ block_pos, uint64_t n_blocks, uint8_t *__restrict__ sign_mantissa) {
   constexpr int kWords = df11i::kEncTile * DF11_MAX_CODE_LEN / 32 + 2;
   __shared__ uint32_t s_bits[kWords];
-  __shared__ uint2 s_lc[256];  // {length, code}
+  __shared__ uint2 s_lc[256];  // {length, left-justified code}
   __shared__ uint32_t s_warp[df11i::kEncThreads / 32];
+  __shared__ uint32_t s_lastlen[df11i::kEncThreads / 32];  // each warp's last code length
+  // gap of each chunk from chunk S0/64 on; 0xFF: the chunk's first code is
+  // not in this tile
+  constexpr int kGapChunks = df11i::kEncTile * DF11_MAX_CODE_LEN / DF11_CHUNK_BITS + 2;
+  __shared__ uint8_t s_gap[kGapChunks];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   s_lc[t] = make_uint2(cb.len[t], cb.code[t]);
+  for (int k = t; k < kGapChunks; k += df11i::kEncThreads) s_gap[k] = 0xFFu;
   const uint64_t tile = blockIdx.x;
   const uint64_t S = tile_start[tile], E = tile_start[tile + 1];
   const uint64_t S0 = S & ~31ull;
   const uint32_t nwords = (uint32_t)((E - S0 + 31) >> 5);
   for (uint32_t k = t; k < nwords + 1 && k < (uint32_t)kWords; k += df11i::kEncThreads) s_bits[k] = 0u;
-  __syncthreads();
+  // the value before the tile (its length is the first code's predecessor)
+  const uint16_t before = (t == 0 && tile > 0) ? w[tile * df11i::kEncTile - 1] : (uint16_t)0;
 
   uint16_t v[16];
   const uint64_t i0 = tile * df11i::kEncTile + (uint64_t)t * df11i::kEncPerThread;
   load_tile_values(w, n, i0, v);
-  uint32_t sum = 0;
+  const uint32_t nk = i0 < n ? (n - i0 < 16 ? (uint32_t)(n - i0) : 16u) : 0u;  // values of this thread
+  // code-length sum, and the length of this thread's last value (the
+  // value before the next thread's first)
+  uint32_t sum = 0, my_last = 0;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) sum += (i0 + k < n) ? s_lc[(v[k] >> 7) & 0xFFu].x : 0u;
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t Lk = (uint32_t)k < nk ? s_lc[(v[k] >> 7) & 0xFFu].x : 0u;
+    sum += Lk;
+    my_last = (uint32_t)k < nk ? Lk : my_last;
+  }
   uint32_t incl = sum;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     uint32_t o = __shfl_up_sync(0xffffffffu, incl, d);
     if (lane >= d) incl += o;
   }
-  if (lane == 31) s_warp[warp] = incl;
+  if (lane == 31) {
+    s_warp[warp] = incl;
+    s_lastlen[warp] = my_last;
+  }
   __syncthreads();
   uint32_t wpre = 0;
   for (int i = 0; i < warp; ++i) wpre += s_warp[i];
   const uint32_t rel = (uint32_t)(S - S0) + wpre + incl - sum;  // bit offset in s_bits
-  uint64_t start = S + wpre + incl - sum;                       // absolute bit offset
-  // length of the value before this thread's first one
-  uint32_t prev_len = 0;
-  if (i0 > 0 && i0 < n) prev_len = s_lc[(w[i0 - 1] >> 7) & 0xFFu].x;
-  const uint64_t C = (total_bits + 63) >> 6;
-  uint32_t *gaps32 = reinterpret_cast<uint32_t *>(gaps);
-  const uint64_t gap_words = gaps_alloc >> 2;
-  // accumulator: bit 63 is bit (wi * 32) of the buffer; nb bits are filled
-  uint64_t acc = 0;
-  uint32_t nb = rel & 31u, wi = rel >> 5;
-  bool first_word = true;
+  const uint64_t start0 = S + wpre + incl - sum;                // absolute offset of the first code
+  // length of the value before this thread's first one: the previous
+  // thread's last (a value of the previous tile for thread 0)
+  const uint32_t up = __shfl_up_sync(0xffffffffu, my_last, 1);
+  uint32_t prev_len = lane ? up : (warp ? s_lastlen[warp - 1] : s_lc[(before >> 7) & 0xFFu].x);
+  if (i0 == 0 || !nk) prev_len = 0;
+  const uint32_t cb0 = (uint32_t)(S0 & 63u);  // S0's offset in its chunk
+  uint32_t hi = 0, lo = 0;                 // the word being filled (word wi) and the next
+  uint32_t nb = rel & 31u, wi = rel >> 5;  // bits of word wi already taken
+  uint32_t off = 0;                        // bits of this thread's codes so far
+  uint32_t last_len = 0;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    const uint64_t i = i0 + k;
-    if (i >= n) break;
+    if ((uint32_t)k >= nk) break;
     const uint2 lc = s_lc[(v[k] >> 7) & 0xFFu];
     const uint32_t L = lc.x;
-    // nb < 32 and L <= 32; a value without a code (L = 0, reported by the
-    // length-sum kernel) adds nothing
-    acc |= L ? ((uint64_t)lc.y << (64 - L)) >> nb : 0ull;
+    hi |= lc.y >> nb;                     // nb < 32
+    lo |= __funnelshift_r(0u, lc.y, nb);  // the code's bits past word wi
     nb += L;
-    if (nb >= 32) {
-      const uint32_t word = (uint32_t)(acc >> 32);
-      if (wi < (uint32_t)kWords) {
-        if (first_word) atomicOr(&s_bits[wi], word);
-        else s_bits[wi] = word;
+    const bool full = nb >= 32;
+    red_or_shared_if(&s_bits[wi < (uint32_t)kWords ? wi : 0u], hi, full && wi < (uint32_t)kWords);
+    wi += full ? 1u : 0u;
+    hi = full ? lo : hi;
+    lo = full ? 0u : lo;
+    nb -= full ? 32u : 0u;
+    // the code starts a chunk (block) when its offset in that chunk (block)
+    // is below the previous code's length; the very first code starts both
+    const uint32_t pos = cb0 + rel + off;  // bit offset from chunk S0/64
+    if ((k == 0 && i0 == 0) || (pos & 63u) < prev_len) {
+      if ((pos >> 6) < (uint32_t)kGapChunks) s_gap[pos >> 6] = (uint8_t)(pos & 63u);
+      if ((k == 0 && i0 == 0) || (((uint32_t)start0 + off) & 16383u) < prev_len) {
+        const uint64_t b = (start0 + off) >> 14;
+        if (b < n_blocks) block_pos[b] = (uint32_t)(i0 + k);
       }
-      first_word = false;
-      ++wi;
-      acc <<= 32;
-      nb -= 32;
-    }
-    // the code starts a new chunk (block) when its offset in that chunk
-    // (block) is below the previous code's length
-    if (i == 0 || (uint32_t)(start & 63u) < prev_len) {
-      or_gap(gaps32, gap_words, start >> 6, (uint32_t)(start & 63u));
-      if (i == 0 || (uint32_t)(start & 16383u) < prev_len) {
-        const uint64_t b = start >> 14;
-        if (b < n_blocks) block_pos[b] = (uint32_t)i;
-      }
-    }
-    if (i + 1 == n) {
-      // the last chunk / block may begin inside the final code
-      if (C > 0 && (start >> 6) < C - 1) or_gap(gaps32, gap_words, C - 1, (uint32_t)(total_bits - 64 * (C - 1)));
-      if (n_blocks > 0 && (start >> 14) < n_blocks - 1) block_pos[n_blocks - 1] = (uint32_t)n;
     }
     prev_len = L;
-    start += L;
+    last_len = L;
+    off += L;
   }
-  if (nb && wi < (uint32_t)kWords) atomicOr(&s_bits[wi], (uint32_t)(acc >> 32));
+  if (nb && wi < (uint32_t)kWords) atomicOr(&s_bits[wi], hi);
+  if (nk && i0 + nk == n) {
+    // the last chunk / block may begin inside the final code: its gap points
+    // at the end of the stream
+    const uint64_t C = (total_bits + 63) >> 6;
+    const uint64_t s64 = start0 + off - last_len;  // the final code's start
+    if (C > 0 && (s64 >> 6) < C - 1) {
+      const uint64_t lc = (C - 1) - (S0 >> 6);
+      if (lc < (uint64_t)kGapChunks) s_gap[lc] = (uint8_t)(total_bits - 64 * (C - 1));
+    }
+    if (n_blocks > 0 && (s64 >> 14) < n_blocks - 1) block_pos[n_blocks - 1] = (uint32_t)n;
+  }
   // sign/mantissa plane ([Format]: kept verbatim, one byte per value)
   if (i0 + 16 <= n) {
     uint32_t pk[4];
@@ -384,7 +402,7 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
   } else {
 #pragma unroll
     for (int k = 0; k < 16; ++k)
-      if (i0 + k < n) sign_mantissa[i0 + k] = (uint8_t)(((v[k] >> 8) & 0x80u) | (v[k] & 0x7Fu));
+      if ((uint32_t)k < nk) sign_mantissa[i0 + k] = (uint8_t)(((v[k] >> 8) & 0x80u) | (v[k] & 0x7Fu));
   }
   __syncthreads();
   uint32_t *stream32 = reinterpret_cast<uint32_t *>(stream);
@@ -396,6 +414,41 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     const uint32_t val = bswap32(s_bits[k]);
     if (k == 0 || k + 1 == nwords) atomicOr(&stream32[gw], val);
     else stream32[gw] = val;
+  }
+  // gaps: chunk c's five bits are bits 5c..5c+4 of the gap stream.  The
+  // chunks this tile may own are local 0 .. nch-1 (chunk S0/64 on); a word
+  // holding a chunk the tile does not own is OR-ed in, others are stored
+  if (E > S) {
+    const uint64_t c_base = S0 >> 6;
+    const uint32_t nch = ((cb0 + (uint32_t)(E - S0) - 1) >> 6) + 1;
+    const uint64_t w_lo = (5 * c_base) >> 5, w_hi = (5 * (c_base + nch) - 1) >> 5;
+    uint32_t *gaps32 = reinterpret_cast<uint32_t *>(gaps);
+    const uint64_t gap_words = gaps_alloc >> 2;
+    for (uint64_t gw = w_lo + t; gw <= w_hi; gw += df11i::kEncThreads) {
+      if (gw >= gap_words) break;
+      // 64-bit window: bit 63 is gap-stream bit 32 gw - 4
+      uint64_t acc = 0;
+      bool owned = true;
+      // the chunks touching the word: cf .. cf + 7 (cf's field begins at
+      // most 4 bits before the word)
+      const uint64_t cf = (32 * gw) / 5;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t c = (int64_t)cf + j;
+        const int64_t rb = 5 * c - (int64_t)(32 * gw) + 4;  // chunk's first bit in the window
+        if (rb > 35) continue;                              // begins after the word
+        const int64_t lc = c - (int64_t)c_base;
+        const uint32_t gv = (lc >= 0 && lc < (int64_t)nch) ? s_gap[lc] : 0xFFu;
+        if (gv == 0xFFu) {
+          owned = false;
+          continue;
+        }
+        acc |= (uint64_t)(gv & 31u) << (59 - rb);
+      }
+      const uint32_t val = bswap32((uint32_t)(acc >> 28));
+      if (owned) gaps32[gw] = val;
+      else if (val) atomicOr(&gaps32[gw], val);
+    }
   }
 }
 
@@ -1099,8 +1152,12 @@ extern "C" df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_c
   if (st != DF11_OK) return st;
   EncCodebook ecb;
   for (int i = 0; i < 256; ++i) {
-    ecb.code[i] = cb->code[i];
-    ecb.len[i] = cb->len[i];
+    // lengths up to the format's limit, codes that fit their length;
+    // the packer takes codes left-justified in 32 bits
+    const uint32_t L = cb->len[i];
+    if (L > DF11_MAX_CODE_LEN || (L < 32 && (cb->code[i] >> L) != 0)) return DF11_ERR_INVALID_ARG;
+    ecb.code[i] = L ? cb->code[i] << (32 - L) : 0u;
+    ecb.len[i] = (uint8_t)L;
   }
   const uint64_t C = cdiv(total_bits, 64);
   const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
@@ -1276,8 +1333,12 @@ extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
   if (st != DF11_OK) return st;
   EncCodebook ecb;
   for (int i = 0; i < 256; ++i) {
-    ecb.code[i] = cb->code[i];
-    ecb.len[i] = cb->len[i];
+    // lengths up to the format's limit, codes that fit their length;
+    // the packer takes codes left-justified in 32 bits
+    const uint32_t L = cb->len[i];
+    if (L > DF11_MAX_CODE_LEN || (L < 32 && (cb->code[i] >> L) != 0)) return DF11_ERR_INVALID_ARG;
+    ecb.code[i] = L ? cb->code[i] << (32 - L) : 0u;
+    ecb.len[i] = (uint8_t)L;
   }
   const uint64_t C = cdiv(total_bits, 64);
   const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
