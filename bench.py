@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-verify", action="store_true")
     ap.add_argument("--cap32", type=int, default=1, help="also time the block coded with cap 32")
+    ap.add_argument("--encode-steps", type=int, default=3,
+                    help="passes of the device-only encode timing (0: skip)")
     return ap.parse_args()
 
 
@@ -344,6 +346,13 @@ def run_df11(args):
         del cms32, abis32
 
     peak, peak_kind = measured_peak()
+    # ---- the encode path on the device alone (S2 histogram + S4 encode):
+    # the kernels of the 7 matrices back to back, codebooks already built,
+    # rewriting the same compressed buffers with the same bytes
+    encode = None
+    if args.encode_steps > 0:
+        encode = time_encode(torch, df11, cms, ws, dev, args.encode_steps, peak, peak_kind)
+
     avg_launch_ms = statistics.mean(per_launch_ms)
     achieved = algo_bytes / (avg_launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -371,8 +380,11 @@ def run_df11(args):
                        "parallelism": f"replica per GPU x{world}"},
             "weights_per_s": n_total * world * args.steps / (total_ms / 1e3),
             "ratio": ratio, "bits_per_weight": 16 * ratio, "bit_exact": bit_exact,
-            "compress": {"gpu_ms": compress_ms, "wall_s": compress_wall,
-                         "input_GBps": 2 * n_total / (compress_ms / 1e3) / 1e9},
+            "compress": {"ms": compress_ms, "wall_s": compress_wall,
+                         "input_GBps": 2 * n_total / (compress_ms / 1e3) / 1e9,
+                         "includes": "per matrix: histogram, its copy to the host, the host "
+                                     "codebook and tables, encode"},
+            "encode": encode,
             "code_len_cap": CAP,
             "max_code_len": max(int(m.codebook.max_len) for m in cms),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "cap32": cap32,
@@ -383,6 +395,48 @@ def run_df11(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def time_encode(torch, df11, cms, ws, dev, steps, peak, peak_kind):
+    """Device time of df11_histogram + df11_encode over the block's matrices
+    (6 kernel launches per matrix), averaged over `steps` passes after one
+    warm-up pass."""
+    stream = torch.cuda.Stream(device=dev)
+    sh = int(stream.cuda_stream)
+    hist = torch.empty(256, dtype=torch.int64, device=dev)
+    wsb = torch.empty(max(16, max(int(m.sizes.workspace_bytes) for m in cms)), dtype=torch.uint8,
+                      device=dev)
+    status = torch.zeros(2, dtype=torch.int32, device=dev)
+    outs = [df11.df11_encoded(stream=m.stream.data_ptr(), gaps=m.gaps.data_ptr(),
+                              block_pos=m.block_pos.data_ptr(),
+                              sign_mantissa=m.sign_mantissa.data_ptr(),
+                              block_max=status.data_ptr() + 4) for m in cms]
+
+    def one_pass():
+        for m, w, o in zip(cms, ws, outs):
+            n = w.numel()
+            df11.check(df11.df11_histogram(w.data_ptr(), n, hist.data_ptr(), sh), "df11_histogram")
+            df11.check(df11.df11_encode(w.data_ptr(), n, m.codebook, m.total_bits, o, wsb.data_ptr(),
+                                        wsb.numel(), status.data_ptr(), sh), "df11_encode")
+
+    one_pass()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one_pass()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if int(status[0].item()) != 0:
+        raise df11.DF11Error(int(status[0].item()), "encode (device)")
+    ms = e0.elapsed_time(e1) / steps
+    n_total = sum(w.numel() for w in ws)
+    algo = 2 * n_total + sum(int(m.stored_bytes) for m in cms)  # input read once + output written
+    return {"ms": ms, "input_GBps": 2 * n_total / (ms / 1e3) / 1e9, "launches": 6 * len(cms),
+            "roofline": {"bound": "hbm", "achieved": algo / (ms / 1e3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": algo / (ms / 1e3) / 1e9 / peak,
+                         "peak_kind": peak_kind, "algorithmic_bytes": algo},
+            "note": "histogram + encode kernels back to back, codebooks built beforehand"}
 
 
 def end_to_end(torch, df11, codec, cms, xs, dev, steps, dist, world):
