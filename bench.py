@@ -22,6 +22,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -91,14 +92,16 @@ DECODE_END = "// ============================================================ la
 
 
 def kernel_hash() -> str:
-    """Fingerprint of the decode kernel's source (the decode section of
-    df11_kernels.cu), so that a stored traffic figure is used only for the
-    kernel it was measured on."""
+    """Fingerprint of the decode kernel's code (the decode section of
+    df11_kernels.cu without comments), so that a stored traffic figure is
+    used only for the kernel it was measured on."""
     with open(KERNEL_SOURCE, encoding="utf-8") as f:
         src = f.read()
     a, b = src.find(DECODE_BEGIN), src.find(DECODE_END)
     section = src[a:b] if 0 <= a < b else src
-    return hashlib.sha256(section.encode()).hexdigest()[:16]
+    # the code alone: line comments and whitespace do not change the kernel
+    code = " ".join(re.sub(r"//[^\n]*", "", section).split())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def profiled_traffic(workload_name: str):

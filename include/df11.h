@@ -53,8 +53,8 @@
 extern "C" {
 #endif
 
-#define DF11_CHUNK_BITS 64u        /* [Kernel]: one thread per n = 8 bytes      */
-#define DF11_BLOCK_CHUNKS 256u     /* chunks (threads) per block of positions   */
+#define DF11_CHUNK_BITS 64u        /* [Kernel]: the page's per-thread n = 8 bytes */
+#define DF11_BLOCK_CHUNKS 256u     /* chunks per block of output positions      */
 #define DF11_GAP_BITS 5u           /* [Kernel]: gaps in [0,31], 5 bits each      */
 #define DF11_MAX_CODE_LEN 32u      /* [Kernel]/[LUT]: longest code, 32 bits      */
 #define DF11_MAX_N 0xFFFFFFFFull   /* [Kernel]: 32-bit block output positions    */

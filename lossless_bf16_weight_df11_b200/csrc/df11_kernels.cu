@@ -19,12 +19,17 @@
 //   enc_scan_kernel     exclusive prefix sum of the tile sums (bit offsets)
 //   enc_pack_kernel     packs codes MSB-first, writes gaps, block positions
 //                       and the sign/mantissa plane
-//   decode_kernel       persistent CTAs over the (matrix, block) list of a
-//                       batch; each block of 256 chunks is fetched with bulk
-//                       copies (TMA, no multicast) one block ahead, decoded
-//                       with a 12-bit shared-memory table, placed by a CTA
-//                       prefix sum of per-chunk code counts, merged with the
-//                       sign/mantissa bytes and stored as 16-byte BF16 rows
+//   enc_block_max_kernel  most codes starting in one block (sizes the
+//                       decoder's staging)
+//   decode_kernel       persistent CTAs over the (matrix, unit) list of a
+//                       batch; a unit is two blocks of 256 chunks, fetched
+//                       with bulk copies (TMA, no multicast) one unit ahead;
+//                       each thread decodes two consecutive chunks with a
+//                       12-bit shared-memory table into warp-interleaved
+//                       private rows; a CTA prefix sum of the per-thread
+//                       code counts places the exponents, which are merged
+//                       with the sign/mantissa bytes and stored as 16-byte
+//                       BF16 rows
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -543,11 +548,9 @@ inline bool smem_layout_aligned(const SmemLayout &S) {
   return ((S.stage0 | S.stage1 | S.sm | S.linear | S.priv | S.bars | S.meta | S.warp) & 15u) == 0;
 }
 
-// Per-thread private region: the codes that can start in a thread's two
-// chunks (ceil(128/min_len)), two codes of overshoot from the last table
-// entry, and the two spare bytes that entry's unconditional three-byte store
-// may touch; an odd number of 32-bit words so that word j of all 32 lanes of
-// a warp falls in 32 different banks.
+// Per-thread private region, in 32-bit rows: the codes that can start in a
+// thread's two chunks (ceil(128/min_len)), two codes of overshoot from the
+// last table entry, and two spare bytes; rounded to an odd number of rows.
 __host__ __device__ constexpr uint32_t region_words_even(uint32_t min_len) {
   return ((64 * kCPT + min_len - 1) / min_len + 4 + 3) / 4;
 }
