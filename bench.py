@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--cap32", type=int, default=1, help="also time the block coded with cap 32")
     ap.add_argument("--encode-steps", type=int, default=3,
                     help="passes of the device-only encode timing (0: skip)")
+    ap.add_argument("--matmul-steps", type=int, default=10,
+                    help="steps of the fused decode -> matmul timing (0: skip)")
     return ap.parse_args()
 
 
@@ -355,6 +357,13 @@ def run_df11(args):
     encode = None
     if args.encode_steps > 0:
         encode = time_encode(torch, df11, cms, ws, dev, args.encode_steps, peak, peak_kind)
+    # ---- fused decode -> matmul (y = x W^T, W never materialised) beside
+    # decode followed by a cuBLAS matmul, and the matmul alone on resident
+    # BF16 weights
+    fused = None
+    if args.matmul_steps > 0:
+        fused = [time_fused_matmul(torch, df11, cms, abis, outs, out_ptrs, status, xs_shapes(mats_def),
+                                   dev, b, args.matmul_steps, peak, peak_kind) for b in (1, 8)]
 
     avg_launch_ms = statistics.mean(per_launch_ms)
     achieved = algo_bytes / (avg_launch_ms / 1e3) / 1e9
@@ -388,6 +397,7 @@ def run_df11(args):
                          "includes": "per matrix: histogram, its copy to the host, the host "
                                      "codebook and tables, encode"},
             "encode": encode,
+            "fused_matmul": fused,
             "code_len_cap": CAP,
             "max_code_len": max(int(m.codebook.max_len) for m in cms),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "cap32": cap32,
@@ -440,6 +450,76 @@ def time_encode(torch, df11, cms, ws, dev, steps, peak, peak_kind):
                          "unit": "GB/s", "frac": algo / (ms / 1e3) / 1e9 / peak,
                          "peak_kind": peak_kind, "algorithmic_bytes": algo},
             "note": "histogram + encode kernels back to back, codebooks built beforehand"}
+
+
+def xs_shapes(mats_def):
+    return [tuple(shape) for _, shape in mats_def]
+
+
+def time_fused_matmul(torch, df11, cms, abis, outs, out_ptrs, status, shapes, dev, batch, steps,
+                      peak, peak_kind):
+    """Per step, for all matrices W_i (rows x cols) of the block and BF16
+    activations x_i (batch x cols): y_i += x_i W_i^T.  Three ways: the fused
+    kernel (one launch); decode into BF16 then torch.matmul (cuBLAS); the
+    matmul alone with the BF16 weights already resident."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + batch)
+    xs = [torch.randn(batch, c, generator=g, device=dev).to(torch.bfloat16) for _, c in shapes]
+    ys = [torch.zeros(batch, r, dtype=torch.float32, device=dev) for r, _ in shapes]
+    ios = [df11.df11_matmul_io(rows=r, cols=c, x=x.data_ptr(), y=y.data_ptr())
+           for (r, c), x, y in zip(shapes, xs, ys)]
+    stream = torch.cuda.current_stream(dev)
+    sh = int(stream.cuda_stream)
+    ws_bf16 = [o.view(r, c) for o, (r, c) in zip(outs, shapes)]
+
+    def fused():
+        df11.check(df11.df11_decode_matmul_batch(abis, ios, batch, status.data_ptr(), sh),
+                   "df11_decode_matmul_batch")
+
+    def decode_then_matmul():
+        df11.check(df11.df11_decode_block_batch(abis, out_ptrs, status.data_ptr(), sh),
+                   "df11_decode_block_batch")
+        for x, w, y in zip(xs, ws_bf16, ys):
+            y.add_(torch.matmul(x, w.t()).float())
+
+    def matmul_only():
+        for x, w, y in zip(xs, ws_bf16, ys):
+            y.add_(torch.matmul(x, w.t()).float())
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    t_fused = timed(fused)
+    # agreement with the unfused path on one step (FP32 sums in another order)
+    for y in ys:
+        y.zero_()
+    fused()
+    ref = [torch.matmul(x.double(), w.double().t()) for x, w in zip(xs, ws_bf16)]
+    bound_ok = all(bool(((y.double() - r).abs() <= (x.double().abs() @ w.double().abs().t())
+                         * (w.shape[1] + 8) * 2.0 ** -24 * 1.01).all())
+                   for x, w, y, r in zip(xs, ws_bf16, ys, ref))
+    del ref
+    t_unfused = timed(decode_then_matmul)
+    t_mm = timed(matmul_only)
+    if int(status.item()) != 0:
+        raise df11.DF11Error(int(status.item()), "fused matmul (device)")
+    algo = (sum(m.read_bytes for m in cms) + sum(2 * x.numel() for x in xs)
+            + sum(8 * y.numel() for y in ys))  # compressed W, x, y read and written
+    return {"batch": batch, "fused_ms": t_fused, "decode_then_matmul_ms": t_unfused,
+            "matmul_only_ms": t_mm, "speedup_vs_decode_then_matmul": t_unfused / t_fused,
+            "within_fp32_sum_bound": bound_ok,
+            "roofline": {"bound": "hbm", "achieved": algo / (t_fused / 1e3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": algo / (t_fused / 1e3) / 1e9 / peak,
+                         "peak_kind": peak_kind, "algorithmic_bytes": algo}}
 
 
 def end_to_end(torch, df11, codec, cms, xs, dev, steps, dist, world):

@@ -239,6 +239,42 @@ df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
                                     uint16_t *const *d_outs, uint32_t *d_status,
                                     df11_stream_t stream);
 
+/* Activations and sums of one matrix for df11_decode_matmul_batch.  The
+ * matrix W holds rows x cols values in row-major order (the order it was
+ * compressed in): rows output features, cols input features. */
+#define DF11_MATMUL_MAX_BATCH 8u    /* activation rows per fused launch          */
+#define DF11_MATMUL_MIN_COLS 256u   /* cols: a multiple of 8, at least this      */
+typedef struct {
+  uint32_t rows, cols;
+  const uint16_t *x;  /* device: batch x cols BF16 activations, row-major,
+                         16-byte aligned                                     */
+  float *y;           /* device: batch x rows FP32; the products are ADDED
+                         (zero it first for y = x W^T), 4-byte aligned      */
+} df11_matmul_io;
+
+/*
+ * df11_decode_matmul_batch -- for every matrix W of the batch,
+ *   y[j][r] += sum_c W[r][c] * x[j][c]   (j < batch),
+ * with W decoded on the fly and never written to device memory.  [GPU]: the
+ * BF16 weights are decompressed right before the matmul that uses them and
+ * discarded after; here the decode and the small-batch matmul are one kernel
+ * (batch 1..DF11_MATMUL_MAX_BATCH, the memory-bound inference case).  The
+ * format has no counterpart; this entry point adds no metadata.
+ *   ms, io   host arrays of count matrices and their activations and sums
+ *   batch    activation rows, 1..DF11_MATMUL_MAX_BATCH
+ *   d_status as for df11_decode (corrupt metadata: DF11_ERR_CORRUPT, the
+ *            offending units contribute nothing)
+ * Products are accumulated in FP32: exact BF16 x BF16 products summed in an
+ * unspecified order (a row is split over several CTAs and combined with
+ * atomic adds), so sums may differ in the last bits from run to run.
+ * Errors: DF11_ERR_INVALID_ARG for rows * cols != n, cols not a multiple of 8
+ * or below DF11_MATMUL_MIN_COLS, batch out of range, misaligned pointers;
+ * otherwise as df11_decode_block_batch.
+ */
+df11_status df11_decode_matmul_batch(const df11_matrix *ms, const df11_matmul_io *io,
+                                     uint32_t count, uint32_t batch, uint32_t *d_status,
+                                     df11_stream_t stream);
+
 /*
  * df11_validate -- host.  Checks stored metadata before it is trusted:
  * sizes derived from n and total_bits, every gap <= 31 and below its chunk's

@@ -67,6 +67,11 @@ class df11_encoded(ctypes.Structure):
                 ("block_max", ctypes.c_void_p)]
 
 
+class df11_matmul_io(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_uint32), ("cols", ctypes.c_uint32),
+                ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
 class DF11Error(RuntimeError):
     def __init__(self, status: int, where: str = ""):
         self.status = status
@@ -99,6 +104,9 @@ def _declare(lib):
         "df11_validate": (ctypes.c_int, [_u64, _u64, _u32, _vp, _u64, _vp, _u64]),
         "df11_encode_static_ws": (ctypes.c_int, [_vp, _u64, ctypes.POINTER(df11_codebook), _u64,
                                                  ctypes.POINTER(df11_encoded), _vp, _vp]),
+        "df11_decode_matmul_batch": (ctypes.c_int, [ctypes.POINTER(df11_matrix),
+                                                    ctypes.POINTER(df11_matmul_io), _u32, _u32,
+                                                    _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -183,6 +191,18 @@ def df11_decode_block_batch(ms, d_outs, d_status: int, stream: int = 0) -> int:
     arr = (df11_matrix * len(ms))(*ms)
     outs = (ctypes.c_void_p * len(d_outs))(*[int(p) for p in d_outs])
     return load().df11_decode_block_batch(arr, len(ms), outs, d_status, stream)
+
+
+MATMUL_MAX_BATCH = 8      # DF11_MATMUL_MAX_BATCH
+MATMUL_MIN_COLS = 256     # DF11_MATMUL_MIN_COLS
+
+
+def df11_decode_matmul_batch(ms, ios, batch: int, d_status: int, stream: int = 0) -> int:
+    """y += x W^T for each (matrix, io) pair with W decoded on the fly; see
+    include/df11.h."""
+    arr = (df11_matrix * len(ms))(*ms)
+    io = (df11_matmul_io * len(ios))(*ios)
+    return load().df11_decode_matmul_batch(arr, io, len(ms), batch, d_status, stream)
 
 
 def df11_validate(n: int, total_bits: int, min_len: int, h_gaps: int, gaps_bytes: int,

@@ -19,7 +19,8 @@ import numpy as np
 import torch
 
 from . import (MAX_CODE_LEN, TABLE_BITS, DF11Error, check, df11_build_codebook, df11_build_tables,
-               df11_codebook, df11_decode, df11_decode_block_batch, df11_encode, df11_encoded,
+               df11_codebook, df11_decode, df11_decode_block_batch, df11_decode_matmul_batch,
+               df11_encode, df11_encoded, df11_matmul_io,
                df11_encoded_sizes, df11_histogram, df11_matrix, df11_sizes, df11_tables_bytes)
 
 
@@ -190,6 +191,35 @@ def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=N
         if s:
             raise DF11Error(s, "df11_decode_block_batch (device)")
     return outs
+
+
+def matmul_block(ms, xs, ys=None, status: torch.Tensor | None = None, stream=None):
+    """y_i = x_i W_i^T for every matrix W_i of a block (each of shape
+    rows x cols, as compressed), decoded on the fly in one launch: the BF16
+    weights never reach device memory.  xs: BF16 tensors of shape
+    (batch, cols_i), batch <= MATMUL_MAX_BATCH; ys: FP32 tensors of shape
+    (batch, rows_i), zeroed here when not given (the products are added)."""
+    dev = ms[0].stream.device
+    batch = int(xs[0].shape[0])
+    for m, x in zip(ms, xs):
+        if len(m.shape) != 2 or x.dtype != torch.bfloat16 or x.shape != (batch, m.shape[1]):
+            raise ValueError("matmul_block: x must be BF16 (batch, cols) for a rows x cols matrix")
+    xs = [x.contiguous() for x in xs]
+    if ys is None:
+        ys = [torch.zeros(batch, m.shape[0], dtype=torch.float32, device=dev) for m in ms]
+    ios = [df11_matmul_io(rows=m.shape[0], cols=m.shape[1], x=x.data_ptr(), y=y.data_ptr())
+           for m, x, y in zip(ms, xs, ys)]
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        check(df11_decode_matmul_batch([m.abi() for m in ms], ios, batch, status.data_ptr(),
+                                       _stream_handle(stream)), "df11_decode_matmul_batch")
+    if own_status:
+        s = int(status.item())
+        if s:
+            raise DF11Error(s, "df11_decode_matmul_batch (device)")
+    return ys
 
 
 def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, stream, gaps,

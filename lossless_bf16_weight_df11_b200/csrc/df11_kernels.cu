@@ -499,6 +499,11 @@ struct DecMat {
   uint64_t total_bits;
   uint32_t n_chunks;  // C = ceil(total_bits / 64) (< 2^31 for n < 2^32)
   uint32_t n_blocks;  // B = ceil(C / 256); pos holds B + 1 entries
+  // fused matmul only: the matrix is rows x cols (row-major), x holds
+  // `batch` rows of cols BF16 activations, y `batch` rows of rows FP32 sums
+  uint32_t rows, cols;
+  const uint16_t *x;
+  float *y;
 };
 
 struct DecParams {
@@ -508,6 +513,7 @@ struct DecParams {
   uint32_t stage_cap;     // bytes: max codes per unit, rounded up to 16
   uint32_t region_bytes;  // private decode region per thread (odd number of words)
   uint32_t min_len;       // shortest code of the batch (regions are sized by it)
+  uint32_t batch;         // fused matmul: activation rows (<= the kernel's NB)
   uint32_t *status;
 };
 
@@ -517,7 +523,7 @@ constexpr uint32_t kStageBytes = kStreamStage + kGapStage + 16;
 static_assert(kStageBytes % 16 == 0 && sizeof(DecodeTables) % 16 == 0, "stage alignment");
 
 struct SmemLayout {
-  uint32_t tables, stage0, stage1, sm, linear, priv, bars, meta, warp, total;
+  uint32_t tables, stage0, stage1, sm, linear, priv, bars, meta, warp, acc, total;
 };
 
 // The linear row holds the unit's exponents from byte P0 % 8 on; the
@@ -529,7 +535,14 @@ struct SmemLayout {
 // writes (linear row), mbarriers (8 bytes).
 __host__ __device__ constexpr uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
-__host__ __device__ inline SmemLayout smem_layout(uint32_t cap, uint32_t region_bytes) {
+// Rows of the fused matmul's per-unit accumulators: a unit's outputs span at
+// most (cols - 8 + units's codes + 15) / cols + 1 rows; with cols >= 256 and
+// at most 32768 codes per unit that is below 136.
+constexpr uint32_t kAccRows = 136;
+constexpr uint32_t kMinMatmulCols = DF11_MATMUL_MIN_COLS;
+
+__host__ __device__ inline SmemLayout smem_layout(uint32_t cap, uint32_t region_bytes,
+                                                  uint32_t nb = 0) {
   SmemLayout S;
   S.tables = 0;
   S.stage0 = round16((uint32_t)sizeof(DecodeTables));
@@ -540,12 +553,14 @@ __host__ __device__ inline SmemLayout smem_layout(uint32_t cap, uint32_t region_
   S.bars = round16(S.priv + kT * region_bytes);
   S.meta = round16(S.bars + 32);
   S.warp = round16(S.meta + 2 * 32);
-  S.total = round16(S.warp + 16 * 4);
+  S.acc = round16(S.warp + 16 * 4);
+  S.total = round16(S.acc + 4 * kAccRows * nb);
   return S;
 }
 
 inline bool smem_layout_aligned(const SmemLayout &S) {
-  return ((S.stage0 | S.stage1 | S.sm | S.linear | S.priv | S.bars | S.meta | S.warp) & 15u) == 0;
+  return ((S.stage0 | S.stage1 | S.sm | S.linear | S.priv | S.bars | S.meta | S.warp | S.acc) &
+          15u) == 0;
 }
 
 // Per-thread private region, in 32-bit rows: the codes that can start in a
@@ -720,6 +735,8 @@ struct Pending {
   uint32_t P0, P1;
   uint16_t *out;
   bool ok;
+  uint32_t m;               // matrix of the batch
+  uint32_t row_lo, col_lo;  // fused matmul: row and column of output P0 & ~7
 };
 
 // Merge a decoded block: exponents in the linear row, sign/mantissa bytes in
@@ -765,12 +782,145 @@ __device__ __forceinline__ void merge_block(const Pending &q, uint32_t lin_a, ui
   }
 }
 
-// MAXW: 32-bit words of a thread's private region.
-template <int MAXW>
+// Fused matmul merge: the unit's decoded weights are multiplied with the
+// activations instead of being stored.  Lane l of warp w takes groups
+// w*32 + l, + 256, ... (8 weights each, flat index base8 + 8k, masked to
+// the unit's outputs); each group's dot products with the NB activation rows
+// are reduced over the warp per output row (32 consecutive groups span at
+// most two rows since cols >= 256) and added into the CTA's per-row
+// accumulators (row offsets from row_lo).  The staging row is cleared behind
+// the reads, as in the plain merge.
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t v, float &a, float &b) {
+  a = __uint_as_float(v << 16);
+  b = __uint_as_float(v & 0xFFFF0000u);
+}
+
+template <int NB>
+__device__ __forceinline__ void merge_block_matmul(const Pending &q, uint32_t lin_a, uint32_t sm_a,
+                                                   int t, float *acc, const DecMat &M,
+                                                   uint32_t batch) {
+  const int lane = t & 31, warp = t >> 5;
+  const uint32_t base8 = q.P0 & ~7u;
+  const uint32_t smb = sm_a + (base8 - (q.P0 & ~15u));
+  const uint32_t head = q.P0 & 7u;
+  const uint32_t span8 = q.P1 - base8;
+  const uint32_t ngroups = (span8 + 7) >> 3;
+  const uint32_t cols = M.cols;
+  // the activations of a group: its 8 columns of each of the batch rows
+  // (rows past the batch read as zero)
+  auto load_x = [&](uint32_t k, uint32_t col, uint4 (&xv)[NB]) {
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+      xv[j] = (k < ngroups && (uint32_t)j < batch)
+                  ? __ldg(reinterpret_cast<const uint4 *>(M.x + (size_t)j * cols + col))
+                  : make_uint4(0u, 0u, 0u, 0u);
+  };
+  // row offset and column of this lane's first group
+  uint32_t col = q.col_lo + 8u * (uint32_t)(warp * 32 + lane), row = 0;
+  while (col >= cols) {
+    col -= cols;
+    ++row;
+  }
+  // with one or two activation rows the next group's activations are
+  // requested before this group is merged (their latency is otherwise
+  // exposed once per group); with more, the registers are not spared
+  constexpr bool kPrefetch = NB <= 2;
+  uint4 xn[NB];
+  if (kPrefetch) load_x((uint32_t)warp * 32 + lane, col, xn);
+  for (uint32_t kb = (uint32_t)warp * 32; kb < ngroups; kb += kT) {
+    const uint32_t k = kb + lane;
+    uint32_t ncol = col + 8u * kT, nrow = row;
+    while (ncol >= cols) {
+      ncol -= cols;
+      ++nrow;
+    }
+    uint4 xv[NB];
+    if (kPrefetch) {
+#pragma unroll
+      for (int j = 0; j < NB; ++j) xv[j] = xn[j];
+      load_x(k + kT, ncol, xn);
+    } else {
+      load_x(k, col, xv);
+    }
+    float d[NB];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) d[j] = 0.f;
+    if (k < ngroups) {
+      uint4 r;
+      merge_group(lin_a, smb, k, r);
+      float w[8];
+      bf16x2_to_f32(r.x, w[0], w[1]);
+      bf16x2_to_f32(r.y, w[2], w[3]);
+      bf16x2_to_f32(r.z, w[4], w[5]);
+      bf16x2_to_f32(r.w, w[6], w[7]);
+      const uint32_t lo = k == 0 ? head : 0u, hi = min(8u, span8 - 8 * k);
+      if (lo != 0 || hi != 8) {
+        // the unit's ragged first or last group: weights outside it are zero
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = ((uint32_t)i >= lo && (uint32_t)i < hi) ? w[i] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        float xf[8];
+        bf16x2_to_f32(xv[j].x, xf[0], xf[1]);
+        bf16x2_to_f32(xv[j].y, xf[2], xf[3]);
+        bf16x2_to_f32(xv[j].z, xf[4], xf[5]);
+        bf16x2_to_f32(xv[j].w, xf[6], xf[7]);
+        float sdot = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sdot = fmaf(w[i], xf[i], sdot);
+        d[j] = sdot;
+      }
+    }
+    // per-row sums over the warp: lane 0's row and the next
+    const uint32_t row0 = __shfl_sync(0xffffffffu, row, 0);
+    const bool second = __any_sync(0xffffffffu, k < ngroups && row != row0);
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      float a = row == row0 ? d[j] : 0.f;
+      float b = d[j] - a;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+      }
+      if (lane == 0 && (uint32_t)j < batch) {
+        if (row0 < kAccRows) atomicAdd(acc + j * kAccRows + row0, a);
+        if (second && row0 + 1 < kAccRows) atomicAdd(acc + j * kAccRows + row0 + 1, b);
+      }
+    }
+    col = ncol;
+    row = nrow;
+  }
+}
+
+// Add a merged unit's row sums to y and clear the accumulators (after a CTA
+// barrier that follows the merge).
+template <int NB>
+__device__ __forceinline__ void flush_matmul(const Pending &q, float *acc, const DecMat &M,
+                                             uint32_t batch, int t) {
+  const uint32_t base8 = q.P0 & ~7u;
+  const uint32_t nrows = min((q.col_lo + (q.P1 - base8) - 1) / M.cols + 1, kAccRows);
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    for (uint32_t r = t; r < nrows; r += kT) {
+      const float v = acc[j * kAccRows + r];
+      if ((uint32_t)j < batch && v != 0.f && q.row_lo + r < M.rows)
+        atomicAdd(M.y + (size_t)j * M.rows + q.row_lo + r, v);
+      acc[j * kAccRows + r] = 0.f;
+    }
+  }
+}
+
+// MAXW: 32-bit words of a thread's private region.  NB: 0 for the plain
+// decode (BF16 stored to out); 1, 2, 4 or 8 for the fused matmul with up to
+// NB activation rows (P.batch of them used).
+template <int MAXW, int NB>
 __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ DecParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t cap = P.stage_cap;
-  const SmemLayout S = smem_layout(cap, 4 * MAXW);
+  const SmemLayout S = smem_layout(cap, 4 * MAXW, NB);
+  float *acc = reinterpret_cast<float *>(smem + S.acc);  // [NB][kAccRows] row sums
   const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem + S.tables);
   const uint32_t sbase = smem_addr(smem);
   const uint32_t lut_a = sbase + S.tables;  // lut is the first member
@@ -808,6 +958,12 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
     meta[stage * 8 + 2] = m;
     meta[stage * 8 + 3] = u;
     meta[stage * 8 + 4] = pm;
+    if (NB > 0) {
+      // fused matmul: row and column of output p0 & ~7
+      const uint32_t base8 = p0 & ~7u;
+      meta[stage * 8 + 5] = base8 / M.cols;
+      meta[stage * 8 + 6] = base8 % M.cols;
+    }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_expect_tx(bar_stage + 8 * stage, sbytes + gbytes);
     bulk_g2s(st, M.stream + (uint64_t)u * (8 * kUnitChunks), sbytes, bar_stage + 8 * stage);
@@ -842,13 +998,16 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
 
   uint32_t cur_m = 0xFFFFFFFFu;
   bool table_ok = false, table_short = false;
-  Pending prev{0, 0, nullptr, false};
+  Pending prev{0, 0, nullptr, false, 0, 0, 0};
+  if constexpr (NB > 0)
+    for (uint32_t k = t; k < NB * kAccRows; k += kT) acc[k] = 0.f;
   for (uint64_t g = g0, it = 0; g < g1; ++g, ++it) {
     const uint32_t s = (uint32_t)(it & 1);
     // [A] the previous unit is relocated into the linear row
     if (it) __syncthreads();
     const uint32_t *mt = meta + s * 8;
     const uint32_t P0 = mt[0], P1 = mt[1], m = mt[2], u = mt[3], PM = mt[4];
+    const uint32_t RL = NB > 0 ? mt[5] : 0u, CL = NB > 0 ? mt[6] : 0u;
     const DecMat &M = P.m[m];
     // positions are trusted only as far as they stay inside the matrix and
     // the staging row; anything else is flagged as corrupt after the count
@@ -970,7 +1129,10 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
     // so that the barrier is never re-armed with a copy in flight
     if (it) {
       if (!mbar_wait(bar_sm, (uint32_t)((it - 1) & 1))) timed_out = true;
-      else if (prev.ok) merge_block(prev, lin_a, sm_a, t);
+      else if (prev.ok) {
+        if constexpr (NB == 0) merge_block(prev, lin_a, sm_a, t);
+        else merge_block_matmul<NB>(prev, lin_a, sm_a, t, acc, P.m[prev.m], P.batch);
+      }
     }
     // ---- [B] CTA prefix sum of the counts
     uint32_t incl = cnt;
@@ -1010,6 +1172,10 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
     // block positions (every stored position is checked)
     const bool ok =
         table_ok && sane && !(flagbits >> 31) && tot == P1 - P0 && tot_first == PM - P0;
+    // fused matmul: the previous unit's row sums (merged before the barrier)
+    if constexpr (NB > 0) {
+      if (it && prev.ok) flush_matmul<NB>(prev, acc, P.m[prev.m], P.batch, t);
+    }
     if (t == 0) {
       if (!ok) set_status(P.status, DF11_ERR_CORRUPT);
       // this unit's sign/mantissa bytes (the previous unit's merge is done),
@@ -1045,14 +1211,18 @@ __global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ D
         for (int k = 0; k < MAXW; ++k) sts32(col_a + 128 * k, 0u);
       }
     }
-    prev = Pending{P0, P1, M.out, ok};
+    prev = Pending{P0, P1, M.out, ok, m, RL, CL};
   }
   // the last unit's merge
   __syncthreads();
-  if (!mbar_wait(bar_sm, (uint32_t)((g1 - g0 - 1) & 1))) {
-    if (lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
-  } else if (prev.ok) {
-    merge_block(prev, lin_a, sm_a, t);
+  const bool got = mbar_wait(bar_sm, (uint32_t)((g1 - g0 - 1) & 1));
+  if (!got && lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
+  if constexpr (NB == 0) {
+    if (got && prev.ok) merge_block(prev, lin_a, sm_a, t);
+  } else {
+    if (got && prev.ok) merge_block_matmul<NB>(prev, lin_a, sm_a, t, acc, P.m[prev.m], P.batch);
+    __syncthreads();
+    if (got && prev.ok) flush_matmul<NB>(prev, acc, P.m[prev.m], P.batch, t);
   }
 }
 
@@ -1067,6 +1237,20 @@ constexpr int kMaxWords2 = 17;  // region_bytes_for(2) / 4
 constexpr int kMaxWords1 = 33;  // region_bytes_for(1) / 4
 static_assert(region_bytes_for(2) == 4 * kMaxWords2 && region_bytes_for(1) == 4 * kMaxWords1,
               "private region sizes");
+
+using DecodeKernel = void (*)(DecParams);
+
+// The instantiation for a batch: regions for codes of >= 2 bits or of 1 bit
+// (wide), and the epilogue (0: store BF16; NB: matmul with up to NB rows).
+DecodeKernel decode_kernel_for(bool wide, uint32_t nb) {
+  switch (nb) {
+    case 0: return wide ? decode_kernel<kMaxWords1, 0> : decode_kernel<kMaxWords2, 0>;
+    case 1: return wide ? decode_kernel<kMaxWords1, 1> : decode_kernel<kMaxWords2, 1>;
+    case 2: return wide ? decode_kernel<kMaxWords1, 2> : decode_kernel<kMaxWords2, 2>;
+    case 4: return wide ? decode_kernel<kMaxWords1, 4> : decode_kernel<kMaxWords2, 4>;
+    default: return wide ? decode_kernel<kMaxWords1, 8> : decode_kernel<kMaxWords2, 8>;
+  }
+}
 
 struct DeviceInfo {
   int sms = 0;
@@ -1090,13 +1274,13 @@ df11_status device_info(int *dev, int *sms) {
     if (cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kHistSmem) != cudaSuccess)
       return DF11_ERR_CUDA;
-    // the largest staging: a unit of codes of one bit
-    const int max_smem = (int)smem_layout(64 * kCPT * kT, region_bytes_for(1)).total;
-    if (cudaFuncSetAttribute(decode_kernel<kMaxWords2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             max_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(decode_kernel<kMaxWords1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             max_smem) != cudaSuccess)
-      return DF11_ERR_CUDA;
+    // the largest staging: a unit of codes of one bit, 8 activation rows
+    const int max_smem = (int)smem_layout(64 * kCPT * kT, region_bytes_for(1), 8).total;
+    for (int wide = 0; wide < 2; ++wide)
+      for (uint32_t nb : {0u, 1u, 2u, 4u, 8u})
+        if (cudaFuncSetAttribute(decode_kernel_for(wide != 0, nb),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) != cudaSuccess)
+          return DF11_ERR_CUDA;
     d.configured = true;
   }
   *sms = d.sms;
@@ -1185,11 +1369,17 @@ extern "C" df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_c
   return launch_status();
 }
 
-extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
-                                               uint16_t *const *d_outs, uint32_t *d_status,
-                                               df11_stream_t stream) {
+namespace {
+
+// Shared by df11_decode_block_batch (io == nullptr: BF16 stored to d_outs)
+// and df11_decode_matmul_batch (d_outs == nullptr: products added to io[i].y).
+df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const *d_outs,
+                          const df11_matmul_io *io, uint32_t batch, uint32_t *d_status,
+                          df11_stream_t stream) {
   if (count == 0) return DF11_OK;
-  if (!ms || !d_outs) return DF11_ERR_INVALID_ARG;
+  if (!ms || (!d_outs && !io)) return DF11_ERR_INVALID_ARG;
+  const uint32_t nb = io ? (batch <= 1 ? 1u : batch <= 2 ? 2u : batch <= 4 ? 4u : 8u) : 0u;
+  if (io && (batch < 1 || batch > DF11_MATMUL_MAX_BATCH)) return DF11_ERR_INVALID_ARG;
   int dev, sms;
   df11_status st = device_info(&dev, &sms);
   if (st != DF11_OK) return st;
@@ -1206,12 +1396,20 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
       const df11_matrix &m = ms[first + i];
       if (m.n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
       if (m.n == 0) continue;
-      if (!m.stream || !m.gaps || !m.block_pos || !m.sign_mantissa || !m.tables ||
-          !d_outs[first + i])
+      if (!m.stream || !m.gaps || !m.block_pos || !m.sign_mantissa || !m.tables)
         return DF11_ERR_INVALID_ARG;
       if (!aligned16(m.stream) || !aligned16(m.gaps) || !aligned16(m.sign_mantissa) ||
-          !aligned16(m.tables) || !aligned16(d_outs[first + i]) || ((uintptr_t)m.block_pos & 3u))
+          !aligned16(m.tables) || ((uintptr_t)m.block_pos & 3u))
         return DF11_ERR_INVALID_ARG;
+      if (io) {
+        // the matrix is rows x cols; activations and sums 16-byte aligned
+        const df11_matmul_io &q = io[first + i];
+        if ((uint64_t)q.rows * q.cols != m.n || q.cols % 8 || q.cols < kMinMatmulCols || !q.x ||
+            !q.y || !aligned16(q.x) || ((uintptr_t)q.y & 3u))
+          return DF11_ERR_INVALID_ARG;
+      } else if (!d_outs[first + i] || !aligned16(d_outs[first + i])) {
+        return DF11_ERR_INVALID_ARG;
+      }
       // a complete code over at most 256 values has a code of at most 8 bits
       if (m.min_len < 1 || m.min_len > 8) return DF11_ERR_INVALID_ARG;
       if (m.total_bits < m.n * (uint64_t)m.min_len || m.total_bits > m.n * 32ull)
@@ -1232,7 +1430,11 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
       d.pos = m.block_pos;
       d.sm = m.sign_mantissa;
       d.tables = reinterpret_cast<const DecodeTables *>(m.tables);
-      d.out = d_outs[first + i];
+      d.out = io ? nullptr : d_outs[first + i];
+      d.rows = io ? io[first + i].rows : 0u;
+      d.cols = io ? io[first + i].cols : 1u;
+      d.x = io ? io[first + i].x : nullptr;
+      d.y = io ? io[first + i].y : nullptr;
       d.n = m.n;
       d.total_bits = m.total_bits;
       d.n_chunks = (uint32_t)C;
@@ -1246,10 +1448,11 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
     P.stage_cap = (unit_codes + 15u) & ~15u;
     P.region_bytes = 4u * (min_len >= 2 ? kMaxWords2 : kMaxWords1);
     P.min_len = min_len;
-    const SmemLayout L = smem_layout(P.stage_cap, P.region_bytes);
+    P.batch = io ? batch : 0u;
+    const SmemLayout L = smem_layout(P.stage_cap, P.region_bytes, nb);
     if (!smem_layout_aligned(L)) return DF11_ERR_INVALID_ARG;
     const uint32_t smem = L.total;
-    auto kern = min_len >= 2 ? decode_kernel<kMaxWords2> : decode_kernel<kMaxWords1>;
+    const DecodeKernel kern = decode_kernel_for(min_len < 2, nb);
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kT, smem) != cudaSuccess)
       return DF11_ERR_CUDA;
@@ -1261,6 +1464,22 @@ extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t c
     if (st != DF11_OK) return st;
   }
   return DF11_OK;
+}
+
+}  // namespace
+
+extern "C" df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
+                                               uint16_t *const *d_outs, uint32_t *d_status,
+                                               df11_stream_t stream) {
+  if (count && !d_outs) return DF11_ERR_INVALID_ARG;
+  return launch_decode(ms, count, d_outs, nullptr, 0, d_status, stream);
+}
+
+extern "C" df11_status df11_decode_matmul_batch(const df11_matrix *ms, const df11_matmul_io *io,
+                                                uint32_t count, uint32_t batch, uint32_t *d_status,
+                                                df11_stream_t stream) {
+  if (count && !io) return DF11_ERR_INVALID_ARG;
+  return launch_decode(ms, count, nullptr, io, batch, d_status, stream);
 }
 
 extern "C" df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32_t *d_status,
