@@ -58,6 +58,8 @@ def parse():
                     help="passes of the device-only encode timing (0: skip)")
     ap.add_argument("--matmul-steps", type=int, default=10,
                     help="steps of the fused decode -> matmul timing (0: skip)")
+    ap.add_argument("--block-steps", type=int, default=5,
+                    help="steps of the DF11 transformer-block forward timing (0: skip)")
     return ap.parse_args()
 
 
@@ -260,6 +262,18 @@ def run_df11(args):
     torch.cuda.synchronize()
     compress_ms = ev0.elapsed_time(ev1)
     compress_wall = time.perf_counter() - comp_t0
+    # the batched compressor (two host round trips for the whole block)
+    codec.compress_block([ws[0][:65536], ws[1][:65536]], cap=CAP)
+    torch.cuda.synchronize()
+    eb0, eb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    eb0.record()
+    cms_b = codec.compress_block(ws, cap=CAP)
+    eb1.record()
+    torch.cuda.synchronize()
+    compress_block_ms = eb0.elapsed_time(eb1)
+    same = all(int(a.total_bits) == int(b.total_bits) and torch.equal(a.stream, b.stream)
+               for a, b in zip(cms, cms_b))
+    del cms_b
     read_bytes = sum(m.read_bytes for m in cms)
     stored = sum(m.stored_bytes for m in cms)
     ratio = stored / (2 * n_total)
@@ -360,6 +374,11 @@ def run_df11(args):
     # ---- fused decode -> matmul (y = x W^T, W never materialised) beside
     # decode followed by a cuBLAS matmul, and the matmul alone on resident
     # BF16 weights
+    # ---- a whole transformer block held in DF11 form: decode (one launch)
+    # then the block's forward, beside the same forward on resident weights
+    blockfw = None
+    if args.block_steps > 0 and wid in BLOCK_SHAPES:
+        blockfw = time_block_forward(torch, cms, ws, mats_def, wid, dev, args.block_steps)
     fused = None
     if args.matmul_steps > 0:
         fused = [time_fused_matmul(torch, df11, cms, abis, outs, out_ptrs, status, xs_shapes(mats_def),
@@ -396,8 +415,14 @@ def run_df11(args):
                          "input_GBps": 2 * n_total / (compress_ms / 1e3) / 1e9,
                          "includes": "per matrix: histogram, its copy to the host, the host "
                                      "codebook and tables, encode"},
+            "compress_block": {"ms": compress_block_ms,
+                               "input_GBps": 2 * n_total / (compress_block_ms / 1e3) / 1e9,
+                               "same_as_per_matrix": same,
+                               "includes": "all histograms, one copy to the host, host codebooks "
+                                           "and tables, all encodes, one copy of the status words"},
             "encode": encode,
             "fused_matmul": fused,
+            "block_forward": blockfw,
             "code_len_cap": CAP,
             "max_code_len": max(int(m.codebook.max_len) for m in cms),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "cap32": cap32,
@@ -450,6 +475,46 @@ def time_encode(torch, df11, cms, ws, dev, steps, peak, peak_kind):
                          "unit": "GB/s", "frac": algo / (ms / 1e3) / 1e9 / peak,
                          "peak_kind": peak_kind, "algorithmic_bytes": algo},
             "note": "histogram + encode kernels back to back, codebooks built beforehand"}
+
+
+# (hidden, heads, kv_heads, ffn) of the block workloads
+BLOCK_SHAPES = {3: (4096, 32, 8, 14336), 5: (8192, 64, 8, 28672)}
+
+
+def time_block_forward(torch, cms, ws, mats_def, wid, dev, steps):
+    """DF11Block.forward (decode of the seven matrices + the block) against the
+    same forward on the resident BF16 weights, for 16 and 2048 tokens."""
+    import dataclasses
+    import lossless_bf16_weight_df11_b200.block as blockmod
+    shape = blockmod.BlockShape(*BLOCK_SHAPES[wid])
+    names = [nm for nm, _ in mats_def]
+    mats = {nm: dataclasses.replace(m, shape=tuple(sh)) for nm, m, (_, sh) in zip(names, cms, mats_def)}
+    wts = {nm: w.view(torch.bfloat16).reshape(sh) for nm, w, (_, sh) in zip(names, ws, mats_def)}
+    blk = blockmod.DF11Block(mats, shape)
+    g = torch.Generator(device=dev)
+    g.manual_seed(77)
+    out = []
+    for tokens in (16, 2048):
+        x = torch.randn(1, tokens, shape.hidden, generator=g, device=dev).to(torch.bfloat16)
+
+        def timed(fn):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / steps
+
+        same = bool(torch.equal(blk.forward(x), blk.forward_reference(x, wts)))
+        t_df11 = timed(lambda: blk.forward(x))
+        t_ref = timed(lambda: blk.forward_reference(x, wts))
+        out.append({"tokens": tokens, "df11_ms": t_df11, "bf16_resident_ms": t_ref,
+                    "decode_overhead_ms": t_df11 - t_ref, "bit_identical": same})
+    return out
 
 
 def xs_shapes(mats_def):

@@ -156,6 +156,64 @@ def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | 
                       max_block_codes=int(st_host[1]), **bufs)
 
 
+def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
+                   check_status: bool = True) -> list[DF11Matrix]:
+    """Compress several BF16 tensors (e.g. the matrices of a transformer block
+    or a whole model) with two host round trips in all: every histogram is
+    computed on the device, copied to the host at once, the codebooks and
+    decode tables are built on the host, and every encode is enqueued
+    before the status words come back in one copy.  The result is the same,
+    array for array, as compress() of each tensor."""
+    if not ws:
+        return []
+    us = [_as_u16(w) for w in ws]
+    dev = us[0].device
+    sh = _stream_handle(stream)
+    hists = torch.empty(len(us), 256, dtype=torch.int64, device=dev)
+    with torch.cuda.device(dev):
+        for i, u in enumerate(us):
+            check(df11_histogram(u.data_ptr(), u.numel(), hists[i].data_ptr(), sh), "df11_histogram")
+    h_all = hists.cpu().numpy().view(np.uint64).copy()  # round trip 1
+    # codebooks, sizes and decode tables on the host; the tables go up in
+    # one copy (the device is idle here: nothing is enqueued yet)
+    cbs, sizes_l = [], []
+    nt = df11_tables_bytes()
+    tables_host = np.zeros((len(us), nt), np.uint8)
+    for i, u in enumerate(us):
+        st, cb = df11_build_codebook(h_all[i], cap)
+        check(st, "df11_build_codebook")
+        st, sizes = df11_encoded_sizes(cb, h_all[i], u.numel())
+        check(st, "df11_encoded_sizes")
+        check(df11_build_tables(cb, tables_host[i].ctypes.data, nt), "df11_build_tables")
+        cbs.append(cb)
+        sizes_l.append(sizes)
+    tables = torch.from_numpy(tables_host).to(dev)
+    ws_bytes = max(16, max(int(sz.workspace_bytes) for sz in sizes_l))
+    wsb = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    status = torch.zeros(len(us), 2, dtype=torch.int32, device=dev)  # [status, most codes per block]
+    mats_bufs = []
+    with torch.cuda.device(dev):
+        for i, (u, cb, sizes) in enumerate(zip(us, cbs, sizes_l)):
+            bufs = alloc_encoded(sizes, dev)
+            out = df11_encoded(stream=bufs["stream"].data_ptr(), gaps=bufs["gaps"].data_ptr(),
+                               block_pos=bufs["block_pos"].data_ptr(),
+                               sign_mantissa=bufs["sign_mantissa"].data_ptr(),
+                               block_max=status[i].data_ptr() + 4)
+            check(df11_encode(u.data_ptr(), u.numel(), cb, sizes.total_bits, out, wsb.data_ptr(),
+                              wsb.numel(), status[i].data_ptr(), sh), "df11_encode")
+            mats_bufs.append(bufs)
+    st_host = status.cpu().numpy()  # round trip 2
+    mats = []
+    for i, (w, u) in enumerate(zip(ws, us)):
+        if check_status and int(st_host[i, 0]):
+            raise DF11Error(int(st_host[i, 0]), f"df11_encode (device), matrix {i}")
+        mats.append(DF11Matrix(shape=tuple(w.shape), n=u.numel(),
+                               total_bits=int(sizes_l[i].total_bits), codebook=cbs[i],
+                               sizes=sizes_l[i], tables=tables[i], hist=h_all[i],
+                               max_block_codes=int(st_host[i, 1]), **mats_bufs[i]))
+    return mats
+
+
 def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     dev = m.stream.device

@@ -189,3 +189,29 @@ def test_encode_reports_value_without_code(codec):
     x[77] = (missing[0] << 7) | 1
     with pytest.raises(df11.DF11Error):
         codec.compress(to_dev(x), codebook=cb)
+
+
+def test_compress_block_matches_compress(codec):
+    """The batched compressor (two host round trips for all matrices) gives,
+    array for array, what compress() gives matrix by matrix: the Llama-3-8B
+    block and a list of edge cases (empty, one value, a ragged tail, one
+    symbol)."""
+    import lossless_bf16_weight_df11_b200 as df11
+    cases = [[workloads.matrix(3, i) for i in range(len(workloads.WORKLOADS[3][1]))],
+             [workloads.random_bf16(0, seed=1), workloads.random_bf16(1, seed=2),
+              workloads.random_bf16(1_000_003, seed=3), workloads.constant(65_537, 0x3F80),
+              workloads.fibonacci_exponents(34)]]
+    for xs in cases:
+        ws = [to_dev(x) for x in xs]
+        got = codec.compress_block(ws)
+        for w, g in zip(ws, got):
+            m = codec.compress(w)
+            a, b = m.host_arrays(), g.host_arrays()
+            for key in ("lengths", "stream", "gaps", "block_pos", "sign_mantissa"):
+                assert np.array_equal(a[key], b[key]), key
+            assert m.total_bits == g.total_bits and m.max_block_codes == g.max_block_codes
+            assert torch.equal(m.tables, g.tables)
+        outs = codec.decompress_block([g for g in got if g.n])
+        for x, o in zip([x for x in xs if x.size], outs):
+            assert np.array_equal(bits_of(o), np.ascontiguousarray(x).reshape(-1))
+        del got
