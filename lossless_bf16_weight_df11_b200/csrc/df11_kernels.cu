@@ -346,6 +346,10 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
   uint32_t prev_len = lane ? up : (warp ? s_lastlen[warp - 1] : s_lc[(before >> 7) & 0xFFu].x);
   if (i0 == 0 || !nk) prev_len = 0;
   const uint32_t cb0 = (uint32_t)(S0 & 63u);  // S0's offset in its chunk
+  // Bounds of the shared indices below: codes are at most 32 bits (checked
+  // by the launcher), so the tile's bits E - S <= 4096 * 32 and every bit
+  // offset rel + off <= 31 + 131072: word index wi <= 4096 < kWords, chunk
+  // index pos / 64 <= 2049 < kGapChunks.
   uint32_t hi = 0, lo = 0;                 // the word being filled (word wi) and the next
   uint32_t nb = rel & 31u, wi = rel >> 5;  // bits of word wi already taken
   uint32_t off = 0;                        // bits of this thread's codes so far
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     lo |= __funnelshift_r(0u, lc.y, nb);  // the code's bits past word wi
     nb += L;
     const bool full = nb >= 32;
-    red_or_shared_if(&s_bits[wi < (uint32_t)kWords ? wi : 0u], hi, full && wi < (uint32_t)kWords);
+    red_or_shared_if(&s_bits[wi], hi, full);
     wi += full ? 1u : 0u;
     hi = full ? lo : hi;
     lo = full ? 0u : lo;
@@ -368,7 +372,7 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     // is below the previous code's length; the very first code starts both
     const uint32_t pos = cb0 + rel + off;  // bit offset from chunk S0/64
     if ((k == 0 && i0 == 0) || (pos & 63u) < prev_len) {
-      if ((pos >> 6) < (uint32_t)kGapChunks) s_gap[pos >> 6] = (uint8_t)(pos & 63u);
+      s_gap[pos >> 6] = (uint8_t)(pos & 63u);
       if ((k == 0 && i0 == 0) || (((uint32_t)start0 + off) & 16383u) < prev_len) {
         const uint64_t b = (start0 + off) >> 14;
         if (b < n_blocks) block_pos[b] = (uint32_t)(i0 + k);
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     last_len = L;
     off += L;
   }
-  if (nb && wi < (uint32_t)kWords) atomicOr(&s_bits[wi], hi);
+  if (nb) atomicOr(&s_bits[wi], hi);
   if (nk && i0 + nk == n) {
     // the last chunk / block may begin inside the final code: its gap points
     // at the end of the stream
