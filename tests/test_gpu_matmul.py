@@ -162,3 +162,14 @@ def test_rejects_bad_shapes(df11, codec):
     io = df11.df11_matmul_io(rows=258, cols=1002, x=xb.data_ptr(), y=y.data_ptr())
     assert df11.df11_decode_matmul_batch([m2.abi()], [io], 1, status.data_ptr(),
                                          stream) == df11.DF11_ERR_INVALID_ARG
+
+
+def test_more_matrices_than_one_launch(codec):
+    """40 matrices (DF11_MAX_BATCH = 32 per launch), batch 2."""
+    shapes = [(16 + 8 * i, 256 + 64 * (i % 5)) for i in range(40)]
+    xs = [workloads.random_bf16(r * c, seed=900 + i).reshape(r, c) for i, (r, c) in enumerate(shapes)]
+    mats = codec.compress_block([to_dev(x).reshape(x.shape) for x in xs])
+    acts = [activations(2, c, seed=40 + i) for i, (_, c) in enumerate(shapes)]
+    ys = run(codec, mats, acts, 2)
+    for y, w, xb in zip(ys, xs, acts):
+        check_close(y, w, xb)

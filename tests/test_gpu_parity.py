@@ -215,3 +215,16 @@ def test_compress_block_matches_compress(codec):
         for x, o in zip([x for x in xs if x.size], outs):
             assert np.array_equal(bits_of(o), np.ascontiguousarray(x).reshape(-1))
         del got
+
+
+def test_batch_larger_than_one_launch(codec):
+    """More matrices than one launch takes (DF11_MAX_BATCH = 32): the call
+    splits them; every output must still be exact (sizes vary, one is empty,
+    one has 1-bit codes)."""
+    xs = [workloads.random_bf16(1_000 + 37_000 * i, seed=500 + i) for i in range(38)]
+    xs[5] = workloads.random_bf16(0, seed=1)
+    xs[17] = workloads.constant(70_001, 0x3F80)
+    mats = codec.compress_block([to_dev(x) for x in xs])
+    outs = codec.decompress_block([m for m in mats if m.n])
+    for x, o in zip([x for x in xs if x.size], outs):
+        assert np.array_equal(bits_of(o), x)
