@@ -11,9 +11,11 @@ xuá»‘ng cÃ²n 70% kÃ­ch thÆ°á»›c" (vi.news.hada.io/topic?id=20542), sections "Äá
 DFloat11" (format), "DÆ° Ä‘á»‹a nÃ©n cÃ²n láº¡i trong exponent cá»§a BFloat16" (exponent
 statistics) and "Kernel GPU hai giai Ä‘oáº¡n vÃ  metadata bá»• trá»£" (chunks, gaps,
 block output positions).  The readings the page leaves open are listed at the
-top of ``df11_oracle.c``.
+top of ``df11_oracle.c``; those of the rANS comparison variant (which the
+page's discussion only names) above its section there.
 
-Parity status: every entry point is pinned by ``tests/test_oracle_pins.py``.
+Parity status: every DF11 entry point is pinned by ``tests/test_oracle_pins.py``
+and every rANS entry point by ``tests/test_oracle_rans.py``.
 """
 from __future__ import annotations
 
@@ -77,6 +79,10 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "oracle_unpack_gaps": (None, [_u8p, c_u64, _u8p]),
         "oracle_decode_serial": (c_int, [_u8p, c_u64, c_u64, _u8p, _u32p, _u8p]),
         "oracle_decode_chunked": (c_int, [_u8p, _u8p, _u32p, c_u64, c_u64, _u8p, _u32p, _u8p]),
+        "oracle_rans_freqs": (c_int, [_u64p, _u32p]),
+        "oracle_rans_bound": (c_u64, [c_u64]),
+        "oracle_rans_encode": (c_int, [_u8p, c_u64, _u32p, _u8p, c_u64, _u32p, _u64p]),
+        "oracle_rans_decode": (c_int, [_u8p, _u32p, c_u64, _u32p, _u8p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -298,3 +304,82 @@ def stored_bytes(enc: Encoded) -> int:
     sign+mantissa plane and the 256 code lengths."""
     return (enc.stream.size + enc.gaps_packed.size + 4 * enc.block_pos.size
             + enc.sign_mantissa.size + 256)
+
+
+# ---- rANS variant of the exponent coding (comparison codec; the format's
+# readings Q1-Q5 are listed in df11_oracle.c)
+
+RANS_M = 4096
+RANS_L = 1 << 16
+RANS_LANES = 32
+RANS_STEPS = 512
+RANS_SEG_STEPS = 64
+RANS_SEGS = RANS_STEPS // RANS_SEG_STEPS
+RANS_UNIT = RANS_LANES * RANS_STEPS
+RANS_HEADER = 4 * RANS_LANES + 2 * RANS_SEGS
+
+
+def rans_freqs(hist: np.ndarray, lib=None) -> np.ndarray:
+    """Frequencies out of 4096 for a 256-bin histogram (Q1)."""
+    lib = lib or load()
+    h = np.ascontiguousarray(hist, dtype=np.uint64)
+    f = np.zeros(256, np.uint32)
+    if lib.oracle_rans_freqs(_p(h, _u64p), _p(f, _u32p)) != OK:
+        raise ValueError("rans_freqs failed")
+    return f
+
+
+@dataclass
+class RansEncoded:
+    n: int
+    hist: np.ndarray          # uint64[256]
+    freq: np.ndarray          # uint32[256], sum 4096 (or all zero for n = 0)
+    stream: np.ndarray        # uint8[bytes]: the units back to back
+    off16: np.ndarray         # uint32[U+1]: unit starts in 16-byte units
+    sign_mantissa: np.ndarray  # uint8[n]
+
+    @property
+    def units(self) -> int:
+        return (self.n + RANS_UNIT - 1) // RANS_UNIT
+
+
+def rans_encode(w: np.ndarray, freq=None, lib=None) -> RansEncoded:
+    """Split, histogram, frequencies (Q1) and the interleaved encode (Q2-Q4)."""
+    lib = lib or load()
+    w = np.ascontiguousarray(w, dtype=np.uint16).reshape(-1)
+    n = w.size
+    e, sm = split(w, lib)
+    h = histogram(e, lib)
+    f = rans_freqs(h, lib) if freq is None else np.ascontiguousarray(freq, np.uint32)
+    units = (n + RANS_UNIT - 1) // RANS_UNIT
+    cap = int(lib.oracle_rans_bound(n))
+    stream = np.zeros(max(cap, 16), np.uint8)
+    off16 = np.zeros(units + 1, np.uint32)
+    nbytes = ctypes.c_uint64(0)
+    r = lib.oracle_rans_encode(_p(e, _u8p), n, _p(f, _u32p), _p(stream, _u8p), stream.size,
+                               _p(off16, _u32p), ctypes.byref(nbytes))
+    if r != OK:
+        raise ValueError(f"oracle_rans_encode failed with {r}")
+    return RansEncoded(n=n, hist=h, freq=f, stream=stream[: int(nbytes.value)].copy(),
+                       off16=off16, sign_mantissa=sm)
+
+
+def rans_decode(enc: RansEncoded, lib=None) -> np.ndarray:
+    """Definition-level decode (linear symbol search per value) -> BF16 words."""
+    lib = lib or load()
+    e = np.zeros(enc.n, np.uint8)
+    s = np.ascontiguousarray(enc.stream, np.uint8)
+    if s.size == 0:
+        s = np.zeros(16, np.uint8)
+    r = lib.oracle_rans_decode(_p(s, _u8p), _p(np.ascontiguousarray(enc.off16, np.uint32), _u32p),
+                               enc.n, _p(np.ascontiguousarray(enc.freq, np.uint32), _u32p),
+                               _p(e, _u8p))
+    if r != OK:
+        raise ValueError("rANS stream is corrupt")
+    return merge(e, enc.sign_mantissa, lib)
+
+
+def rans_stored_bytes(enc: RansEncoded) -> int:
+    """Bytes the rANS variant stores: the unit streams, the unit offsets,
+    the sign+mantissa plane and 256 frequencies (2 bytes each)."""
+    return enc.stream.size + 4 * enc.off16.size + enc.sign_mantissa.size + 512

@@ -542,3 +542,198 @@ int oracle_decode_chunked(const uint8_t *stream, const uint8_t *gap,
   }
   return OR_OK;
 }
+
+/* ======================================================================
+ * rANS variant of the exponent coding (a comparison codec).  The method's
+ * pages only name rANS as an alternative to Huffman; the format below is a
+ * reading, written here from the definition of range ANS (Duda 2013) with
+ * its usual byte-oriented renormalisation:
+ *   Q1 probabilities: each exponent present with count c gets a frequency
+ *      f >= 1 out of M = 4096; f = floor(c*M/n) (at least 1), then the sum is
+ *      brought to M one step at a time: while below, +1 to the symbol with
+ *      the largest deficit c*M - f*n (ties: smaller symbol); while above, -1
+ *      to the symbol with f > 1 and the smallest deficit (ties: smaller
+ *      symbol).  One symbol alone gets f = M.  cum[s] = sum of f[t], t < s.
+ *   Q2 state: 32-bit, kept in [2^16, 2^32); renormalisation moves 16-bit
+ *      words.  Encoding symbol s: if x >= f[s] << 20, emit the low 16 bits
+ *      and shift right by 16; then x = (x / f[s]) * M + x % f[s] + cum[s].
+ *      Decoding: slot = x % M, s the symbol with cum[s] <= slot < cum[s] +
+ *      f[s], x = f[s] * (x / M) + slot - cum[s]; if x < 2^16, x = (x << 16)
+ *      | next word.
+ *   Q3 interleaving: values are grouped in units of 16384; value
+ *      u*16384 + 32*k + l is coded by state l (0..31) of unit u as its k-th
+ *      symbol.  Decoding runs k = 0..511 and, for each k, l = 0..31; the
+ *      words are read in that order from one stream per unit.  Encoding
+ *      runs the exact reverse order, each state starting at 2^16.  A unit's
+ *      steps form 8 segments of 64.
+ *   Q4 unit layout: the 32 final encoder states (little-endian uint32,
+ *      the decoder's initial states), then 8 little-endian uint16: the
+ *      index of the first word read in each segment (the first is 0), then
+ *      the words in decoding order (little-endian uint16), zero-padded to a
+ *      multiple of 16 bytes.  off16[u] = start of unit u in 16-byte units;
+ *      off16[U] = total.
+ *   Q5 integrity: after decoding a unit every state is back at 2^16 and
+ *      every word has been read.
+ * ====================================================================== */
+
+#define OR_RANS_BITS 12u
+#define OR_RANS_M (1u << OR_RANS_BITS)
+#define OR_RANS_L (1u << 16)
+#define OR_RANS_LANES 32u
+#define OR_RANS_STEPS 512u
+#define OR_RANS_SEG_STEPS 64u
+#define OR_RANS_SEGS (OR_RANS_STEPS / OR_RANS_SEG_STEPS)
+#define OR_RANS_UNIT (OR_RANS_LANES * OR_RANS_STEPS)
+#define OR_RANS_HEADER (4 * OR_RANS_LANES + 2 * OR_RANS_SEGS)
+
+int oracle_rans_freqs(const uint64_t hist[256], uint32_t freq[256]) {
+  uint64_t n = 0;
+  int present = 0, only = -1;
+  for (int s = 0; s < 256; s++) {
+    n += hist[s];
+    if (hist[s]) { present++; only = s; }
+  }
+  for (int s = 0; s < 256; s++) freq[s] = 0;
+  if (n == 0) return OR_OK;
+  if (present == 1) { freq[only] = OR_RANS_M; return OR_OK; }
+  int64_t sum = 0;
+  for (int s = 0; s < 256; s++) {
+    if (!hist[s]) continue;
+    uint64_t f = hist[s] * OR_RANS_M / n;
+    freq[s] = f ? (uint32_t)f : 1u;
+    sum += freq[s];
+  }
+  while (sum != (int64_t)OR_RANS_M) {
+    int pick = -1;
+    int64_t best = 0;
+    for (int s = 0; s < 256; s++) {
+      if (!hist[s]) continue;
+      int64_t d = (int64_t)(hist[s] * OR_RANS_M) - (int64_t)freq[s] * (int64_t)n;  /* deficit */
+      if (sum < (int64_t)OR_RANS_M) {
+        if (pick < 0 || d > best) { pick = s; best = d; }
+      } else {
+        if (freq[s] > 1 && (pick < 0 || d < best)) { pick = s; best = d; }
+      }
+    }
+    if (pick < 0) return OR_ERR_ARG;
+    if (sum < (int64_t)OR_RANS_M) { freq[pick]++; sum++; }
+    else { freq[pick]--; sum--; }
+  }
+  return OR_OK;
+}
+
+static void rans_cum(const uint32_t freq[256], uint32_t cum[257]) {
+  cum[0] = 0;
+  for (int s = 0; s < 256; s++) cum[s + 1] = cum[s] + freq[s];
+}
+
+/* Bytes the encoded stream needs at most: per unit the header and one word
+ * per value, padded. */
+uint64_t oracle_rans_bound(uint64_t n) {
+  uint64_t units = (n + OR_RANS_UNIT - 1) / OR_RANS_UNIT;
+  return units * (OR_RANS_HEADER + 2 * OR_RANS_UNIT + 16);
+}
+
+int oracle_rans_encode(const uint8_t *exponent, uint64_t n, const uint32_t freq[256],
+                       uint8_t *stream, uint64_t cap, uint32_t *off16, uint64_t *bytes) {
+  uint32_t cum[257];
+  rans_cum(freq, cum);
+  uint64_t units = (n + OR_RANS_UNIT - 1) / OR_RANS_UNIT;
+  uint16_t *words = (uint16_t *)malloc(sizeof(uint16_t) * (OR_RANS_UNIT + 1));
+  if (!words) return OR_ERR_ARG;
+  uint64_t at = 0;  /* bytes written so far */
+  for (uint64_t u = 0; u < units; u++) {
+    uint32_t x[OR_RANS_LANES];
+    for (unsigned l = 0; l < OR_RANS_LANES; l++) x[l] = OR_RANS_L;
+    uint64_t nw = 0;  /* words emitted, in reverse decoding order */
+    uint64_t seg_words[OR_RANS_SEGS];
+    for (unsigned g = 0; g < OR_RANS_SEGS; g++) seg_words[g] = 0;
+    for (int k = (int)OR_RANS_STEPS - 1; k >= 0; k--) {
+      for (int l = (int)OR_RANS_LANES - 1; l >= 0; l--) {
+        uint64_t i = u * OR_RANS_UNIT + (uint64_t)k * OR_RANS_LANES + (uint64_t)l;
+        if (i >= n) continue;
+        unsigned s = exponent[i];
+        uint32_t f = freq[s];
+        if (f == 0) { free(words); return OR_ERR_SYMBOL; }
+        if ((uint64_t)x[l] >= ((uint64_t)f << 20)) {  /* Q2: x_max = (L / M) * 2^16 * f */
+          words[nw++] = (uint16_t)(x[l] & 0xFFFFu);
+          x[l] >>= 16;
+          seg_words[(unsigned)k / OR_RANS_SEG_STEPS]++;  /* read by the decoder at step k */
+        }
+        x[l] = (x[l] / f) * OR_RANS_M + x[l] % f + cum[s];
+      }
+    }
+    uint64_t ubytes = OR_RANS_HEADER + 2 * nw;
+    uint64_t padded = (ubytes + 15) / 16 * 16;
+    if (at + padded > cap) { free(words); return OR_ERR_ARG; }
+    off16[u] = (uint32_t)(at / 16);
+    uint8_t *p = stream + at;
+    for (unsigned l = 0; l < OR_RANS_LANES; l++)
+      for (unsigned b = 0; b < 4; b++) p[4 * l + b] = (uint8_t)(x[l] >> (8 * b));
+    uint64_t first = 0;  /* decoding index of each segment's first word */
+    for (unsigned g = 0; g < OR_RANS_SEGS; g++) {
+      p[4 * OR_RANS_LANES + 2 * g] = (uint8_t)(first & 0xFF);
+      p[4 * OR_RANS_LANES + 2 * g + 1] = (uint8_t)(first >> 8);
+      first += seg_words[g];
+    }
+    for (uint64_t j = 0; j < nw; j++) {  /* decoding order: last emitted first */
+      uint16_t wv = words[nw - 1 - j];
+      p[OR_RANS_HEADER + 2 * j] = (uint8_t)(wv & 0xFF);
+      p[OR_RANS_HEADER + 2 * j + 1] = (uint8_t)(wv >> 8);
+    }
+    for (uint64_t j = ubytes; j < padded; j++) p[j] = 0;
+    at += padded;
+  }
+  off16[units] = (uint32_t)(at / 16);
+  *bytes = at;
+  free(words);
+  return OR_OK;
+}
+
+int oracle_rans_decode(const uint8_t *stream, const uint32_t *off16, uint64_t n,
+                       const uint32_t freq[256], uint8_t *exponent) {
+  uint32_t cum[257];
+  rans_cum(freq, cum);
+  uint64_t units = (n + OR_RANS_UNIT - 1) / OR_RANS_UNIT;
+  for (uint64_t u = 0; u < units; u++) {
+    const uint8_t *p = stream + (uint64_t)off16[u] * 16;
+    uint64_t ubytes = ((uint64_t)off16[u + 1] - off16[u]) * 16;
+    if (ubytes < OR_RANS_HEADER) return OR_ERR_CORRUPT;
+    uint64_t nwords = (ubytes - OR_RANS_HEADER) / 2, wp = 0;
+    uint32_t x[OR_RANS_LANES];
+    for (unsigned l = 0; l < OR_RANS_LANES; l++)
+      x[l] = (uint32_t)p[4 * l] | (uint32_t)p[4 * l + 1] << 8 | (uint32_t)p[4 * l + 2] << 16 |
+             (uint32_t)p[4 * l + 3] << 24;
+    for (unsigned k = 0; k < OR_RANS_STEPS; k++) {
+      if (k % OR_RANS_SEG_STEPS == 0) {  /* the recorded start of the segment */
+        unsigned g = k / OR_RANS_SEG_STEPS;
+        uint64_t first = (uint64_t)p[4 * OR_RANS_LANES + 2 * g] |
+                         (uint64_t)p[4 * OR_RANS_LANES + 2 * g + 1] << 8;
+        if (first != wp) return OR_ERR_CORRUPT;
+      }
+      for (unsigned l = 0; l < OR_RANS_LANES; l++) {
+        uint64_t i = u * OR_RANS_UNIT + (uint64_t)k * OR_RANS_LANES + l;
+        if (i >= n) continue;
+        uint32_t slot = x[l] % OR_RANS_M;
+        int s = -1;
+        for (int t = 0; t < 256; t++)
+          if (freq[t] && cum[t] <= slot && slot < cum[t] + freq[t]) { s = t; break; }
+        if (s < 0) return OR_ERR_CORRUPT;
+        exponent[i] = (uint8_t)s;
+        x[l] = freq[s] * (x[l] / OR_RANS_M) + slot - cum[s];
+        if (x[l] < OR_RANS_L) {
+          if (wp >= nwords) return OR_ERR_CORRUPT;
+          uint32_t wv = (uint32_t)p[OR_RANS_HEADER + 2 * wp] |
+                        (uint32_t)p[OR_RANS_HEADER + 2 * wp + 1] << 8;
+          wp++;
+          x[l] = (x[l] << 16) | wv;
+        }
+      }
+    }
+    for (unsigned l = 0; l < OR_RANS_LANES; l++)
+      if (x[l] != OR_RANS_L) return OR_ERR_CORRUPT;          /* Q5 */
+    for (uint64_t j = wp; j < nwords; j++)                   /* only padding may remain */
+      if (p[OR_RANS_HEADER + 2 * j] || p[OR_RANS_HEADER + 2 * j + 1]) return OR_ERR_CORRUPT;
+  }
+  return OR_OK;
+}

@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import workloads
+import test_oracle_rans as rp
 from test_oracle_pins import GOLDEN, cost, kraft, textbook_huffman_cost, hist_from
 
 MUTATIONS = {
@@ -37,6 +38,21 @@ MUTATIONS = {
     "tail_chunk_not_clipped": [("      if (limit > total_bits) limit = total_bits;\n      if (gap[c] > 31)",
                                 "      if (gap[c] > 31)")],
     "canonical_no_shift": [("    c = (c + bl_count[bits - 1]) << 1;", "    c = (c + bl_count[bits - 1]);")],
+    "rans_renorm_strict": [("if ((uint64_t)x[l] >= ((uint64_t)f << 20)) {",
+                            "if ((uint64_t)x[l] > ((uint64_t)f << 20)) {")],
+    "rans_threshold_one_bit_low": [("if ((uint64_t)x[l] >= ((uint64_t)f << 20)) {",
+                                    "if ((uint64_t)x[l] >= ((uint64_t)f << 19)) {")],
+    "rans_words_in_emission_order": [("uint16_t wv = words[nw - 1 - j];", "uint16_t wv = words[j];")],
+    "rans_cum_starts_at_one": [("  cum[0] = 0;\n  for (int s = 0; s < 256; s++) cum[s + 1]",
+                                "  cum[0] = 1;\n  for (int s = 0; s < 256; s++) cum[s + 1]")],
+    "rans_ties_to_larger_symbol": [("if (pick < 0 || d > best) { pick = s; best = d; }",
+                                    "if (pick < 0 || d >= best) { pick = s; best = d; }")],
+    "rans_initial_state_off": [("for (unsigned l = 0; l < OR_RANS_LANES; l++) x[l] = OR_RANS_L;",
+                                "for (unsigned l = 0; l < OR_RANS_LANES; l++) x[l] = OR_RANS_L + 16;")],
+    "rans_segment_start_inclusive": [("      first += seg_words[g];\n    }",
+                                      "    }")],
+    "rans_lanes_forward_in_encoder": [("for (int l = (int)OR_RANS_LANES - 1; l >= 0; l--) {",
+                                       "for (int l = 0; l < (int)OR_RANS_LANES; l++) {")],
 }
 
 
@@ -94,7 +110,24 @@ def _check_round_trip(lib):
         assert np.array_equal(oracle.decode(enc, chunked=True, lib=lib), x)
 
 
-CHECKS = [_check_uniform, _check_tie, _check_costs, _check_golden, _check_layout, _check_round_trip]
+def _check_rans(lib):
+    f = oracle.rans_freqs(rp.hist_of({0: 1, 1: 1, 2: 1}), lib)
+    assert f[:3].tolist() == [1366, 1365, 1365]
+    for case in rp.golden_cases():
+        w = rp.weights_with_exponents(rp.golden_exponents(case))
+        enc = oracle.rans_encode(w, freq=rp.freq_array(case["freq"]), lib=lib)
+        assert enc.stream.tobytes() == rp.unit_bytes_from_fields(case)
+    x = workloads.shuffled_patterns(copies=1, seed=11)[: 3 * 16384 + 77]
+    enc = oracle.rans_encode(x, freq=np.full(256, 16, np.uint32), lib=lib)
+    assert np.array_equal(oracle.rans_decode(enc, lib=lib), x)
+    for n in (65, 40_000):
+        x = workloads.random_bf16(n, seed=n)
+        enc = oracle.rans_encode(x, lib=lib)
+        assert np.array_equal(oracle.rans_decode(enc, lib=lib), x)
+
+
+CHECKS = [_check_uniform, _check_tie, _check_costs, _check_golden, _check_layout, _check_round_trip,
+          _check_rans]
 
 
 def _failures(lib):
