@@ -1,4 +1,5 @@
-"""Python binding of the DF11 C ABI (``include/df11.h``).
+"""Python binding of the DF11 C ABI (``include/df11.h``, and the rANS
+comparison variant of ``include/df11_rans.h``).
 
 Argument marshalling only: every entry point of ``libdf11_b200.so`` is exposed
 under its C name with the same arguments (device pointers and streams as
@@ -18,7 +19,9 @@ import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdf11_b200.so")
-HEADER = os.path.join(os.path.dirname(HERE), "include", "df11.h")
+INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+HEADER = os.path.join(INCLUDE, "df11.h")
+HEADERS = [HEADER, os.path.join(INCLUDE, "df11_rans.h")]
 
 CHUNK_BITS = 64
 BLOCK_CHUNKS = 256
@@ -72,6 +75,11 @@ class df11_matmul_io(ctypes.Structure):
                 ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 
+class df11_rans_matrix(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_uint64), ("stream", ctypes.c_void_p), ("off16", ctypes.c_void_p),
+                ("sign_mantissa", ctypes.c_void_p), ("tables", ctypes.c_void_p)]
+
+
 class DF11Error(RuntimeError):
     def __init__(self, status: int, where: str = ""):
         self.status = status
@@ -107,6 +115,14 @@ def _declare(lib):
         "df11_decode_matmul_batch": (ctypes.c_int, [ctypes.POINTER(df11_matrix),
                                                     ctypes.POINTER(df11_matmul_io), _u32, _u32,
                                                     _vp, _vp]),
+        "df11_rans_freqs": (ctypes.c_int, [_u64p, ctypes.POINTER(ctypes.c_uint32)]),
+        "df11_rans_build_tables": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _vp,
+                                                  ctypes.c_size_t]),
+        "df11_rans_units": (_u64, [_u64]),
+        "df11_rans_encode_sizes": (ctypes.c_int, [_vp, _u64, _vp, _vp, _vp, _vp, _vp]),
+        "df11_rans_encode": (ctypes.c_int, [_vp, _u64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "df11_rans_decode_batch": (ctypes.c_int, [ctypes.POINTER(df11_rans_matrix), _u32,
+                                                  ctypes.POINTER(ctypes.c_void_p), _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -133,9 +149,12 @@ def load():
 
 
 def declared_functions() -> list[str]:
-    """Names of the functions declared in include/df11.h."""
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(df11_\w+)\s*\(", text, re.M)))
+    """Names of the functions declared in the headers under include/."""
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        names |= set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(df11_\w+)\s*\(", text, re.M))
+    return sorted(names)
 
 
 # ------------------------------------------------------------- entry points
@@ -220,3 +239,46 @@ def df11_encode_static_ws(d_w: int, n: int, cb: df11_codebook, total_bits: int, 
     allocate device memory at the call site; see include/df11.h."""
     return load().df11_encode_static_ws(d_w, n, ctypes.byref(cb), total_bits, ctypes.byref(out),
                                         d_status, stream)
+
+
+# ------------------------------------------------ rANS variant (df11_rans.h)
+
+RANS_PROB_BITS = 12
+RANS_UNIT = 16384
+RANS_HEADER_BYTES = 144
+RANS_TABLES_BYTES = 17408
+RANS_MAX_BATCH = 32
+
+
+def df11_rans_freqs(hist256):
+    """Returns (status, list of 256 frequencies out of 4096)."""
+    h = (ctypes.c_uint64 * 256)(*[int(x) for x in hist256])
+    f = (ctypes.c_uint32 * 256)()
+    st = load().df11_rans_freqs(h, f)
+    return st, list(f)
+
+
+def df11_rans_build_tables(freq, h_tables: int, nbytes: int) -> int:
+    f = (ctypes.c_uint32 * 256)(*[int(x) for x in freq])
+    return load().df11_rans_build_tables(f, h_tables, nbytes)
+
+
+def df11_rans_units(n: int) -> int:
+    return int(load().df11_rans_units(n))
+
+
+def df11_rans_encode_sizes(d_w: int, n: int, d_tables: int, d_unit_words: int, d_off16: int,
+                           d_status: int, stream: int = 0) -> int:
+    return load().df11_rans_encode_sizes(d_w, n, d_tables, d_unit_words, d_off16, d_status, stream)
+
+
+def df11_rans_encode(d_w: int, n: int, d_tables: int, d_unit_words: int, d_off16: int,
+                     d_stream: int, d_sign_mantissa: int, d_status: int, stream: int = 0) -> int:
+    return load().df11_rans_encode(d_w, n, d_tables, d_unit_words, d_off16, d_stream,
+                                   d_sign_mantissa, d_status, stream)
+
+
+def df11_rans_decode_batch(ms, d_outs, d_status: int, stream: int = 0) -> int:
+    arr = (df11_rans_matrix * max(1, len(ms)))(*ms)
+    outs = (ctypes.c_void_p * max(1, len(d_outs)))(*[int(p) for p in d_outs])
+    return load().df11_rans_decode_batch(arr, len(ms), outs, d_status, stream)
