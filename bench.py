@@ -58,6 +58,8 @@ def parse():
                     help="passes of the device-only encode timing (0: skip)")
     ap.add_argument("--matmul-steps", type=int, default=10,
                     help="steps of the fused decode -> matmul timing (0: skip)")
+    ap.add_argument("--rans-steps", type=int, default=10,
+                    help="decode launches of the block coded with the rANS variant (0: skip)")
     ap.add_argument("--block-steps", type=int, default=5,
                     help="steps of the DF11 transformer-block forward timing (0: skip)")
     return ap.parse_args()
@@ -327,6 +329,14 @@ def run_df11(args):
     if int(status.item()) != 0:
         raise df11.DF11Error(int(status.item()), "decode (device)")
 
+    # ---- the rANS variant of the exponent coding on the same block: its
+    # ratio and decode time beside the Huffman format's, launches alternated
+    rans_line = None
+    if args.rans_steps > 0:
+        peak_r, peak_kind_r = measured_peak()
+        rans_line = time_rans(torch, df11, ws, outs, out_ptrs, status, dev, args.rans_steps,
+                              args.warmup, peak_r, peak_kind_r, n_total, ratio, step, stream)
+
     # ---- end to end through the C ABI with host buffers (pinned)
     e2e = None
     if args.e2e_steps > 0:
@@ -423,6 +433,7 @@ def run_df11(args):
             "encode": encode,
             "fused_matmul": fused,
             "block_forward": blockfw,
+            "rans": rans_line,
             "code_len_cap": CAP,
             "max_code_len": max(int(m.codebook.max_len) for m in cms),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "cap32": cap32,
@@ -433,6 +444,79 @@ def run_df11(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def time_rans(torch, df11, ws, outs, out_ptrs, status, dev, steps, warmup, peak, peak_kind,
+              n_total, huffman_ratio, huffman_step, huffman_stream):
+    """The block coded with the rANS variant (df11_rans.h): compression on the
+    device, then `steps` decode launches (all matrices in one launch), each
+    followed by one launch of the Huffman format's decode (huffman_step, on
+    huffman_stream), every launch timed with CUDA events on its stream, after
+    `warmup` untimed ones and a bit-exactness check.  Alternating the two
+    gives both the same clocks and the same L2 history."""
+    import lossless_bf16_weight_df11_b200.rans as rans
+    rans.compress_block([ws[0][:65536]])
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record()
+    rms = rans.compress_block(ws)
+    c1.record()
+    torch.cuda.synchronize()
+    abis = [m.abi() for m in rms]
+    stream = torch.cuda.Stream(device=dev)
+    sh = int(stream.cuda_stream)
+    status.zero_()
+
+    def step():
+        st = df11.df11_rans_decode_batch(abis, out_ptrs, status.data_ptr(), sh)
+        if st:
+            raise df11.DF11Error(st, "df11_rans_decode_batch")
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            step()
+    torch.cuda.synchronize()
+    ok = int(status.item()) == 0 and all(
+        torch.equal(o.reshape(-1).view(torch.int16), w) for o, w in zip(outs, ws))
+    def pair():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    evs = [pair() for _ in range(steps)]
+    evh = [pair() for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for (a, b), (c, d) in zip(evs, evh):
+            with torch.cuda.stream(stream):
+                a.record(stream)
+                step()
+                b.record(stream)
+            stream.synchronize()
+            with torch.cuda.stream(huffman_stream):
+                c.record(huffman_stream)
+                huffman_step()
+                d.record(huffman_stream)
+            torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise df11.DF11Error(int(status.item()), "decode (device)")
+    t = [a.elapsed_time(b) for a, b in evs]
+    th = [c.elapsed_time(d) for c, d in evh]
+    avg = statistics.mean(t)
+    algo = sum(m.read_bytes for m in rms) + 2 * n_total
+    r = sum(m.stored_bytes for m in rms) / (2 * n_total)
+    out = {"ratio": r, "bits_per_weight": 16 * r, "bit_exact": ok, "launches": steps,
+           "ms_per_launch": avg, "median_ms": statistics.median(t),
+           "value": 2 * n_total / (avg / 1e3) / 1e9, "unit": "GB/s",
+           "compress_block_ms": c0.elapsed_time(c1),
+           "roofline": {"bound": "hbm", "achieved": algo / (avg / 1e3) / 1e9, "peak": peak,
+                        "unit": "GB/s", "frac": algo / (avg / 1e3) / 1e9 / peak,
+                        "peak_kind": peak_kind, "kernel": "rans_decode_kernel",
+                        "algorithmic_bytes_per_launch": algo},
+           "vs_huffman": {"stored_size": r / huffman_ratio,
+                          "huffman_median_ms_alternated": statistics.median(th),
+                          "decode_time": statistics.median(t) / statistics.median(th)},
+           "clocks": clk.summary()}
+    del rms
+    return out
 
 
 def time_encode(torch, df11, cms, ws, dev, steps, peak, peak_kind):
