@@ -276,6 +276,18 @@ def run_df11(args):
     same = all(int(a.total_bits) == int(b.total_bits) and torch.equal(a.stream, b.stream)
                for a, b in zip(cms, cms_b))
     del cms_b
+    # the all-device compressor (codebooks built by a kernel)
+    codec.compress_block_device([ws[0][:65536], ws[1][:65536]], cap=CAP)
+    torch.cuda.synchronize()
+    ed0, ed1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ed0.record()
+    cms_d = codec.compress_block_device(ws, cap=CAP)
+    ed1.record()
+    torch.cuda.synchronize()
+    compress_device_ms = ed0.elapsed_time(ed1)
+    same_device = all(int(a.total_bits) == int(b.total_bits) and torch.equal(a.stream, b.stream)
+                      and torch.equal(a.tables, b.tables) for a, b in zip(cms, cms_d))
+    del cms_d
     read_bytes = sum(m.read_bytes for m in cms)
     stored = sum(m.stored_bytes for m in cms)
     ratio = stored / (2 * n_total)
@@ -430,6 +442,12 @@ def run_df11(args):
                                "same_as_per_matrix": same,
                                "includes": "all histograms, one copy to the host, host codebooks "
                                            "and tables, all encodes, one copy of the status words"},
+            "compress_block_device": {"ms": compress_device_ms,
+                                      "input_GBps": 2 * n_total / (compress_device_ms / 1e3) / 1e9,
+                                      "same_as_per_matrix": same_device,
+                                      "includes": "all histograms, codebooks and tables built on the "
+                                                  "device, one copy of codebooks and sizes to the "
+                                                  "host, all encodes, one copy of the status words"},
             "encode": encode,
             "fused_matmul": fused,
             "block_forward": blockfw,

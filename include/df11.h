@@ -163,6 +163,34 @@ df11_status df11_build_codebook(const uint64_t hist256[256], uint32_t cap,
 df11_status df11_encoded_sizes(const df11_codebook *cb, const uint64_t hist256[256],
                                uint64_t n, df11_sizes *out);
 
+/*
+ * df11_sizes_from_bits -- host.  The sizes df11_encoded_sizes gives, from n
+ * and total_bits alone (for a codebook built on the device: its total_bits
+ * comes back from df11_build_codebook_device).  DF11_ERR_INVALID_ARG unless
+ * n <= total_bits <= 32 n.
+ */
+df11_status df11_sizes_from_bits(uint64_t n, uint64_t total_bits, df11_sizes *out);
+
+/*
+ * df11_build_codebook_device -- S3 on the device: the codebook, its decode
+ * tables and the encoded size from a device histogram, in one kernel launch
+ * (one CTA), with no host round trip.  [Format], [LUT]: the same rule as
+ * df11_build_codebook; the results equal, byte for byte, those of
+ * df11_build_codebook + df11_build_tables + df11_encoded_sizes on the host
+ * (one implementation serves both).
+ *   d_hist256     256 uint64 counts (df11_histogram's output).
+ *   cap           1..32 (checked on the host).
+ *   d_cb          device df11_codebook, written.
+ *   d_tables      df11_tables_bytes() device bytes (16-byte aligned), written.
+ *   d_total_bits  device uint64: sum over e of hist[e] * len[e], written.
+ *   d_status      DF11_ERR_INVALID_ARG if 2^cap is below the number of
+ *                 distinct exponents (then nothing else is written).
+ */
+df11_status df11_build_codebook_device(const uint64_t *d_hist256, uint32_t cap,
+                                       df11_codebook *d_cb, void *d_tables,
+                                       uint64_t *d_total_bits, uint32_t *d_status,
+                                       df11_stream_t stream);
+
 /* Bytes of the decode tables of one codebook (a constant). */
 size_t df11_tables_bytes(void);
 
@@ -191,6 +219,20 @@ df11_status df11_build_tables(const df11_codebook *cb, void *h_tables, size_t by
 df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_codebook *cb,
                         uint64_t total_bits, const df11_encoded *out, void *d_workspace,
                         size_t workspace_bytes, uint32_t *d_status, df11_stream_t stream);
+
+/*
+ * df11_encode_device_codebook -- df11_encode with the codebook in device
+ * memory (d_cb, as written by df11_build_codebook_device), for a compressor
+ * that keeps every step on the device.  total_bits is the value
+ * df11_build_codebook_device wrote (the caller reads it back to size the
+ * buffers).  A length above 32 in d_cb is treated as 32 and a code that does
+ * not fit its length is cut to it; the device check of total_bits then
+ * reports DF11_ERR_CORRUPT.  Otherwise as df11_encode.
+ */
+df11_status df11_encode_device_codebook(const uint16_t *d_w, uint64_t n, const df11_codebook *d_cb,
+                                        uint64_t total_bits, const df11_encoded *out,
+                                        void *d_workspace, size_t workspace_bytes,
+                                        uint32_t *d_status, df11_stream_t stream);
 
 /*
  * df11_encode_static_ws -- df11_encode for callers that cannot allocate

@@ -115,6 +115,11 @@ def _declare(lib):
         "df11_decode_matmul_batch": (ctypes.c_int, [ctypes.POINTER(df11_matrix),
                                                     ctypes.POINTER(df11_matmul_io), _u32, _u32,
                                                     _vp, _vp]),
+        "df11_sizes_from_bits": (ctypes.c_int, [_u64, _u64, ctypes.POINTER(df11_sizes)]),
+        "df11_build_codebook_device": (ctypes.c_int, [_vp, _u32, _vp, _vp, _vp, _vp, _vp]),
+        "df11_encode_device_codebook": (ctypes.c_int, [_vp, _u64, _vp, _u64,
+                                                       ctypes.POINTER(df11_encoded), _vp,
+                                                       ctypes.c_size_t, _vp, _vp]),
         "df11_rans_freqs": (ctypes.c_int, [_u64p, ctypes.POINTER(ctypes.c_uint32)]),
         "df11_rans_build_tables": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _vp,
                                                   ctypes.c_size_t]),
@@ -228,6 +233,30 @@ def df11_validate(n: int, total_bits: int, min_len: int, h_gaps: int, gaps_bytes
                   h_block_pos: int, block_pos_count: int) -> int:
     return load().df11_validate(n, total_bits, min_len, h_gaps, gaps_bytes, h_block_pos,
                                 block_pos_count)
+
+
+def df11_sizes_from_bits(n: int, total_bits: int):
+    out = df11_sizes()
+    st = load().df11_sizes_from_bits(n, total_bits, ctypes.byref(out))
+    return st, out
+
+
+def df11_build_codebook_device(d_hist256: int, cap: int, d_cb: int, d_tables: int,
+                               d_total_bits: int, d_status: int, stream: int = 0) -> int:
+    """Codebook, decode tables and total_bits built on the device from a
+    device histogram; see include/df11.h."""
+    return load().df11_build_codebook_device(d_hist256, cap, d_cb, d_tables, d_total_bits,
+                                             d_status, stream)
+
+
+def df11_encode_device_codebook(d_w: int, n: int, d_cb: int, total_bits: int, out: df11_encoded,
+                                d_workspace: int, workspace_bytes: int, d_status: int,
+                                stream: int = 0) -> int:
+    return load().df11_encode_device_codebook(d_w, n, d_cb, total_bits, ctypes.byref(out),
+                                              d_workspace, workspace_bytes, d_status, stream)
+
+
+CODEBOOK_BYTES = ctypes.sizeof(df11_codebook)   # 1296
 
 
 STATIC_WS_MAX_N = 268431360  # DF11_STATIC_WS_MAX_N

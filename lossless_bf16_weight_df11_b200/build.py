@@ -12,8 +12,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdf11_b200.so")
 SOURCES = [os.path.join(CSRC, "df11_kernels.cu"), os.path.join(CSRC, "df11_host.cpp"),
            os.path.join(CSRC, "rans_kernels.cu"), os.path.join(CSRC, "rans_host.cpp")]
-HEADERS = [os.path.join(CSRC, "df11_internal.h"), os.path.join(INCLUDE, "df11.h"),
-           os.path.join(INCLUDE, "df11_rans.h")]
+HEADERS = [os.path.join(CSRC, "df11_internal.h"), os.path.join(CSRC, "df11_codebook.h"),
+           os.path.join(INCLUDE, "df11.h"), os.path.join(INCLUDE, "df11_rans.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

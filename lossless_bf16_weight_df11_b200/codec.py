@@ -18,10 +18,11 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-from . import (MAX_CODE_LEN, TABLE_BITS, DF11Error, check, df11_build_codebook, df11_build_tables,
-               df11_codebook, df11_decode, df11_decode_block_batch, df11_decode_matmul_batch,
-               df11_encode, df11_encoded, df11_matmul_io,
-               df11_encoded_sizes, df11_histogram, df11_matrix, df11_sizes, df11_tables_bytes)
+from . import (CODEBOOK_BYTES, MAX_CODE_LEN, TABLE_BITS, DF11Error, check, df11_build_codebook,
+               df11_build_codebook_device, df11_build_tables, df11_codebook, df11_decode,
+               df11_decode_block_batch, df11_decode_matmul_batch, df11_encode,
+               df11_encode_device_codebook, df11_encoded, df11_matmul_io, df11_encoded_sizes,
+               df11_histogram, df11_matrix, df11_sizes, df11_sizes_from_bits, df11_tables_bytes)
 
 
 def _stream_handle(stream) -> int:
@@ -210,6 +211,79 @@ def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
         mats.append(DF11Matrix(shape=tuple(w.shape), n=u.numel(),
                                total_bits=int(sizes_l[i].total_bits), codebook=cbs[i],
                                sizes=sizes_l[i], tables=tables[i], hist=h_all[i],
+                               max_block_codes=int(st_host[i, 1]), **mats_bufs[i]))
+    return mats
+
+
+# one row per matrix of the device compressor's metadata: the codebook, then
+# total_bits (8-byte aligned), padded to 16 bytes
+_META_ROW = (CODEBOOK_BYTES + 8 + 15) // 16 * 16
+_META_BITS = CODEBOOK_BYTES // 8 * 8
+
+
+def compress_block_device(ws, cap: int = DEFAULT_CAP, stream=None,
+                          check_status: bool = True) -> list[DF11Matrix]:
+    """compress_block with every step on the device: histograms, codebooks
+    and decode tables (df11_build_codebook_device), encodes with the device
+    codebooks (df11_encode_device_codebook).  The host only sizes the
+    buffers: one copy of every codebook and bit count, and one copy of the
+    status words.  The result equals compress_block's, array for array."""
+    if not ws:
+        return []
+    if CODEBOOK_BYTES % 8:
+        raise RuntimeError("unexpected df11_codebook size")
+    us = [_as_u16(w) for w in ws]
+    dev = us[0].device
+    sh = _stream_handle(stream)
+    k = len(us)
+    nt = df11_tables_bytes()
+    hists = torch.empty(k, 256, dtype=torch.int64, device=dev)
+    meta = torch.zeros(k, _META_ROW, dtype=torch.uint8, device=dev)
+    tables = torch.empty(k, nt, dtype=torch.uint8, device=dev)
+    status = torch.zeros(k, 4, dtype=torch.int32, device=dev)  # [status, most codes per block, ...]
+    with torch.cuda.device(dev):
+        for i, u in enumerate(us):
+            check(df11_histogram(u.data_ptr(), u.numel(), hists[i].data_ptr(), sh), "df11_histogram")
+            check(df11_build_codebook_device(hists[i].data_ptr(), cap, meta[i].data_ptr(),
+                                             tables[i].data_ptr(), meta[i].data_ptr() + _META_BITS,
+                                             status[i].data_ptr(), sh),
+                  "df11_build_codebook_device")
+    meta_h = meta.cpu().numpy()                                      # round trip 1
+    st_h = status[:, 0].cpu().numpy()
+    h_all = hists.cpu().numpy().view(np.uint64)
+    cbs, sizes_l = [], []
+    for i, u in enumerate(us):
+        if int(st_h[i]):
+            raise DF11Error(int(st_h[i]), f"df11_build_codebook_device (device), matrix {i}")
+        cb = df11_codebook.from_buffer_copy(meta_h[i, :CODEBOOK_BYTES].tobytes())
+        bits = int(meta_h[i, _META_BITS:_META_BITS + 8].view(np.uint64)[0])
+        st, sizes = df11_sizes_from_bits(u.numel(), bits)
+        check(st, "df11_sizes_from_bits")
+        cbs.append(cb)
+        sizes_l.append(sizes)
+    ws_bytes = max(16, max(int(sz.workspace_bytes) for sz in sizes_l))
+    wsb = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    mats_bufs = []
+    with torch.cuda.device(dev):
+        for i, (u, sizes) in enumerate(zip(us, sizes_l)):
+            bufs = alloc_encoded(sizes, dev)
+            out = df11_encoded(stream=bufs["stream"].data_ptr(), gaps=bufs["gaps"].data_ptr(),
+                               block_pos=bufs["block_pos"].data_ptr(),
+                               sign_mantissa=bufs["sign_mantissa"].data_ptr(),
+                               block_max=status[i].data_ptr() + 4)
+            check(df11_encode_device_codebook(u.data_ptr(), u.numel(), meta[i].data_ptr(),
+                                              sizes.total_bits, out, wsb.data_ptr(), wsb.numel(),
+                                              status[i].data_ptr(), sh),
+                  "df11_encode_device_codebook")
+            mats_bufs.append(bufs)
+    st_host = status.cpu().numpy()                                   # round trip 2
+    mats = []
+    for i, (w, u) in enumerate(zip(ws, us)):
+        if check_status and int(st_host[i, 0]):
+            raise DF11Error(int(st_host[i, 0]), f"df11_encode_device_codebook (device), matrix {i}")
+        mats.append(DF11Matrix(shape=tuple(w.shape), n=u.numel(),
+                               total_bits=int(sizes_l[i].total_bits), codebook=cbs[i],
+                               sizes=sizes_l[i], tables=tables[i], hist=h_all[i].copy(),
                                max_block_codes=int(st_host[i, 1]), **mats_bufs[i]))
     return mats
 

@@ -42,7 +42,12 @@ static_assert(sizeof(DecodeTables) % 16 == 0, "tables are copied in 16-byte unit
 
 constexpr uint32_t kLutLongFlag = 1u << 26;
 constexpr uint32_t kLutCountMask = 3u << 24;
-inline constexpr uint32_t lut_entry(uint32_t syms, uint32_t count, uint32_t used) {
+#ifdef __CUDACC__
+#define DF11I_HD __host__ __device__
+#else
+#define DF11I_HD
+#endif
+DF11I_HD inline constexpr uint32_t lut_entry(uint32_t syms, uint32_t count, uint32_t used) {
   return syms | (count << 24) | (used << 28);
 }
 

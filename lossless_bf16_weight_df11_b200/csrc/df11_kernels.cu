@@ -38,6 +38,7 @@
 #include <mutex>
 
 #include "df11.h"
+#include "df11_codebook.h"
 #include "df11_internal.h"
 
 using df11i::DecodeTables;
@@ -153,6 +154,19 @@ struct EncCodebook {
   uint8_t len[256];
 };
 
+// Entry t of the encoder's codebook: {length, code left-justified in 32 bits},
+// from the launch parameters, or from a device codebook (df11_codebook) when
+// dcb is given.  A device length above 32 counts as 32; a code's bits above
+// its length fall off.
+__device__ __forceinline__ uint2 enc_entry(const EncCodebook &cb, const df11_codebook *dcb, int t) {
+  if (dcb) {
+    uint32_t L = dcb->len[t];
+    L = L > DF11_MAX_CODE_LEN ? DF11_MAX_CODE_LEN : L;
+    return make_uint2(L, L ? dcb->code[t] << (32 - L) : 0u);
+  }
+  return make_uint2(cb.len[t], cb.code[t]);
+}
+
 __device__ __forceinline__ void load_tile_values(const uint16_t *__restrict__ w, uint64_t n,
                                                  uint64_t i0, uint16_t v[16]) {
   if (i0 + 16 <= n) {
@@ -173,13 +187,13 @@ __device__ __forceinline__ void load_tile_values(const uint16_t *__restrict__ w,
 // Sum of code lengths of each tile of kEncTile values; also clears the
 // stream and gap buffers (their padding must read as zero bits).
 __global__ void __launch_bounds__(df11i::kEncThreads) enc_sum_kernel(
-    const uint16_t *__restrict__ w, uint64_t n, EncCodebook cb, uint64_t *__restrict__ tile_sum,
-    uint64_t n_tiles, uint4 *__restrict__ stream, uint64_t stream_vecs, uint4 *__restrict__ gaps,
-    uint64_t gap_vecs, uint32_t *status) {
+    const uint16_t *__restrict__ w, uint64_t n, EncCodebook cb, const df11_codebook *dcb,
+    uint64_t *__restrict__ tile_sum, uint64_t n_tiles, uint4 *__restrict__ stream,
+    uint64_t stream_vecs, uint4 *__restrict__ gaps, uint64_t gap_vecs, uint32_t *status) {
   __shared__ uint8_t s_len[256];
   __shared__ uint32_t s_warp[df11i::kEncThreads / 32];
   const int t = threadIdx.x;
-  s_len[t] = cb.len[t];
+  s_len[t] = (uint8_t)enc_entry(cb, dcb, t).x;
   const uint64_t gtid = (uint64_t)blockIdx.x * blockDim.x + t;
   const uint64_t gstride = (uint64_t)gridDim.x * blockDim.x;
   for (uint64_t i = gtid; i < stream_vecs; i += gstride) stream[i] = make_uint4(0, 0, 0, 0);
@@ -288,7 +302,7 @@ __device__ __forceinline__ void red_or_shared_if(uint32_t *p, uint32_t v, bool c
 }
 
 __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
-    const uint16_t *__restrict__ w, uint64_t n, EncCodebook cb,
+    const uint16_t *__restrict__ w, uint64_t n, EncCodebook cb, const df11_codebook *dcb,
     const uint64_t *__restrict__ tile_start, uint64_t total_bits, uint8_t *__restrict__ stream,
     uint64_t stream_alloc, uint8_t *__restrict__ gaps, uint64_t gaps_alloc,
     uint32_t *__restrict__ block_pos, uint64_t n_blocks, uint8_t *__restrict__ sign_mantissa) {
@@ -302,7 +316,7 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
   constexpr int kGapChunks = df11i::kEncTile * DF11_MAX_CODE_LEN / DF11_CHUNK_BITS + 2;
   __shared__ uint8_t s_gap[kGapChunks];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  s_lc[t] = make_uint2(cb.len[t], cb.code[t]);
+  s_lc[t] = enc_entry(cb, dcb, t);
   for (int k = t; k < kGapChunks; k += df11i::kEncThreads) s_gap[k] = 0xFFu;
   const uint64_t tile = blockIdx.x;
   const uint64_t S = tile_start[tile], E = tile_start[tile + 1];
@@ -316,6 +330,9 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
   const uint64_t i0 = tile * df11i::kEncTile + (uint64_t)t * df11i::kEncPerThread;
   load_tile_values(w, n, i0, v);
   const uint32_t nk = i0 < n ? (n - i0 < 16 ? (uint32_t)(n - i0) : 16u) : 0u;  // values of this thread
+  // every thread reads the whole code table (and later the cleared bit and
+  // gap buffers): the fills above must be complete first
+  __syncthreads();
   // code-length sum, and the length of this thread's last value (the
   // value before the next thread's first)
   uint32_t sum = 0, my_last = 0;
@@ -471,6 +488,90 @@ __global__ void __launch_bounds__(256) enc_block_max_kernel(const uint32_t *__re
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) best = max(best, __shfl_down_sync(0xffffffffu, best, d));
   if ((threadIdx.x & 31) == 0 && best) atomicMax(out, best);
+}
+
+// ============================================================ codebook on the device
+
+// One CTA of 256 threads, thread t standing for exponent t.  The ranks, the
+// normalised lengths, the canonical codes, the encoded size and the lookup
+// table are computed in parallel; the two tree constructions (Huffman, and
+// package-merge when the cap binds) run on thread 0.  Every step is the
+// shared implementation df11_build_codebook uses on the host.
+constexpr int kCbThreads = 256;
+
+__global__ void __launch_bounds__(kCbThreads) codebook_kernel(
+    const uint64_t *__restrict__ hist, uint32_t cap, df11_codebook *__restrict__ cb_out,
+    DecodeTables *__restrict__ t_out, uint64_t *__restrict__ total_bits, uint32_t *status) {
+  __shared__ df11cb::Scratch sc;
+  __shared__ df11cb::TableAux aux;
+  __shared__ df11_codebook cb;
+  __shared__ uint64_t h[256];
+  __shared__ uint32_t len_count[DF11_MAX_CODE_LEN + 1];
+  __shared__ uint64_t next[DF11_MAX_CODE_LEN + 1];
+  __shared__ uint64_t s_bits[kCbThreads / 32];
+  __shared__ int s_ok;
+  const int t = threadIdx.x;
+  h[t] = hist[t];
+  if (t <= (int)DF11_MAX_CODE_LEN) len_count[t] = 0;
+  __syncthreads();
+  const bool present = h[t] != 0;
+  if (present) sc.hist_sorted[df11cb::ascending_rank(h, t)] = h[t];
+  const int m = __syncthreads_count(present);
+  if (t == 0) {
+    int longest = m ? df11cb::huffman_depths(m, sc) : 0;
+    if (longest > (int)cap) longest = df11cb::package_merge_depths(m, (int)cap, sc);
+    s_ok = longest >= 0;
+    if (s_ok) {
+      for (int i = 0; i < m; ++i) ++len_count[sc.depth[i]];
+      df11cb::first_codes(len_count, next);
+    }
+  }
+  __syncthreads();
+  if (!s_ok) {
+    if (t == 0) set_status(status, DF11_ERR_INVALID_ARG);
+    return;
+  }
+  uint32_t *tz = reinterpret_cast<uint32_t *>(t_out);  // padding included
+  for (uint32_t i = t; i < sizeof(DecodeTables) / 4; i += kCbThreads) tz[i] = 0u;
+  cb.len[t] = df11cb::normalised_length(h, len_count, t);
+  __syncthreads();
+  cb.code[t] = df11cb::canonical_code(cb.len, next, t);
+  uint64_t bits = h[t] * cb.len[t];
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) bits += __shfl_down_sync(0xffffffffu, bits, d);
+  if ((t & 31) == 0) s_bits[t >> 5] = bits;
+  __syncthreads();
+  if (t == 0) {
+    uint64_t tot = 0;
+    uint32_t mx = 0, mn = m ? DF11_MAX_CODE_LEN : 0u;
+    for (int i = 0; i < kCbThreads / 32; ++i) tot += s_bits[i];
+    for (int i = 0; i < 256; ++i)
+      if (cb.len[i]) {
+        mx = cb.len[i] > mx ? cb.len[i] : mx;
+        mn = cb.len[i] < mn ? cb.len[i] : mn;
+      }
+    cb.max_len = mx;
+    cb.min_len = mn;
+    cb.n_symbols = (uint32_t)m;
+    cb.cap = cap;
+    *total_bits = tot;
+    s_ok = df11cb::table_header(&cb, t_out, aux) == DF11_OK;
+  }
+  __syncthreads();
+  if (!s_ok) {  // cannot happen for a codebook built here
+    if (t == 0) set_status(status, DF11_ERR_INVALID_ARG);
+    return;
+  }
+  for (uint32_t v = t; v < (uint32_t)df11i::kLutSize; v += kCbThreads)
+    t_out->lut[v] = df11cb::lut_entry_for(*t_out, aux, cb.max_len, v);
+  cb_out->len[t] = cb.len[t];
+  cb_out->code[t] = cb.code[t];
+  if (t == 0) {
+    cb_out->max_len = cb.max_len;
+    cb_out->min_len = cb.min_len;
+    cb_out->n_symbols = cb.n_symbols;
+    cb_out->cap = cb.cap;
+  }
 }
 
 // ============================================================ decode
@@ -1322,54 +1423,114 @@ extern "C" df11_status df11_histogram(const uint16_t *d_w, uint64_t n, uint64_t 
   return launch_status();
 }
 
+namespace {
+
+// The codebook of the launch parameters: lengths up to the format's limit,
+// codes that fit their length, left-justified in 32 bits for the packer.
+df11_status host_enc_codebook(const df11_codebook *cb, EncCodebook *ecb) {
+  for (int i = 0; i < 256; ++i) {
+    const uint32_t L = cb->len[i];
+    if (L > DF11_MAX_CODE_LEN || (L < 32 && (cb->code[i] >> L) != 0)) return DF11_ERR_INVALID_ARG;
+    ecb->code[i] = L ? cb->code[i] << (32 - L) : 0u;
+    ecb->len[i] = (uint8_t)L;
+  }
+  return DF11_OK;
+}
+
+df11_status check_encode_out(const uint16_t *d_w, uint64_t n, uint64_t total_bits,
+                             const df11_encoded *out) {
+  if ((n && (!d_w || !aligned16(d_w))) || !out->stream || !out->gaps || !out->block_pos ||
+      !out->sign_mantissa)
+    return DF11_ERR_INVALID_ARG;
+  if (!aligned16(out->stream) || !aligned16(out->gaps) || !aligned16(out->block_pos) ||
+      !aligned16(out->sign_mantissa))
+    return DF11_ERR_INVALID_ARG;
+  if (total_bits > n * (uint64_t)DF11_MAX_CODE_LEN || (n && total_bits < n))
+    return DF11_ERR_INVALID_ARG;
+  return DF11_OK;
+}
+
+// Length sums per tile (clearing the stream and gap buffers), their prefix
+// sum, packing, and the largest block.  ws: n_tiles + 1 uint64 of scratch.
+df11_status launch_encode(const uint16_t *d_w, uint64_t n, const EncCodebook &ecb,
+                          const df11_codebook *dcb, uint64_t total_bits, const df11_encoded *out,
+                          uint64_t *ws, uint32_t *d_status, cudaStream_t s) {
+  const uint64_t n_tiles = cdiv(n, df11i::kEncTile);
+  const uint64_t C = cdiv(total_bits, 64);
+  const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
+  // the stream and gap allocations of the format (df11_encoded_sizes)
+  const uint64_t stream_alloc = (uint64_t)kBlockStreamBytes * B + 16;
+  const uint64_t gaps_alloc = (uint64_t)kBlockGapBytes * B + 16;
+  const uint64_t grid1 = std::max<uint64_t>(n_tiles, 1);
+  enc_sum_kernel<<<(unsigned)grid1, df11i::kEncThreads, 0, s>>>(
+      d_w, n, ecb, dcb, ws, n_tiles, reinterpret_cast<uint4 *>(out->stream), stream_alloc / 16,
+      reinterpret_cast<uint4 *>(out->gaps), gaps_alloc / 16, d_status);
+  enc_scan_kernel<<<1, kScanThreads, 0, s>>>(ws, n_tiles, total_bits, out->block_pos, B, n,
+                                            d_status, out->block_max);
+  if (n_tiles)
+    enc_pack_kernel<<<(unsigned)n_tiles, df11i::kEncThreads, 0, s>>>(
+        d_w, n, ecb, dcb, ws, total_bits, out->stream, stream_alloc, out->gaps, gaps_alloc,
+        out->block_pos, B, out->sign_mantissa);
+  if (out->block_max && B)
+    enc_block_max_kernel<<<(unsigned)std::min<uint64_t>(cdiv(B, 256), 1024), 256, 0, s>>>(
+        out->block_pos, B, out->block_max);
+  return launch_status();
+}
+
+}  // namespace
+
 extern "C" df11_status df11_encode(const uint16_t *d_w, uint64_t n, const df11_codebook *cb,
                                    uint64_t total_bits, const df11_encoded *out, void *d_workspace,
                                    size_t workspace_bytes, uint32_t *d_status,
                                    df11_stream_t stream) {
   if (!cb || !out || !d_status) return DF11_ERR_INVALID_ARG;
   if (n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
-  if ((n && (!d_w || !aligned16(d_w))) || !out->stream || !out->gaps || !out->block_pos ||
-      !out->sign_mantissa || !d_workspace)
+  df11_status st = check_encode_out(d_w, n, total_bits, out);
+  if (st != DF11_OK) return st;
+  if (!d_workspace || !aligned16(d_workspace)) return DF11_ERR_INVALID_ARG;
+  if (workspace_bytes < 8 * (cdiv(n, df11i::kEncTile) + 1)) return DF11_ERR_INVALID_ARG;
+  EncCodebook ecb;
+  if ((st = host_enc_codebook(cb, &ecb)) != DF11_OK) return st;
+  int dev, sms;
+  if ((st = device_info(&dev, &sms)) != DF11_OK) return st;
+  return launch_encode(d_w, n, ecb, nullptr, total_bits, out,
+                       reinterpret_cast<uint64_t *>(d_workspace), d_status,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" df11_status df11_encode_device_codebook(const uint16_t *d_w, uint64_t n,
+                                                   const df11_codebook *d_cb, uint64_t total_bits,
+                                                   const df11_encoded *out, void *d_workspace,
+                                                   size_t workspace_bytes, uint32_t *d_status,
+                                                   df11_stream_t stream) {
+  if (!d_cb || !out || !d_status || ((uintptr_t)d_cb & 3u)) return DF11_ERR_INVALID_ARG;
+  if (n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
+  df11_status st = check_encode_out(d_w, n, total_bits, out);
+  if (st != DF11_OK) return st;
+  if (!d_workspace || !aligned16(d_workspace)) return DF11_ERR_INVALID_ARG;
+  if (workspace_bytes < 8 * (cdiv(n, df11i::kEncTile) + 1)) return DF11_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_info(&dev, &sms)) != DF11_OK) return st;
+  EncCodebook unused{};
+  return launch_encode(d_w, n, unused, d_cb, total_bits, out,
+                       reinterpret_cast<uint64_t *>(d_workspace), d_status,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" df11_status df11_build_codebook_device(const uint64_t *d_hist256, uint32_t cap,
+                                                  df11_codebook *d_cb, void *d_tables,
+                                                  uint64_t *d_total_bits, uint32_t *d_status,
+                                                  df11_stream_t stream) {
+  if (!d_hist256 || !d_cb || !d_tables || !d_total_bits || cap < 1 || cap > DF11_MAX_CODE_LEN)
     return DF11_ERR_INVALID_ARG;
-  if (!aligned16(out->stream) || !aligned16(out->gaps) || !aligned16(out->block_pos) ||
-      !aligned16(out->sign_mantissa) || !aligned16(d_workspace))
+  if (((uintptr_t)d_hist256 & 7u) || ((uintptr_t)d_cb & 3u) || !aligned16(d_tables) ||
+      ((uintptr_t)d_total_bits & 7u))
     return DF11_ERR_INVALID_ARG;
-  if (total_bits > n * (uint64_t)DF11_MAX_CODE_LEN || (n && total_bits < n))
-    return DF11_ERR_INVALID_ARG;
-  const uint64_t n_tiles = cdiv(n, df11i::kEncTile);
-  if (workspace_bytes < 8 * (n_tiles + 1)) return DF11_ERR_INVALID_ARG;
   int dev, sms;
   df11_status st = device_info(&dev, &sms);
   if (st != DF11_OK) return st;
-  EncCodebook ecb;
-  for (int i = 0; i < 256; ++i) {
-    // lengths up to the format's limit, codes that fit their length;
-    // the packer takes codes left-justified in 32 bits
-    const uint32_t L = cb->len[i];
-    if (L > DF11_MAX_CODE_LEN || (L < 32 && (cb->code[i] >> L) != 0)) return DF11_ERR_INVALID_ARG;
-    ecb.code[i] = L ? cb->code[i] << (32 - L) : 0u;
-    ecb.len[i] = (uint8_t)L;
-  }
-  const uint64_t C = cdiv(total_bits, 64);
-  const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
-  // the stream and gap allocations of the format (df11_encoded_sizes)
-  const uint64_t stream_alloc = (uint64_t)kBlockStreamBytes * B + 16;
-  const uint64_t gaps_alloc = (uint64_t)kBlockGapBytes * B + 16;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  auto *ws = reinterpret_cast<uint64_t *>(d_workspace);
-  const uint64_t grid1 = std::max<uint64_t>(n_tiles, 1);
-  enc_sum_kernel<<<(unsigned)grid1, df11i::kEncThreads, 0, s>>>(
-      d_w, n, ecb, ws, n_tiles, reinterpret_cast<uint4 *>(out->stream), stream_alloc / 16,
-      reinterpret_cast<uint4 *>(out->gaps), gaps_alloc / 16, d_status);
-  enc_scan_kernel<<<1, kScanThreads, 0, s>>>(ws, n_tiles, total_bits, out->block_pos, B, n,
-                                            d_status, out->block_max);
-  if (n_tiles)
-    enc_pack_kernel<<<(unsigned)n_tiles, df11i::kEncThreads, 0, s>>>(
-        d_w, n, ecb, ws, total_bits, out->stream, stream_alloc, out->gaps, gaps_alloc,
-        out->block_pos, B, out->sign_mantissa);
-  if (out->block_max && B)
-    enc_block_max_kernel<<<(unsigned)std::min<uint64_t>(cdiv(B, 256), 1024), 256, 0, s>>>(
-        out->block_pos, B, out->block_max);
+  codebook_kernel<<<1, kCbThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      d_hist256, cap, d_cb, reinterpret_cast<DecodeTables *>(d_tables), d_total_bits, d_status);
   return launch_status();
 }
 
@@ -1541,51 +1702,17 @@ extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
                                              df11_stream_t stream) {
   if (!cb || !out || !d_status) return DF11_ERR_INVALID_ARG;
   if (n > DF11_STATIC_WS_MAX_N) return DF11_ERR_TOO_LARGE;
-  if ((n && (!d_w || !aligned16(d_w))) || !out->stream || !out->gaps || !out->block_pos ||
-      !out->sign_mantissa)
-    return DF11_ERR_INVALID_ARG;
-  if (!aligned16(out->stream) || !aligned16(out->gaps) || !aligned16(out->block_pos) ||
-      !aligned16(out->sign_mantissa))
-    return DF11_ERR_INVALID_ARG;
-  if (total_bits > n * (uint64_t)DF11_MAX_CODE_LEN || (n && total_bits < n))
-    return DF11_ERR_INVALID_ARG;
-  const uint64_t n_tiles = cdiv(n, df11i::kEncTile);
-  if (n_tiles + 1 > kStaticTiles) return DF11_ERR_TOO_LARGE;
-  int dev, sms;
-  df11_status st = device_info(&dev, &sms);
+  df11_status st = check_encode_out(d_w, n, total_bits, out);
   if (st != DF11_OK) return st;
-  uint64_t *ws = nullptr;
-  st = static_scratch(dev, &ws);
-  if (st != DF11_OK) return st;
+  if (cdiv(n, df11i::kEncTile) + 1 > kStaticTiles) return DF11_ERR_TOO_LARGE;
   EncCodebook ecb;
-  for (int i = 0; i < 256; ++i) {
-    // lengths up to the format's limit, codes that fit their length;
-    // the packer takes codes left-justified in 32 bits
-    const uint32_t L = cb->len[i];
-    if (L > DF11_MAX_CODE_LEN || (L < 32 && (cb->code[i] >> L) != 0)) return DF11_ERR_INVALID_ARG;
-    ecb.code[i] = L ? cb->code[i] << (32 - L) : 0u;
-    ecb.len[i] = (uint8_t)L;
-  }
-  const uint64_t C = cdiv(total_bits, 64);
-  const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
-  // the stream and gap allocations of the format (df11_encoded_sizes)
-  const uint64_t stream_alloc = (uint64_t)kBlockStreamBytes * B + 16;
-  const uint64_t gaps_alloc = (uint64_t)kBlockGapBytes * B + 16;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = host_enc_codebook(cb, &ecb)) != DF11_OK) return st;
+  int dev, sms;
+  if ((st = device_info(&dev, &sms)) != DF11_OK) return st;
+  uint64_t *ws = nullptr;
+  if ((st = static_scratch(dev, &ws)) != DF11_OK) return st;
   // nothing in the array needs clearing: every tile offset a call reads is
   // written earlier in the same call
-  const uint64_t grid1 = std::max<uint64_t>(n_tiles, 1);
-  enc_sum_kernel<<<(unsigned)grid1, df11i::kEncThreads, 0, s>>>(
-      d_w, n, ecb, ws, n_tiles, reinterpret_cast<uint4 *>(out->stream), stream_alloc / 16,
-      reinterpret_cast<uint4 *>(out->gaps), gaps_alloc / 16, d_status);
-  enc_scan_kernel<<<1, kScanThreads, 0, s>>>(ws, n_tiles, total_bits, out->block_pos, B, n,
-                                            d_status, out->block_max);
-  if (n_tiles)
-    enc_pack_kernel<<<(unsigned)n_tiles, df11i::kEncThreads, 0, s>>>(
-        d_w, n, ecb, ws, total_bits, out->stream, stream_alloc, out->gaps, gaps_alloc,
-        out->block_pos, B, out->sign_mantissa);
-  if (out->block_max && B)
-    enc_block_max_kernel<<<(unsigned)std::min<uint64_t>(cdiv(B, 256), 1024), 256, 0, s>>>(
-        out->block_pos, B, out->block_max);
-  return launch_status();
+  return launch_encode(d_w, n, ecb, nullptr, total_bits, out, ws, d_status,
+                       reinterpret_cast<cudaStream_t>(stream));
 }

@@ -216,3 +216,50 @@ def test_validate_accepts_oracle_metadata_and_rejects_corruption(lib):
     if tail[-1] > enc.total_bits - 64 * (C - 1):
         gp = oracle.pack_gaps(tail)
         assert val(gaps=gp) == df11.DF11_ERR_CORRUPT
+
+
+def test_sizes_from_bits_equal_encoded_sizes():
+    g = np.random.default_rng(8)
+    for _ in range(200):
+        h = np.zeros(256, np.uint64)
+        m = int(g.integers(1, 257))
+        h[g.choice(256, m, replace=False)] = g.integers(1, 10 ** int(g.integers(1, 6)), m)
+        st, cb = df11.df11_build_codebook(h, int(g.integers(8, 33)))
+        if st:
+            continue
+        n = int(h.sum())
+        st, a = df11.df11_encoded_sizes(cb, h, n)
+        assert st == df11.DF11_OK
+        st, b = df11.df11_sizes_from_bits(n, a.total_bits)
+        assert st == df11.DF11_OK
+        assert bytes(a) == bytes(b)
+    assert df11.df11_sizes_from_bits(10, 9)[0] == df11.DF11_ERR_INVALID_ARG     # < 1 bit a value
+    assert df11.df11_sizes_from_bits(10, 321)[0] == df11.DF11_ERR_INVALID_ARG   # > 32 bits a value
+    assert df11.df11_sizes_from_bits(2 ** 32, 2 ** 33)[0] == df11.DF11_ERR_TOO_LARGE
+    assert df11.df11_sizes_from_bits(0, 0)[0] == df11.DF11_OK
+
+
+def test_device_codebook_launchers_check_arguments_first():
+    """Argument errors are returned before any device query."""
+    assert df11.df11_build_codebook_device(0, 12, 16, 16, 16, 0, 0) == df11.DF11_ERR_INVALID_ARG
+    assert df11.df11_build_codebook_device(16, 0, 16, 16, 16, 0, 0) == df11.DF11_ERR_INVALID_ARG
+    assert df11.df11_build_codebook_device(16, 33, 16, 16, 16, 0, 0) == df11.DF11_ERR_INVALID_ARG
+    assert df11.df11_build_codebook_device(16, 12, 16, 24, 16, 0, 0) == df11.DF11_ERR_INVALID_ARG
+    out = df11.df11_encoded(stream=16, gaps=16, block_pos=16, sign_mantissa=16, block_max=0)
+    assert df11.df11_encode_device_codebook(16, 100, 0, 300, out, 16, 4096, 16, 0) == \
+        df11.DF11_ERR_INVALID_ARG
+    assert df11.df11_encode_device_codebook(16, 100, 18, 300, out, 16, 4096, 16, 0) == \
+        df11.DF11_ERR_INVALID_ARG
+    assert df11.df11_encode_device_codebook(16, 100, 16, 99, out, 16, 4096, 16, 0) == \
+        df11.DF11_ERR_INVALID_ARG
+    assert df11.df11_encode_device_codebook(16, 2 ** 33, 16, 2 ** 34, out, 16, 4096, 16, 0) == \
+        df11.DF11_ERR_TOO_LARGE
+
+
+def test_shared_codebook_code_matches_the_oracle_when_the_cap_binds():
+    """The host builder (shared with the device kernel) against the oracle on
+    Fibonacci counts at every cap from the smallest feasible to 32."""
+    f = workloads.fibonacci_counts(34)
+    h = hist_from(f, first=50)
+    for cap in range(6, 33):
+        assert_same_codebook(h, cap)
