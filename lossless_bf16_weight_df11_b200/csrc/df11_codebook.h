@@ -241,23 +241,31 @@ DF11_HD inline df11_status build_codebook(const uint64_t *hist, uint32_t cap, df
   return DF11_OK;
 }
 
-// Everything of the decode tables but the lookup table; t must be zeroed.
-DF11_HD inline df11_status table_header(const df11_codebook *cb, df11i::DecodeTables *t,
-                                        TableAux &aux) {
-  for (int l = 0; l <= (int)DF11_MAX_CODE_LEN; ++l) aux.count[l] = aux.first[l] = 0;
-  for (int l = 0; l <= (int)DF11_MAX_CODE_LEN + 1; ++l) aux.rank_start[l] = 0;
+// The per-length part of the decode tables: counts, canonical first codes,
+// rank starts, limit/base, and the scalar fields (everything but sym[] and
+// the lookup table); t must be zeroed.  DF11_ERR_INVALID_ARG for a length
+// above 32 or codes that are not canonical.
+DF11_HD inline df11_status table_lengths(const df11_codebook *cb, df11i::DecodeTables *t,
+                                         TableAux &aux) {
+  bool seen[DF11_MAX_CODE_LEN + 1];
+  for (int l = 0; l <= (int)DF11_MAX_CODE_LEN; ++l) {
+    aux.count[l] = aux.first[l] = 0;
+    seen[l] = false;
+  }
   for (int s = 0; s < kMaxSyms; ++s) {
-    if (cb->len[s] > DF11_MAX_CODE_LEN) return DF11_ERR_INVALID_ARG;
-    if (cb->len[s]) ++aux.count[cb->len[s]];
+    const unsigned L = cb->len[s];
+    if (L > DF11_MAX_CODE_LEN) return DF11_ERR_INVALID_ARG;
+    if (!L) continue;
+    ++aux.count[L];
+    if (!seen[L]) {  // the smallest value of each length holds its first code
+      seen[L] = true;
+      aux.first[L] = cb->code[s];
+    }
   }
   int r = 0;
-  for (unsigned l = 1; l <= DF11_MAX_CODE_LEN; ++l) {
+  for (unsigned l = 0; l <= DF11_MAX_CODE_LEN + 1; ++l) {
     aux.rank_start[l] = r;
-    for (int s = 0; s < kMaxSyms; ++s)
-      if (cb->len[s] == l) {
-        if (r == aux.rank_start[l]) aux.first[l] = cb->code[s];
-        t->sym[r++] = (uint8_t)s;
-      }
+    if (l >= 1 && l <= DF11_MAX_CODE_LEN) r += (int)aux.count[l];
   }
   // a length without codes still gets the canonical start so limits stay monotone
   uint64_t c = 0;
@@ -271,11 +279,34 @@ DF11_HD inline df11_status table_header(const df11_codebook *cb, df11i::DecodeTa
     t->base[l] = (uint32_t)((int64_t)aux.rank_start[l] - (int64_t)aux.first[l]);
   }
   t->limit[0] = 0;
-  for (int s = 0; s < kMaxSyms; ++s) t->codelen[s] = cb->len[s];
   t->max_len = cb->max_len;
   t->min_len = cb->min_len;
   t->n_symbols = cb->n_symbols;
   t->lut_bits = df11i::kLutBits;
+  return DF11_OK;
+}
+
+// The per-value part: value s (with a code) goes to sym[] at its rank in
+// (length asc, value asc) order, and its length to codelen[s].
+DF11_HD inline void table_value(const df11_codebook *cb, df11i::DecodeTables *t, int s) {
+  const unsigned L = cb->len[s];
+  t->codelen[s] = (uint8_t)L;
+  if (!L) return;
+  int r = 0;
+  for (int u = 0; u < kMaxSyms; ++u) {
+    const unsigned Lu = cb->len[u];
+    r += Lu && (Lu < L || (Lu == L && u < s));
+  }
+  t->sym[r] = (uint8_t)s;
+}
+
+// Everything of the decode tables but the lookup table, sequentially; t must
+// be zeroed.
+DF11_HD inline df11_status table_header(const df11_codebook *cb, df11i::DecodeTables *t,
+                                        TableAux &aux) {
+  const df11_status st = table_lengths(cb, t, aux);
+  if (st != DF11_OK) return st;
+  for (int s = 0; s < kMaxSyms; ++s) table_value(cb, t, s);
   return DF11_OK;
 }
 

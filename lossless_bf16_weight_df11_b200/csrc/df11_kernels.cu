@@ -555,13 +555,15 @@ __global__ void __launch_bounds__(kCbThreads) codebook_kernel(
     cb.n_symbols = (uint32_t)m;
     cb.cap = cap;
     *total_bits = tot;
-    s_ok = df11cb::table_header(&cb, t_out, aux) == DF11_OK;
+    s_ok = df11cb::table_lengths(&cb, t_out, aux) == DF11_OK;
   }
   __syncthreads();
   if (!s_ok) {  // cannot happen for a codebook built here
     if (t == 0) set_status(status, DF11_ERR_INVALID_ARG);
     return;
   }
+  df11cb::table_value(&cb, t_out, t);
+  __syncthreads();
   for (uint32_t v = t; v < (uint32_t)df11i::kLutSize; v += kCbThreads)
     t_out->lut[v] = df11cb::lut_entry_for(*t_out, aux, cb.max_len, v);
   cb_out->len[t] = cb.len[t];

@@ -176,7 +176,25 @@ def test_decode_table_against_oracle_codes(lib, which):
     ln, code, cb = lib_codebook(h)
     oln, ocode = oracle.codebook(h)
     codes_by_str = {format(int(ocode[s]), f"0{int(oln[s])}b"): s for s in range(256) if oln[s]}
-    lut = tables_of(cb)[: 4 * 4096].view(np.uint32)
+    tab = tables_of(cb)
+    lut = tab[: 4 * 4096].view(np.uint32)
+    # the long-code arrays: limit u64[33], base u32[33], codelen u8[256], sym u8[256], then
+    # max_len, min_len, n_symbols, lut_bits
+    limit = tab[16384:16384 + 264].view(np.uint64)
+    base = tab[16648:16648 + 132].view(np.uint32)
+    codelen = tab[16780:16780 + 256]
+    sym = tab[17036:17036 + 256]
+    max_len, min_len, n_sym, lut_bits = tab[17292:17308].view(np.uint32)
+    assert np.array_equal(codelen, oln)
+    nz = oln[oln > 0]
+    assert (max_len, min_len, n_sym, lut_bits) == (nz.max(), nz.min(), nz.size, 12)
+    for L in range(1, 33):
+        at_L = [s_ for s_ in range(256) if oln[s_] == L]
+        for s_ in at_L:   # canonical decoding of a long code: sym[code + base[L]]
+            assert sym[(int(ocode[s_]) + int(base[L])) % 2 ** 32] == s_
+        if at_L:
+            first = min(int(ocode[s_]) for s_ in at_L)
+            assert int(limit[L]) == (first + len(at_L)) << (32 - L)
     for v in range(4096):
         syms, used = greedy_window(codes_by_str, format(v, "012b"))
         e = int(lut[v])
