@@ -186,3 +186,79 @@ def test_decode_is_repeatable_in_a_batch_of_the_block(rans):
         outs = rans.decompress_block(ms)
         for x, y in zip(xs, outs):
             assert torch.equal(y.view(torch.int16).reshape(-1), to_dev(x))
+
+
+GUARD = 4096   # bytes on each side, a multiple of 16
+PATTERN = 0xA5
+
+
+class Guarded:
+    def __init__(self, nbytes, fill=PATTERN):
+        self.nbytes = int(nbytes)
+        self.full = torch.full((self.nbytes + 2 * GUARD,), PATTERN, dtype=torch.uint8, device="cuda")
+        self.inner = self.full[GUARD:GUARD + self.nbytes]
+        if fill != PATTERN:
+            self.inner.fill_(fill)
+
+    @property
+    def ptr(self):
+        return self.inner.data_ptr()
+
+    def margins_intact(self):
+        f = self.full.cpu().numpy()
+        return bool((f[:GUARD] == PATTERN).all() and (f[GUARD + self.nbytes:] == PATTERN).all())
+
+
+@pytest.mark.parametrize("name,gen", [
+    ("fibonacci_rare", lambda: workloads.fibonacci_exponents(30)[: 3 * 16384 + 999]),
+    ("ragged_16385", lambda: workloads.random_bf16(16385, seed=21)),
+    ("uniform_unstaged", lambda: workloads.shuffled_patterns(copies=1, seed=5)),
+    ("seventeen", lambda: workloads.random_bf16(17, seed=22)),
+], ids=lambda v: v if isinstance(v, str) else "")
+def test_encode_and_decode_stay_inside_their_buffers(df11, name, gen):
+    """Every buffer of the C ABI calls sits between guard bands: encode
+    writes only its outputs (exactly the format's bytes), decode only its
+    output, and neither touches its inputs."""
+    x = np.ascontiguousarray(gen(), np.uint16).reshape(-1)
+    n = x.size
+    units = df11.df11_rans_units(n)
+    w = Guarded(2 * n)
+    w.inner.copy_(torch.from_numpy(x.view(np.uint8).copy()).cuda())
+    hist = torch.empty(256, dtype=torch.int64, device="cuda")
+    df11.check(df11.df11_histogram(w.ptr, n, hist.data_ptr(), 0))
+    st, freq = df11.df11_rans_freqs(hist.cpu().numpy().view(np.uint64))
+    df11.check(st)
+    host_t = np.zeros(df11.RANS_TABLES_BYTES, np.uint8)
+    df11.check(df11.df11_rans_build_tables(freq, host_t.ctypes.data, host_t.size))
+    tables = Guarded(host_t.size)
+    tables.inner.copy_(torch.from_numpy(host_t).cuda())
+    uw, off = Guarded(4 * units, fill=0x5A), Guarded(4 * (units + 1), fill=0x5A)
+    status = Guarded(16, fill=0)
+    df11.check(df11.df11_rans_encode_sizes(w.ptr, n, tables.ptr, uw.ptr, off.ptr, status.ptr, 0))
+    torch.cuda.synchronize()
+    total16 = int(off.inner.cpu().numpy().view(np.uint32)[units])
+    stream, sm = Guarded(16 * total16, fill=0x5A), Guarded(n, fill=0x5A)
+    df11.check(df11.df11_rans_encode(w.ptr, n, tables.ptr, uw.ptr, off.ptr, stream.ptr, sm.ptr,
+                                     status.ptr, 0))
+    torch.cuda.synchronize()
+    assert int(status.inner.cpu().numpy().view(np.uint32)[0]) == 0
+    for g, what in ((w, "input"), (tables, "tables"), (uw, "unit words"), (off, "off16"),
+                    (stream, "stream"), (sm, "sign/mantissa"), (status, "status")):
+        assert g.margins_intact(), f"encode wrote outside {what}"
+    enc = oracle.rans_encode(x)
+    assert np.array_equal(stream.inner.cpu().numpy(), enc.stream)
+    assert np.array_equal(off.inner.cpu().numpy().view(np.uint32), enc.off16)
+    assert np.array_equal(sm.inner.cpu().numpy(), enc.sign_mantissa)
+    before = {k: g.full.clone() for k, g in (("stream", stream), ("off16", off), ("sm", sm),
+                                               ("tables", tables))}
+    out = Guarded(2 * n, fill=0)
+    st2 = Guarded(16, fill=0)
+    m = df11.df11_rans_matrix(n=n, stream=stream.ptr, off16=off.ptr, sign_mantissa=sm.ptr,
+                              tables=tables.ptr)
+    df11.check(df11.df11_rans_decode_batch([m], [out.ptr], st2.ptr, 0))
+    torch.cuda.synchronize()
+    assert int(st2.inner.cpu().numpy().view(np.uint32)[0]) == 0
+    assert out.margins_intact() and st2.margins_intact()
+    for k, g in (("stream", stream), ("off16", off), ("sm", sm), ("tables", tables)):
+        assert torch.equal(g.full, before[k]), f"decode modified its input {k}"
+    assert np.array_equal(out.inner.cpu().numpy().view(np.uint16), x)
