@@ -113,6 +113,28 @@ df11_status df11_rans_encode(const uint16_t *d_w, uint64_t n, const void *d_tabl
                              uint8_t *d_stream, uint8_t *d_sign_mantissa, uint32_t *d_status,
                              df11_stream_t stream);
 
+/*
+ * df11_rans_validate -- host.  Checks stored rANS metadata before it is
+ * trusted, without decoding:
+ *   - off16 has U + 1 entries, starts at 0, never decreases, and its last
+ *     entry times 16 equals stream_bytes;
+ *   - every unit holds its 144-byte header and at most one word per value
+ *     (plus padding below 16 bytes);
+ *   - each unit's segment word starts begin at 0, never decrease, and stay
+ *     within the unit's words;
+ *   - every initial state is at least 2^16 (the encoder never ends below),
+ *     and a state that codes no value (lanes past n in the last unit) is
+ *     exactly 2^16.
+ *   h_stream  the stream (host copy), stream_bytes bytes.
+ *   h_off16   off16_count entries (host copy).
+ * DF11_ERR_INVALID_ARG for null pointers or a wrong off16_count,
+ * DF11_ERR_TOO_LARGE for n > DF11_MAX_N, DF11_ERR_CORRUPT otherwise.
+ * What only a decode can check (every word read, states back at 2^16) is
+ * left to df11_rans_decode_batch.
+ */
+df11_status df11_rans_validate(uint64_t n, const uint8_t *h_stream, uint64_t stream_bytes,
+                               const uint32_t *h_off16, uint64_t off16_count);
+
 /* One rANS-coded matrix (host struct of device pointers). */
 typedef struct {
   uint64_t n;

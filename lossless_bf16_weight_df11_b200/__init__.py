@@ -124,6 +124,7 @@ def _declare(lib):
         "df11_rans_build_tables": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _vp,
                                                   ctypes.c_size_t]),
         "df11_rans_units": (_u64, [_u64]),
+        "df11_rans_validate": (ctypes.c_int, [_u64, _vp, _u64, _vp, _u64]),
         "df11_rans_encode_sizes": (ctypes.c_int, [_vp, _u64, _vp, _vp, _vp, _vp, _vp]),
         "df11_rans_encode": (ctypes.c_int, [_vp, _u64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
         "df11_rans_decode_batch": (ctypes.c_int, [ctypes.POINTER(df11_rans_matrix), _u32,
@@ -311,3 +312,9 @@ def df11_rans_decode_batch(ms, d_outs, d_status: int, stream: int = 0) -> int:
     arr = (df11_rans_matrix * max(1, len(ms)))(*ms)
     outs = (ctypes.c_void_p * max(1, len(d_outs)))(*[int(p) for p in d_outs])
     return load().df11_rans_decode_batch(arr, len(ms), outs, d_status, stream)
+
+
+def df11_rans_validate(n: int, h_stream: int, stream_bytes: int, h_off16: int,
+                       off16_count: int) -> int:
+    """Host check of rANS metadata (host copies); see include/df11_rans.h."""
+    return load().df11_rans_validate(n, h_stream, stream_bytes, h_off16, off16_count)

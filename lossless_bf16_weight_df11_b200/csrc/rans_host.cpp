@@ -96,3 +96,39 @@ extern "C" df11_status df11_rans_build_tables(const uint32_t freq[256], void *h_
 extern "C" uint64_t df11_rans_units(uint64_t n) {
   return (n + DF11_RANS_UNIT - 1) / DF11_RANS_UNIT;
 }
+
+extern "C" df11_status df11_rans_validate(uint64_t n, const uint8_t *h_stream,
+                                          uint64_t stream_bytes, const uint32_t *h_off16,
+                                          uint64_t off16_count) {
+  if (n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
+  const uint64_t units = df11_rans_units(n);
+  if (!h_off16 || off16_count != units + 1 || (stream_bytes && !h_stream))
+    return DF11_ERR_INVALID_ARG;
+  if (h_off16[0] != 0 || (uint64_t)h_off16[units] * 16 != stream_bytes) return DF11_ERR_CORRUPT;
+  // every offset first, so that every unit read below lies inside the stream
+  for (uint64_t u = 0; u < units; ++u)
+    if (h_off16[u + 1] < h_off16[u]) return DF11_ERR_CORRUPT;
+  const uint64_t max_unit = DF11_RANS_HEADER_BYTES + 2ull * DF11_RANS_UNIT + 15;
+  for (uint64_t u = 0; u < units; ++u) {
+    const uint64_t bytes = (uint64_t)(h_off16[u + 1] - h_off16[u]) * 16;
+    if (bytes < DF11_RANS_HEADER_BYTES || bytes > max_unit) return DF11_ERR_CORRUPT;
+    const uint8_t *p = h_stream + (uint64_t)h_off16[u] * 16;
+    const uint64_t words = (bytes - DF11_RANS_HEADER_BYTES) / 2;
+    uint64_t prev = 0;
+    for (unsigned g = 0; g < DF11_RANS_SEGMENTS; ++g) {
+      const uint64_t st = (uint64_t)p[128 + 2 * g] | (uint64_t)p[129 + 2 * g] << 8;
+      if ((g == 0 && st != 0) || st < prev || st > words) return DF11_ERR_CORRUPT;
+      prev = st;
+    }
+    // values of this unit: lane l codes ceil((m - l) / 32) of them
+    const uint64_t m = n - u * DF11_RANS_UNIT < DF11_RANS_UNIT ? n - u * DF11_RANS_UNIT
+                                                               : DF11_RANS_UNIT;
+    for (unsigned l = 0; l < DF11_RANS_LANES; ++l) {
+      const uint32_t x = (uint32_t)p[4 * l] | (uint32_t)p[4 * l + 1] << 8 |
+                         (uint32_t)p[4 * l + 2] << 16 | (uint32_t)p[4 * l + 3] << 24;
+      if (x < (1u << 16)) return DF11_ERR_CORRUPT;
+      if (l >= m && x != (1u << 16)) return DF11_ERR_CORRUPT;
+    }
+  }
+  return DF11_OK;
+}

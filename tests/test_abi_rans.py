@@ -114,3 +114,58 @@ def test_launchers_reject_bad_arguments_without_a_device():
     assert df11.df11_rans_decode_batch([m], [16], 0, 0) == df11.DF11_ERR_INVALID_ARG
     m = df11.df11_rans_matrix(n=2 ** 33, stream=16, off16=16, sign_mantissa=16, tables=16)
     assert df11.df11_rans_decode_batch([m], [16], 0, 0) == df11.DF11_ERR_TOO_LARGE
+
+
+def validate(enc, stream=None, off16=None, n=None):
+    s = np.ascontiguousarray(enc.stream if stream is None else stream, np.uint8)
+    o = np.ascontiguousarray(enc.off16 if off16 is None else off16, np.uint32)
+    return df11.df11_rans_validate(enc.n if n is None else n, s.ctypes.data, s.size,
+                                   o.ctypes.data, o.size)
+
+
+@pytest.mark.parametrize("n", [0, 1, 31, 16384, 16385, 100_003])
+def test_validate_accepts_the_oracle_encoding(n):
+    enc = oracle.rans_encode(workloads.random_bf16(n, seed=n + 3))
+    assert validate(enc) == df11.DF11_OK
+
+
+def test_validate_accepts_edge_encodings():
+    for x in (workloads.constant(70_000, 0x3F80), workloads.shuffled_patterns(copies=1, seed=2),
+              workloads.fibonacci_exponents(30)[:50_000]):
+        assert validate(oracle.rans_encode(x)) == df11.DF11_OK
+
+
+def test_validate_rejects_corrupt_metadata():
+    enc = oracle.rans_encode(workloads.random_bf16(3 * 16384 + 100, seed=7))
+    u1 = 16 * int(enc.off16[1])
+
+    def stream_with(pos, value, width=1):
+        s = enc.stream.copy()
+        s[pos:pos + width] = np.frombuffer(int(value).to_bytes(width, "little"), np.uint8)
+        return s
+
+    off = enc.off16.copy()
+    off[2], off[1] = off[1], off[2]                  # decreasing offsets
+    assert validate(enc, off16=off) == df11.DF11_ERR_CORRUPT
+    off = enc.off16.copy()
+    off[-1] += 1                                      # last offset past the stream
+    assert validate(enc, off16=off) == df11.DF11_ERR_CORRUPT
+    off = enc.off16.copy()
+    off[1] = off[0] + 8                               # a unit smaller than its header
+    off[2] = max(off[2], off[1])
+    assert validate(enc, off16=off) == df11.DF11_ERR_CORRUPT
+    off = enc.off16.copy()
+    off[1] = off[-1] + 100                            # an offset beyond the end (read guard)
+    assert validate(enc, off16=off) == df11.DF11_ERR_CORRUPT
+    assert validate(enc, stream=stream_with(u1 + 128, 3, 2)) == df11.DF11_ERR_CORRUPT   # start[0]
+    assert validate(enc, stream=stream_with(u1 + 130, 0xFFFF, 2)) == df11.DF11_ERR_CORRUPT
+    assert validate(enc, stream=stream_with(u1 + 4 * 9, 0x1234, 4)) == df11.DF11_ERR_CORRUPT
+    # a last unit of 20 values: lanes 20..31 code nothing, so their states must be exactly 2^16
+    tail = oracle.rans_encode(workloads.random_bf16(3 * 16384 + 20, seed=8))
+    last = 16 * int(tail.off16[3])
+    s = tail.stream.copy()
+    s[last + 4 * 31: last + 4 * 32] = np.frombuffer(((1 << 16) + 1).to_bytes(4, "little"), np.uint8)
+    assert validate(tail) == df11.DF11_OK
+    assert validate(tail, stream=s) == df11.DF11_ERR_CORRUPT
+    assert validate(enc, off16=enc.off16[:-1]) == df11.DF11_ERR_INVALID_ARG
+    assert validate(enc, n=2 ** 33) == df11.DF11_ERR_TOO_LARGE
