@@ -59,7 +59,7 @@ extern "C" {
 #define DF11_MAX_CODE_LEN 32u      /* [Kernel]/[LUT]: longest code, 32 bits      */
 #define DF11_MAX_N 0xFFFFFFFFull   /* [Kernel]: 32-bit block output positions    */
 #define DF11_MAX_BATCH 32u         /* matrices per decode launch (more = split)  */
-#define DF11_TABLE_BITS 12u        /* reach of the decode table: codebooks whose
+#define DF11_TABLE_BITS 11u        /* reach of the decode table: codebooks whose
                                       codes are all this short decode on the
                                       fast path; longer codes (up to 32) take a
                                       length search.  The codec's default cap.  */
@@ -75,7 +75,11 @@ typedef enum {
   DF11_ERR_CORRUPT = 4,                /* stream/metadata inconsistent          */
   DF11_ERR_SYMBOL_NOT_IN_CODEBOOK = 5, /* a value to encode has no code         */
   DF11_ERR_TIMEOUT = 6,                /* a bounded wait inside a kernel ran out */
-  DF11_ERR_NO_DEVICE = 7               /* no usable CUDA device                 */
+  DF11_ERR_NO_DEVICE = 7,              /* no usable CUDA device                 */
+  DF11_ERR_BOUNDS = 8                  /* a bounds check of the checked build
+                                          (DF11_CHECKED) failed; the access was
+                                          skipped.  The product build never
+                                          reports it                            */
 } df11_status;
 
 /* Canonical, length-limited code for the 256 exponent values. */
@@ -198,9 +202,12 @@ size_t df11_tables_bytes(void);
  * df11_build_tables -- host.  Decode tables for cb, written to h_tables
  * (bytes >= df11_tables_bytes()); the caller copies them to device memory and
  * points df11_matrix.tables at the copy.  [LUT]: table lookups replace the
- * bit-serial tree walk; here one 4096-entry table maps the next 12 stream bits
- * to up to three whole codes, and codes longer than 12 bits go through a
- * canonical length search.
+ * bit-serial tree walk; here one 2048-entry table maps the next
+ * DF11_TABLE_BITS (11) stream bits to up to four whole codes (8 bytes an
+ * entry: the exponents and the start of each code), and codes longer than 11
+ * bits go through a canonical length search.  The decoder checks every entry
+ * before use: a table that could make it write outside its staging is
+ * rejected and the matrix reported as DF11_ERR_CORRUPT.
  */
 df11_status df11_build_tables(const df11_codebook *cb, void *h_tables, size_t bytes);
 
@@ -246,7 +253,9 @@ df11_status df11_encode_device_codebook(const uint16_t *d_w, uint64_t n, const d
  * the process exits.  Nothing is allocated.
  *   n <= DF11_STATIC_WS_MAX_N, else DF11_ERR_TOO_LARGE (nothing launched).
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * that device current); make that first call before any stream capture.  The
+ * address is kept for the life of the process: resetting a device
+ * (cudaDeviceReset) after that first call is not supported.
  * All calls share the one array: calls whose work overlaps on the GPU (other
  * streams, other host threads) race on it and must be serialised by the
  * caller.  Each call rewrites every entry it reads, so nothing needs clearing
@@ -262,8 +271,17 @@ df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n, const df11_co
  *   m      host struct describing device buffers.
  *   d_out  n uint16 BF16 words, 16-byte aligned; written in full.
  *   d_status  DF11_ERR_CORRUPT if a block's decoded count disagrees with its
- *          stored positions or a code is invalid; DF11_ERR_TIMEOUT if a bulk
- *          copy did not land within the kernel's wait limit.
+ *          stored positions, a code is invalid or the tables are malformed;
+ *          DF11_ERR_TIMEOUT if a bulk copy did not land within the kernel's
+ *          bounded wait (the kernel then stops, with nothing of its own in
+ *          flight).
+ * Detection of corrupt data is limited to what the format lets the decoder
+ * check: every block's code count against its stored positions and every
+ * code against the codebook.  The format carries no checksum, so a
+ * corruption of the stream or of the sign/mantissa plane that keeps those
+ * counts can decode, silently, to other BF16 values.  Memory safety does not
+ * depend on the data: whatever the buffers hold, the decoder reads and writes
+ * only inside the allocations the format defines.
  * One kernel launch (the batch kernel with one matrix).
  */
 df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32_t *d_status,
@@ -328,6 +346,77 @@ df11_status df11_decode_matmul_batch(const df11_matrix *ms, const df11_matmul_io
 df11_status df11_validate(uint64_t n, uint64_t total_bits, uint32_t min_len,
                           const uint8_t *h_gaps, uint64_t gaps_bytes,
                           const uint32_t *h_block_pos, uint64_t block_pos_count);
+
+/*
+ * Serialised form of one compressed matrix (the ".df11" container).  [Format]:
+ * what a DF11 model stores per weight matrix is its code lengths, the
+ * exponent bitstream with its gaps and block positions, and the sign/mantissa
+ * plane; this fixes a byte layout for them (the page names the parts, not a
+ * file layout).  All fields little-endian:
+ *   0    char[4]    "DF11"
+ *   4    uint32     version (1)
+ *   8    uint64     n
+ *   16   uint64     total_bits
+ *   24   uint32     cap (the length cap the code was built under)
+ *   28   uint32     max_block_codes (0 = not recorded)
+ *   32   uint32     ndim (0..4)
+ *   36   uint32     0
+ *   40   uint64[4]  shape (unused dimensions 0; their product is n if ndim)
+ *   72   uint8[256] code lengths
+ *   328  uint8[8]   0
+ *   336  gaps (ceil(5C/8) bytes), then block_pos (uint32[B+1]), stream (8C
+ *        bytes), sign_mantissa (n bytes) and a uint32 CRC-32 (IEEE 802.3, as
+ *        zlib's crc32) of every byte before it; each of these five starts at
+ *        the next multiple of 16 bytes, the gap before it zero
+ * The container's checksum covers the whole matrix; the DF11 format itself
+ * has none (df11_decode).
+ */
+#define DF11_FILE_VERSION 1u
+#define DF11_FILE_HEADER_BYTES 336u
+
+/* One matrix as host arrays (non-owning; stored sizes, no padding). */
+typedef struct {
+  uint64_t n, total_bits;
+  uint32_t cap, max_block_codes;
+  uint32_t ndim;
+  uint64_t shape[4];
+  const uint8_t *lengths;        /* 256 code lengths                         */
+  const uint8_t *gaps;           /* df11_sizes.gaps_bytes                    */
+  const uint32_t *block_pos;     /* n_blocks + 1 entries                     */
+  const uint8_t *stream;         /* df11_sizes.stream_bytes                  */
+  const uint8_t *sign_mantissa;  /* n bytes                                  */
+} df11_host_matrix;
+
+/* Bytes df11_write produces for a matrix of n values and total_bits code
+ * bits (0 if the pair is invalid, see df11_sizes_from_bits). */
+uint64_t df11_file_bytes(uint64_t n, uint64_t total_bits);
+
+/*
+ * df11_write -- host.  Serialise m into buf (buf_bytes >= df11_file_bytes).
+ * DF11_ERR_INVALID_ARG for a null array, ndim > 4, a shape whose product is
+ * not n, or a buffer too small; the lengths must describe a code (lengths
+ * <= 32, Kraft sum <= 1).  *written receives the byte count.
+ */
+df11_status df11_write(const df11_host_matrix *m, void *buf, uint64_t buf_bytes,
+                       uint64_t *written);
+
+/*
+ * df11_read -- host.  Parse a serialised matrix: checks the magic, version,
+ * sizes (derived from n and total_bits, df11_sizes_from_bits) against
+ * buf_bytes, the CRC-32, and the stored metadata (df11_validate), then points
+ * out's arrays into buf (zero copy; buf must outlive them).  Returns
+ * DF11_ERR_CORRUPT for a bad magic, version, size, checksum or metadata.
+ */
+df11_status df11_read(const void *buf, uint64_t buf_bytes, df11_host_matrix *out);
+
+/*
+ * df11_codebook_from_lengths -- host.  The codebook whose lengths are len
+ * (code values canonical, RFC 1951 section 3.2.2, as df11_build_codebook
+ * assigns them): what a reader rebuilds from a stored matrix.
+ * DF11_ERR_INVALID_ARG if a length exceeds 32 or the lengths over-fill the
+ * code space (Kraft sum > 1).
+ */
+df11_status df11_codebook_from_lengths(const uint8_t len[256], uint32_t cap, df11_codebook *out);
 
 #ifdef __cplusplus
 }

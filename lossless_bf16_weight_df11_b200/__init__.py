@@ -18,7 +18,9 @@ import re
 import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libdf11_b200.so")
+# The product library; DF11_LIB may name another build of the same sources (the
+# checked build, libdf11_b200_checked.so) to run the tests against it.
+LIB_PATH = os.environ.get("DF11_LIB") or os.path.join(HERE, "libdf11_b200.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 HEADER = os.path.join(INCLUDE, "df11.h")
 HEADERS = [HEADER, os.path.join(INCLUDE, "df11_rans.h")]
@@ -29,7 +31,7 @@ GAP_BITS = 5
 MAX_CODE_LEN = 32
 MAX_N = 0xFFFFFFFF
 MAX_BATCH = 32
-TABLE_BITS = 12  # decode-table reach; the codec's default length cap
+TABLE_BITS = 11  # decode-table reach; the codec's default length cap
 
 DF11_OK = 0
 DF11_ERR_INVALID_ARG = 1
@@ -39,6 +41,7 @@ DF11_ERR_CORRUPT = 4
 DF11_ERR_SYMBOL_NOT_IN_CODEBOOK = 5
 DF11_ERR_TIMEOUT = 6
 DF11_ERR_NO_DEVICE = 7
+DF11_ERR_BOUNDS = 8
 
 
 class df11_codebook(ctypes.Structure):
@@ -73,6 +76,19 @@ class df11_encoded(ctypes.Structure):
 class df11_matmul_io(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_uint32), ("cols", ctypes.c_uint32),
                 ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
+class df11_host_matrix(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_uint64), ("total_bits", ctypes.c_uint64),
+                ("cap", ctypes.c_uint32), ("max_block_codes", ctypes.c_uint32),
+                ("ndim", ctypes.c_uint32), ("shape", ctypes.c_uint64 * 4),
+                ("lengths", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
+                ("block_pos", ctypes.c_void_p), ("stream", ctypes.c_void_p),
+                ("sign_mantissa", ctypes.c_void_p)]
+
+
+FILE_VERSION = 1          # DF11_FILE_VERSION
+FILE_HEADER_BYTES = 336   # DF11_FILE_HEADER_BYTES
 
 
 class df11_rans_matrix(ctypes.Structure):
@@ -116,6 +132,11 @@ def _declare(lib):
                                                     ctypes.POINTER(df11_matmul_io), _u32, _u32,
                                                     _vp, _vp]),
         "df11_sizes_from_bits": (ctypes.c_int, [_u64, _u64, ctypes.POINTER(df11_sizes)]),
+        "df11_file_bytes": (_u64, [_u64, _u64]),
+        "df11_write": (ctypes.c_int, [ctypes.POINTER(df11_host_matrix), _vp, _u64,
+                                      ctypes.POINTER(ctypes.c_uint64)]),
+        "df11_read": (ctypes.c_int, [_vp, _u64, ctypes.POINTER(df11_host_matrix)]),
+        "df11_codebook_from_lengths": (ctypes.c_int, [_vp, _u32, ctypes.POINTER(df11_codebook)]),
         "df11_build_codebook_device": (ctypes.c_int, [_vp, _u32, _vp, _vp, _vp, _vp, _vp]),
         "df11_encode_device_codebook": (ctypes.c_int, [_vp, _u64, _vp, _u64,
                                                        ctypes.POINTER(df11_encoded), _vp,
@@ -240,6 +261,32 @@ def df11_sizes_from_bits(n: int, total_bits: int):
     out = df11_sizes()
     st = load().df11_sizes_from_bits(n, total_bits, ctypes.byref(out))
     return st, out
+
+
+def df11_file_bytes(n: int, total_bits: int) -> int:
+    return int(load().df11_file_bytes(n, total_bits))
+
+
+def df11_write(m: df11_host_matrix, buf: int, buf_bytes: int):
+    """Serialise m into the host buffer at address buf; returns (status, bytes)."""
+    written = ctypes.c_uint64(0)
+    st = load().df11_write(ctypes.byref(m), buf, buf_bytes, ctypes.byref(written))
+    return st, int(written.value)
+
+
+def df11_read(buf: int, buf_bytes: int):
+    """Parse a serialised matrix in the host buffer at address buf; returns
+    (status, df11_host_matrix whose arrays point into that buffer)."""
+    out = df11_host_matrix()
+    st = load().df11_read(buf, buf_bytes, ctypes.byref(out))
+    return st, out
+
+
+def df11_codebook_from_lengths(lengths: int, cap: int = MAX_CODE_LEN):
+    """lengths: host address of 256 code lengths.  Returns (status, df11_codebook)."""
+    cb = df11_codebook()
+    st = load().df11_codebook_from_lengths(lengths, cap, ctypes.byref(cb))
+    return st, cb
 
 
 def df11_build_codebook_device(d_hist256: int, cap: int, d_cb: int, d_tables: int,

@@ -287,7 +287,8 @@ DF11_HD inline df11_status table_lengths(const df11_codebook *cb, df11i::DecodeT
 }
 
 // The per-value part: value s (with a code) goes to sym[] at its rank in
-// (length asc, value asc) order, and its length to codelen[s].
+// (length asc, value asc) order, rotated as the decoder stores exponents
+// (df11i::ror8), and its length to codelen[s].
 DF11_HD inline void table_value(const df11_codebook *cb, df11i::DecodeTables *t, int s) {
   const unsigned L = cb->len[s];
   t->codelen[s] = (uint8_t)L;
@@ -297,7 +298,7 @@ DF11_HD inline void table_value(const df11_codebook *cb, df11i::DecodeTables *t,
     const unsigned Lu = cb->len[u];
     r += Lu && (Lu < L || (Lu == L && u < s));
   }
-  t->sym[r] = (uint8_t)s;
+  t->sym[r] = (uint8_t)df11i::ror8((uint32_t)s);
 }
 
 // Everything of the decode tables but the lookup table, sequentially; t must
@@ -310,14 +311,17 @@ DF11_HD inline df11_status table_header(const df11_codebook *cb, df11i::DecodeTa
   return DF11_OK;
 }
 
-// Lookup-table entry for the 12-bit window v: the whole codes (at most three)
-// in it, decoded greedily, or the long-code flag.
-DF11_HD inline uint32_t lut_entry_for(const df11i::DecodeTables &t, const TableAux &aux,
-                                      uint32_t max_len, uint32_t v) {
+// Lookup-table entry for the kLutBits-bit window v: the whole codes (at most
+// four) in it, decoded greedily, with the start of each code after the first,
+// or the long-code flag when the window does not hold a whole first code.
+DF11_HD inline df11i::LutEntry lut_entry_for(const df11i::DecodeTables &t, const TableAux &aux,
+                                             uint32_t max_len, uint32_t v) {
   const int K = df11i::kLutBits;
   const unsigned maxl = max_len ? max_len : 1;
   uint32_t used = 0, nsym = 0, syms = 0;
-  while (nsym < 3) {
+  uint32_t start[df11i::kLutMaxCodes] = {0, df11i::kCtrlNoStart, df11i::kCtrlNoStart,
+                                         df11i::kCtrlNoStart};
+  while (nsym < df11i::kLutMaxCodes) {
     uint64_t window = ((uint64_t)v << (32 - K)) << used;  // left-justified, zeros after
     window &= 0xFFFFFFFFull;
     int found = -1;
@@ -331,12 +335,25 @@ DF11_HD inline uint32_t lut_entry_for(const df11i::DecodeTables &t, const TableA
       }
     }
     if (found < 0) break;
-    syms |= (uint32_t)found << (8 * nsym);
+    syms |= (uint32_t)found << (8 * nsym);  // sym[] holds rotated exponents
+    start[nsym] = used;
     ++nsym;
     used += L;
   }
-  return nsym ? df11i::lut_entry(syms, nsym, used)
-              : (df11i::lut_entry(0, 0, (uint32_t)K) | df11i::kLutLongFlag);
+  df11i::LutEntry e;
+  if (nsym) {
+    e.x = syms;
+    e.y = df11i::lut_ctrl(nsym, start[1], start[2], start[3], used);
+  } else {
+    e.x = 0;
+    // no codes; the bits consumed are the window's, so that a decoder that
+    // does not test the flag (codebooks within the table's reach, where a
+    // flagged window only occurs in a corrupt stream) still moves on
+    e.y = df11i::lut_ctrl(0, df11i::kCtrlNoStart, df11i::kCtrlNoStart, df11i::kCtrlNoStart,
+                          (uint32_t)K) |
+          df11i::kCtrlLongFlag;
+  }
+  return e;
 }
 
 }  // namespace df11cb

@@ -45,8 +45,13 @@ using df11i::DecodeTables;
 
 namespace {
 
-constexpr int kT = 256;  // threads per decode CTA
-constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls
+constexpr int kT = 256;  // threads per decode group (a CTA holds up to four)
+// Bounded mbarrier polls before a wait gives up (DF11_ERR_TIMEOUT).  The test
+// build (DF11_TEST_HOOKS) compiles with a small limit.
+#ifndef DF11_WAIT_LIMIT
+#define DF11_WAIT_LIMIT (1u << 22)
+#endif
+constexpr uint32_t kWaitLimit = DF11_WAIT_LIMIT;
 
 __device__ __forceinline__ void set_status(uint32_t *st, uint32_t code) {
   if (st) atomicCAS(st, 0u, code);
@@ -579,13 +584,22 @@ __global__ void __launch_bounds__(kCbThreads) codebook_kernel(
 // ============================================================ decode
 //
 // Work unit: kUnitChunks = 512 consecutive chunks of one matrix (two of the
-// format's 256-chunk blocks; the last unit of a matrix may hold one).  A CTA
-// of 256 threads decodes a unit, each thread two consecutive chunks: it
-// starts at the first chunk's gap and decodes straight on through the second,
-// because the first code starting in the second chunk begins exactly where
-// the last code starting in the first one ends.  The unit's first output is
-// pos[2u] and its outputs end at pos[min(2u + 2, B)].
+// format's 256-chunk blocks; the last unit of a matrix may hold one).  A group
+// of 256 threads decodes a unit, each thread two consecutive chunks: it starts
+// at the first chunk's gap and decodes straight on through the second, because
+// the first code starting in the second chunk begins exactly where the last
+// code starting in the first one ends.  The unit's first output is pos[2u] and
+// its outputs end at pos[min(2u + 2, B)].
+//
+// A CTA (one per SM) holds up to kMaxGroups such groups.  They share one copy
+// of the current matrix's decode tables in shared memory; everything else (the
+// stages the unit's bytes are copied into, the staging rows, the mbarriers) is
+// the group's own, and a group synchronises with a named barrier of its own.
+// The CTA as a whole synchronises only where the tables change: its share of
+// the batch's (matrix, unit) list is split at matrix boundaries, and within
+// one matrix the units are dealt out to the groups in turn.
 
+constexpr int kMaxGroups = 4;
 constexpr int kCPT = 2;                                       // chunks per thread
 constexpr uint32_t kUnitChunks = kT * kCPT;                   // 512
 constexpr uint32_t kUnitBlocks = kUnitChunks / DF11_BLOCK_CHUNKS;  // 2
@@ -617,29 +631,23 @@ struct DecParams {
   DecMat m[DF11_MAX_BATCH];
   uint64_t unit_start[DF11_MAX_BATCH + 1];  // prefix sums of units per matrix
   uint32_t count;
-  uint32_t stage_cap;     // bytes: max codes per unit, rounded up to 16
-  uint32_t region_bytes;  // private decode region per thread (odd number of words)
-  uint32_t min_len;       // shortest code of the batch (regions are sized by it)
-  uint32_t batch;         // fused matmul: activation rows (<= the kernel's NB)
+  uint32_t stage_cap;  // bytes: max codes per unit, rounded up to 16
+  uint32_t min_len;    // shortest code of the batch (regions are sized by it)
+  uint32_t batch;      // fused matmul: activation rows (<= the kernel's NB)
   uint32_t *status;
+#ifdef DF11_TEST_HOOKS
+  // test build only: bytes every stream-stage barrier expects beyond what its
+  // bulk copies deliver, so that the copies land but the waits run out
+  uint32_t starve_tx;
+#endif
 };
 
 constexpr uint32_t kStreamStage = 8 * kUnitChunks + 16;         // a unit of chunks + the next word
 constexpr uint32_t kGapStage = DF11_GAP_BITS * kUnitChunks / 8;  // 320 B
 constexpr uint32_t kStageBytes = kStreamStage + kGapStage + 16;
+constexpr uint32_t kTablesSmem = (uint32_t)((sizeof(DecodeTables) + 127) & ~(size_t)127);
 static_assert(kStageBytes % 16 == 0 && sizeof(DecodeTables) % 16 == 0, "stage alignment");
 
-struct SmemLayout {
-  uint32_t tables, stage0, stage1, sm, linear, priv, bars, meta, warp, acc, total;
-};
-
-// The linear row holds the unit's exponents from byte P0 % 8 on; the
-// relocation of the thread with the last codes ORs region_bytes + 4 bytes
-// from a 4-byte boundary at most 7 + cap bytes in, so the row carries that
-// much slack.
-// Every section starts on a 16-byte boundary: bulk-copy destinations and
-// 16-byte reads (stages, sign/mantissa row, warp totals), 8-byte reads and
-// writes (linear row), mbarriers (8 bytes).
 __host__ __device__ constexpr uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
 // Rows of the fused matmul's per-unit accumulators: a unit's outputs span at
@@ -648,33 +656,43 @@ __host__ __device__ constexpr uint32_t round16(uint32_t x) { return (x + 15u) & 
 constexpr uint32_t kAccRows = 136;
 constexpr uint32_t kMinMatmulCols = DF11_MATMUL_MIN_COLS;
 
-__host__ __device__ inline SmemLayout smem_layout(uint32_t cap, uint32_t region_bytes,
-                                                  uint32_t nb = 0) {
-  SmemLayout S;
-  S.tables = 0;
-  S.stage0 = round16((uint32_t)sizeof(DecodeTables));
-  S.stage1 = round16(S.stage0 + kStageBytes);
-  S.sm = round16(S.stage1 + kStageBytes);
-  S.linear = round16(S.sm + cap + 32);
-  S.priv = round16(S.linear + cap + region_bytes + 32);
-  S.bars = round16(S.priv + kT * region_bytes);
-  S.meta = round16(S.bars + 32);
-  S.warp = round16(S.meta + 2 * 32);
-  S.acc = round16(S.warp + 16 * 4);
-  S.total = round16(S.acc + 4 * kAccRows * nb);
-  return S;
-}
+// One group's shared memory, as offsets from the group's base (every section
+// on a 16-byte boundary: bulk-copy destinations, 16-byte accesses, mbarriers):
+//   stage0/1  a unit's stream bytes (+ the next 16) and gap bytes, each
+//   sm        the sign/mantissa bytes of outputs P0 & ~15 .. P1 (<= cap + 32)
+//   linear    the unit's exponents in output order, byte j for output
+//             (P0 & ~15) + j; the merge reads it in 16-byte groups up to
+//             round16(15 + cap) and relocation writes up to 15 + cap
+//   priv      the threads' private rows (region_bytes per thread)
+//   bars      mbarriers of stage 0, stage 1 and the sign/mantissa copy
+//   meta      per stage: P0, P1, matrix, unit, PM (+ row, col for the matmul)
+//   warp      per-warp code totals
+//   acc       fused matmul row sums [NB][kAccRows]
+struct GroupLayout {
+  uint32_t stage0, stage1, sm, linear, priv, bars, meta, warp, acc, size;
+};
 
-inline bool smem_layout_aligned(const SmemLayout &S) {
-  return ((S.stage0 | S.stage1 | S.sm | S.linear | S.priv | S.bars | S.meta | S.warp | S.acc) &
-          15u) == 0;
+__host__ __device__ inline GroupLayout group_layout(uint32_t cap, uint32_t region_bytes,
+                                                    uint32_t nb) {
+  GroupLayout G;
+  G.stage0 = 0;
+  G.stage1 = kStageBytes;
+  G.sm = 2 * kStageBytes;
+  G.linear = round16(G.sm + cap + 32);
+  G.priv = round16(G.linear + cap + 32);
+  G.bars = round16(G.priv + kT * region_bytes);
+  G.meta = G.bars + 32;
+  G.warp = G.meta + 64;
+  G.acc = G.warp + 32;
+  G.size = (G.acc + 4 * kAccRows * nb + 127u) & ~127u;
+  return G;
 }
 
 // Per-thread private region, in 32-bit rows: the codes that can start in a
-// thread's two chunks (ceil(128/min_len)), two codes of overshoot from the
-// last table entry, and two spare bytes; rounded to an odd number of rows.
+// thread's two chunks (ceil(128/min_len)), three codes of overshoot from the
+// last table entry; rounded to an odd number of rows.
 __host__ __device__ constexpr uint32_t region_words_even(uint32_t min_len) {
-  return ((64 * kCPT + min_len - 1) / min_len + 4 + 3) / 4;
+  return ((64 * kCPT + min_len - 1) / min_len + 3 + 4) / 4;
 }
 __host__ __device__ constexpr uint32_t region_bytes_for(uint32_t min_len) {
   return 4 * (region_words_even(min_len) + (region_words_even(min_len) % 2 == 0 ? 1 : 0));
@@ -684,22 +702,59 @@ __host__ __device__ constexpr uint32_t region_bytes_for(uint32_t min_len) {
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
+
+// The checked build (DF11_CHECKED): every access of the decode path through
+// the helpers below is checked against the CTA's dynamic shared memory (range
+// and alignment), every global store and bulk-copy source against its buffer;
+// a failed check skips the access and sets DF11_ERR_BOUNDS in the launch's
+// status word, so an indexing error shows as a status, not a fault.  The
+// product build compiles the checks away.
+#ifdef DF11_CHECKED
+__shared__ uint32_t *s_check_status;
+extern __shared__ __align__(128) uint8_t df11_dyn_smem[];
+__device__ __forceinline__ void check_failed() {
+  if (s_check_status) atomicCAS(s_check_status, 0u, (uint32_t)DF11_ERR_BOUNDS);
+}
+__device__ __forceinline__ bool smem_ok(uint32_t a, uint32_t bytes) {
+  uint32_t size;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(size));
+  const uint32_t lo = smem_addr(df11_dyn_smem);
+  const bool ok = a >= lo && a - lo <= size && bytes <= size - (a - lo) && (a & (bytes - 1)) == 0;
+  if (!ok) check_failed();
+  return ok;
+}
+#define DF11_SMEM_CHECK(a, bytes, on_fail) \
+  if (!smem_ok((a), (bytes))) on_fail;
+#define DF11_GLOBAL_CHECK(cond, on_fail) \
+  if (!(cond)) {                         \
+    check_failed();                      \
+    on_fail;                             \
+  }
+#else
+#define DF11_SMEM_CHECK(a, bytes, on_fail)
+#define DF11_GLOBAL_CHECK(cond, on_fail)
+#endif
+
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  DF11_SMEM_CHECK(a, 4, return 0u)
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
   return v;
 }
 __device__ __forceinline__ uint32_t lds8(uint32_t a) {
+  DF11_SMEM_CHECK(a, 1, return 0u)
   uint32_t v;
   asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
   return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t a) {
+  DF11_SMEM_CHECK(a, 8, return make_uint2(0u, 0u))
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
   return v;
 }
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
+  DF11_SMEM_CHECK(a, 16, return make_uint4(0u, 0u, 0u, 0u))
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
@@ -708,31 +763,31 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   return v;
 }
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+  DF11_SMEM_CHECK(a, 4, return)
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 __device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+  DF11_SMEM_CHECK(a, 8, return)
   asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
 }
+__device__ __forceinline__ void sts128_zero(uint32_t a) {
+  DF11_SMEM_CHECK(a, 16, return)
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+}
 __device__ __forceinline__ void red_or32(uint32_t a, uint32_t v) {
+  DF11_SMEM_CHECK(a, 4, return)
   asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
-// predicated store: the compiler cannot predicate an asm statement itself,
-// so the predicate is passed in and applied inside (no branch)
-__device__ __forceinline__ void sts8_if(uint32_t a, uint32_t v, bool c) {
-  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q st.shared.u8 [%0], %1;\n}\n" ::"r"(a),
-               "r"(v), "r"((uint32_t)c)
-               : "memory");
-}
-// (a * b) >> 32 and ((a * b) >> 32) + c: field extraction on the multiply pipe
-__device__ __forceinline__ uint32_t mulhi(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
+// (a * b) >> 32 + c: field extraction on the multiply pipe
 __device__ __forceinline__ uint32_t madhi(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t r;
   asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
+}
+
+// Barrier of one decode group (named barrier id, the group's 256 threads).
+__device__ __forceinline__ void group_sync(uint32_t id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kT) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -778,80 +833,72 @@ __device__ __forceinline__ uint32_t long_code_len(uint32_t w32, const DecodeTabl
   return 0;
 }
 
+// The control word of a code decoded by the length search: one code, no
+// further starts, no bits counted (the trim after the loop then keeps it).
+constexpr uint32_t kLongCodeCtrl =
+    df11i::lut_ctrl(1, df11i::kCtrlNoStart, df11i::kCtrlNoStart, df11i::kCtrlNoStart, 0);
+
 // Appending decoded exponents to a thread's private bytes.  The private
 // regions of a warp are interleaved by 32-bit word: word j of lane l is
 // shared word 32 j + l of the warp's region, so any access in which every
 // lane touches one word of its own falls in 32 different banks.  The word
 // being filled is kept in a register (cur) and written through on every
-// step with one 32-bit store at row_a; nb counts the bits appended (8 per
-// exponent).  x holds the step's exponents from the low byte up (absent
-// slots zero), cm its count in bits 24-25.
-#define DF11_APPEND(x, cm)                                                  \
+// step with one 32-bit store at row_a.  nb counts the bits appended (8 per
+// exponent) in its bits 0..10; a table entry's control word is added to it
+// whole (its bits 0..10 are 8 x its count, its higher bits land above the
+// count and are never read).  xs holds the step's exponents from the low byte
+// up (absent slots zero).
+#define DF11_APPEND(xs, add)                                                \
   {                                                                         \
-    const uint32_t xs = (x);                                                \
-    const uint32_t lo = cur | __funnelshift_l(0u, xs, nb);                  \
-    const uint32_t hi = __funnelshift_l(xs, 0u, nb);                        \
+    const uint32_t lo = cur | __funnelshift_l(0u, (xs), nb);                \
+    const uint32_t hi = __funnelshift_l((xs), 0u, nb);                      \
     sts32(row_a, lo);                                                       \
-    const uint32_t nb2 = madhi((cm), 1u << 11, nb);                         \
-    row_a = col_a + ((nb2 >> 5) << 7);                                      \
+    const uint32_t nb2 = nb + (add);                                        \
+    row_a = col_a + ((nb2 & 0x7E0u) << 2);                                  \
     cur = __funnelshift_rc(lo, hi, (nb ^ nb2) & 32u);                       \
     nb = nb2;                                                               \
   }
 
-// One table step of the decoder on window w: the entry's exponents are
-// appended and p advances by the bits they use.  In the flagged form an
-// entry whose first code is longer than the table's reach sets f and leaves
-// the loop before anything is appended.
-#define DF11_STEP_FLAG(w, f)                                                \
-  e = lds32(lut_a + (mulhi((w), 1u << df11i::kLutBits) << 2));              \
-  if (e & df11i::kLutLongFlag) {                                            \
-    f = true;                                                               \
-    break;                                                                  \
-  }                                                                         \
-  DF11_APPEND(e & 0x00FFFFFFu, e & df11i::kLutCountMask)                    \
-  p = madhi(e, 1u << 4, p);
-
-#define DF11_STEP(w)                                                        \
+// One table step on the window of stream words hw:lw at bit p: the entry's
+// exponents are appended and p advances by the bits they use.
+#define DF11_STEP(hw, lw)                                                   \
   {                                                                         \
-    e = lds32(lut_a + (mulhi((w), 1u << df11i::kLutBits) << 2));            \
-    DF11_APPEND(e & 0x00FFFFFFu, e & df11i::kLutCountMask)                  \
-    p = madhi(e, 1u << 4, p);                                               \
+    const uint32_t w = __funnelshift_l((lw), (hw), p);                      \
+    const uint2 e = lds64(lut_a + ((w >> (32 - df11i::kLutBits)) << 3));    \
+    ctrl = e.y;                                                             \
+    DF11_APPEND(e.x, ctrl)                                                  \
+    p = madhi(ctrl, 1u << (32 - df11i::kCtrlUsedShift), p);                 \
   }
 
-// 4 exponents + 4 sign/mantissa bytes -> 4 BF16 words (two 32-bit halves).
-__device__ __forceinline__ void merge4(uint32_t e4, uint32_t s4, uint32_t &w01, uint32_t &w23) {
-  const uint32_t hi4 = (s4 & 0x80808080u) | ((e4 >> 1) & 0x7F7F7F7Fu);
-  const uint32_t lo4 = (s4 & 0x7F7F7F7Fu) | ((e4 << 7) & 0x80808080u);
+// 4 rotated exponents + 4 sign/mantissa bytes -> 4 BF16 words (two 32-bit
+// halves).  Byte i of r4 is ror8(e_i): its bits 0..6 are the exponent's high
+// seven bits (the BF16 high byte's bits 0..6), bit 7 its low bit (the low
+// byte's bit 7); the sign/mantissa byte supplies the other bit of each.
+__device__ __forceinline__ void merge4(uint32_t r4, uint32_t s4, uint32_t &w01, uint32_t &w23) {
+  const uint32_t hi4 = (s4 & 0x80808080u) | (r4 & 0x7F7F7F7Fu);
+  const uint32_t lo4 = (r4 & 0x80808080u) | (s4 & 0x7F7F7F7Fu);
   w01 = __byte_perm(lo4, hi4, 0x5140);
   w23 = __byte_perm(lo4, hi4, 0x7362);
 }
 
-struct UnitRef {
-  uint32_t m;  // matrix of the batch
-  uint32_t u;  // unit within the matrix
-};
-
-__device__ __forceinline__ UnitRef locate(const DecParams &P, uint64_t g, uint32_t hint) {
-  uint32_t m = hint;
-  while (m + 1 < P.count && g >= P.unit_start[m + 1]) ++m;
-  return UnitRef{m, (uint32_t)(g - P.unit_start[m])};
-}
-
-// A decoded block waiting for its merge: positions, output, staging.
+// A decoded unit waiting for its merge: positions, output, staging.
 struct Pending {
   uint32_t P0, P1;
   uint16_t *out;
   bool ok;
   uint32_t m;               // matrix of the batch
   uint32_t row_lo, col_lo;  // fused matmul: row and column of output P0 & ~7
+  uint32_t n;               // values of the matrix (bounds of out)
 };
 
-// Merge a decoded block: exponents in the linear row, sign/mantissa bytes in
-// the sm stage.  Thread t takes the whole 8-output groups t, t+256, ...; each
-// is one 16-byte store.  The ragged first and last groups are written
-// element by element by threads 0 and 1.  The row is cleared behind the
-// reads.
-__device__ __forceinline__ void merge_group(uint32_t lin_a, uint32_t smb, uint32_t k, uint4 &r) {
+// Merge a decoded unit: exponents in the linear row, sign/mantissa bytes in
+// the sm stage, both indexed from output P0 & ~15 (so byte j of either is
+// output (P0 & ~15) + j).  Thread t takes the whole 8-output groups t, t+256,
+// ... from output P0 & ~7 on: each is one 16-byte store, and a warp's 32
+// stores fill 512 contiguous bytes.  The ragged first and last groups are
+// written element by element by threads 0 and 1.  The row is cleared behind
+// the reads (relocation ORs the words shared by two threads into it).
+__device__ __forceinline__ void merge_group8(uint32_t lin_a, uint32_t smb, uint32_t k, uint4 &r) {
   const uint2 e8 = lds64(lin_a + 8 * k);
   sts64(lin_a + 8 * k, 0u, 0u);
   const uint2 s8 = lds64(smb + 8 * k);
@@ -859,56 +906,64 @@ __device__ __forceinline__ void merge_group(uint32_t lin_a, uint32_t smb, uint32
   merge4(e8.y, s8.y, r.z, r.w);
 }
 
-__device__ __forceinline__ void merge_block(const Pending &q, uint32_t lin_a, uint32_t sm_a, int t) {
+__device__ __forceinline__ void merge_unit(const Pending &q, uint32_t lin_a, uint32_t sm_a, int t) {
   const uint32_t base8 = q.P0 & ~7u;
-  const uint32_t smb = sm_a + (base8 - (q.P0 & ~15u));
-  const uint32_t head = q.P0 & 7u;         // outputs of group 0 before the block
-  const uint32_t span8 = q.P1 - base8;     // outputs from base8 to the block's end
+  const uint32_t off8 = base8 - (q.P0 & ~15u);  // 0 or 8: where base8 sits in the rows
+  const uint32_t lin8 = lin_a + off8, smb = sm_a + off8;
+  const uint32_t head = q.P0 & 7u;         // outputs of group 0 before the unit
+  const uint32_t span8 = q.P1 - base8;     // outputs from base8 to the unit's end
   const uint32_t full0 = head ? 1u : 0u;
   const uint32_t full1 = span8 >> 3;
   uint4 *out4 = reinterpret_cast<uint4 *>(q.out + base8);
   for (uint32_t k = full0 + t; k < full1; k += kT) {
     uint4 r;
-    merge_group(lin_a, smb, k, r);
+    merge_group8(lin8, smb, k, r);
+    DF11_GLOBAL_CHECK(base8 + 8 * k + 8 <= q.n, continue)
     out4[k] = r;
   }
-  // ragged first group (thread 0) and last group (thread 1, unless it is
-  // the first one); element j of group k is output base8 + 8k + j
+  // ragged first group (thread 0) and last group (thread 1, unless it is the
+  // first one); element j of group k is output base8 + 8k + j
   const bool last_edge = (span8 & 7u) != 0 && !(head && full1 == 0);
   if ((t == 0 && head) || (t == 1 && last_edge)) {
     const uint32_t k = t == 0 ? 0u : full1;
     const uint32_t lo = t == 0 ? head : 0u;
     const uint32_t hi = min(8u, span8 - 8 * k);
     uint4 r;
-    merge_group(lin_a, smb, k, r);
+    merge_group8(lin8, smb, k, r);
     const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
     uint16_t *o = q.out + base8 + 8 * k;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if ((uint32_t)j >= lo && (uint32_t)j < hi) o[j] = (uint16_t)(wv[j >> 1] >> (16 * (j & 1)));
+      if ((uint32_t)j >= lo && (uint32_t)j < hi) {
+        DF11_GLOBAL_CHECK(base8 + 8 * k + j < q.n, continue)
+        o[j] = (uint16_t)(wv[j >> 1] >> (16 * (j & 1)));
+      }
   }
+  // (the linear row's words before base8 were never written: relocation
+  // starts at byte P0 & 15 >= base8 - (P0 & ~15))
 }
 
 // Fused matmul merge: the unit's decoded weights are multiplied with the
-// activations instead of being stored.  Lane l of warp w takes groups
-// w*32 + l, + 256, ... (8 weights each, flat index base8 + 8k, masked to
-// the unit's outputs); each group's dot products with the NB activation rows
-// are reduced over the warp per output row (32 consecutive groups span at
-// most two rows since cols >= 256) and added into the CTA's per-row
-// accumulators (row offsets from row_lo).  The staging row is cleared behind
-// the reads, as in the plain merge.
+// activations instead of being stored.  Lane l of warp w takes 8-weight
+// groups w*32 + l, + 256, ... (flat index base8 + 8k, masked to the unit's
+// outputs); each group's dot products with the NB activation rows are reduced
+// over the warp per output row (32 consecutive groups span at most two rows
+// since cols >= 256) and added into the group's per-row accumulators (row
+// offsets from row_lo).  The staging row is cleared behind the reads, as in
+// the plain merge.
 __device__ __forceinline__ void bf16x2_to_f32(uint32_t v, float &a, float &b) {
   a = __uint_as_float(v << 16);
   b = __uint_as_float(v & 0xFFFF0000u);
 }
 
 template <int NB>
-__device__ __forceinline__ void merge_block_matmul(const Pending &q, uint32_t lin_a, uint32_t sm_a,
-                                                   int t, float *acc, const DecMat &M,
-                                                   uint32_t batch) {
+__device__ __forceinline__ void merge_unit_matmul(const Pending &q, uint32_t lin_a, uint32_t sm_a,
+                                                  int t, float *acc, const DecMat &M,
+                                                  uint32_t batch) {
   const int lane = t & 31, warp = t >> 5;
   const uint32_t base8 = q.P0 & ~7u;
-  const uint32_t smb = sm_a + (base8 - (q.P0 & ~15u));
+  const uint32_t off8 = base8 - (q.P0 & ~15u);  // 0 or 8: where base8 sits in the rows
+  const uint32_t lin8 = lin_a + off8, smb = sm_a + off8;
   const uint32_t head = q.P0 & 7u;
   const uint32_t span8 = q.P1 - base8;
   const uint32_t ngroups = (span8 + 7) >> 3;
@@ -917,10 +972,12 @@ __device__ __forceinline__ void merge_block_matmul(const Pending &q, uint32_t li
   // (rows past the batch read as zero)
   auto load_x = [&](uint32_t k, uint32_t col, uint4 (&xv)[NB]) {
 #pragma unroll
-    for (int j = 0; j < NB; ++j)
-      xv[j] = (k < ngroups && (uint32_t)j < batch)
-                  ? __ldg(reinterpret_cast<const uint4 *>(M.x + (size_t)j * cols + col))
+    for (int j = 0; j < NB; ++j) {
+      bool use = k < ngroups && (uint32_t)j < batch;
+      DF11_GLOBAL_CHECK(!use || col + 8 <= cols, use = false)
+      xv[j] = use ? __ldg(reinterpret_cast<const uint4 *>(M.x + (size_t)j * cols + col))
                   : make_uint4(0u, 0u, 0u, 0u);
+    }
   };
   // row offset and column of this lane's first group
   uint32_t col = q.col_lo + 8u * (uint32_t)(warp * 32 + lane), row = 0;
@@ -954,7 +1011,7 @@ __device__ __forceinline__ void merge_block_matmul(const Pending &q, uint32_t li
     for (int j = 0; j < NB; ++j) d[j] = 0.f;
     if (k < ngroups) {
       uint4 r;
-      merge_group(lin_a, smb, k, r);
+      merge_group8(lin8, smb, k, r);
       float w[8];
       bf16x2_to_f32(r.x, w[0], w[1]);
       bf16x2_to_f32(r.y, w[2], w[3]);
@@ -999,9 +1056,10 @@ __device__ __forceinline__ void merge_block_matmul(const Pending &q, uint32_t li
     col = ncol;
     row = nrow;
   }
+  // the linear row's words before base8 were never written: nothing to clear
 }
 
-// Add a merged unit's row sums to y and clear the accumulators (after a CTA
+// Add a merged unit's row sums to y and clear the accumulators (after a group
 // barrier that follows the merge).
 template <int NB>
 __device__ __forceinline__ void flush_matmul(const Pending &q, float *acc, const DecMat &M,
@@ -1014,327 +1072,380 @@ __device__ __forceinline__ void flush_matmul(const Pending &q, float *acc, const
       const float v = acc[j * kAccRows + r];
       if ((uint32_t)j < batch && v != 0.f && q.row_lo + r < M.rows)
         atomicAdd(M.y + (size_t)j * M.rows + q.row_lo + r, v);
+      DF11_GLOBAL_CHECK(j * kAccRows + r < NB * kAccRows, continue)
       acc[j * kAccRows + r] = 0.f;
     }
   }
 }
 
+// Whether a lookup-table entry could take the decoder outside its private
+// region.  A valid entry has its reserved control bits clear and either one
+// to four codes, each at least min_len bits long (start fields increasing by
+// at least min_len, the last code ending by `used` <= the window; absent
+// codes' fields 15), or the long-code flag with no codes, no starts and the
+// whole window consumed.  With every code at least min_len bits, at most
+// ceil(128 / min_len) codes start in a thread's two chunks, plus three more
+// from the last entry: the region holds them.
+__device__ __forceinline__ bool lut_entry_bad(uint32_t c, uint32_t min_len) {
+  const uint32_t n = (c >> df11i::kCtrlCountShift) & 7u, used = c >> df11i::kCtrlUsedShift;
+  const uint32_t starts = (c >> df11i::kCtrlStartShift) & 0xFFFu;
+  if (c & df11i::kCtrlReserved) return true;
+  if (c & df11i::kCtrlLongFlag) return n != 0 || used != (uint32_t)df11i::kLutBits || starts != 0xFFFu;
+  if (n == 0 || n > df11i::kLutMaxCodes || used > (uint32_t)df11i::kLutBits) return true;
+  bool bad = false;
+  uint32_t prev = 0;
+#pragma unroll
+  for (uint32_t j = 1; j < df11i::kLutMaxCodes; ++j) {
+    const uint32_t sj = (starts >> (4 * (j - 1))) & 15u;
+    if (j < n) {
+      bad |= sj < prev + min_len;
+      prev = sj;
+    } else {
+      bad |= sj != df11i::kCtrlNoStart;
+    }
+  }
+  return bad || used < prev + min_len;
+}
+
 // MAXW: 32-bit words of a thread's private region.  NB: 0 for the plain
 // decode (BF16 stored to out); 1, 2, 4 or 8 for the fused matmul with up to
-// NB activation rows (P.batch of them used).
+// NB activation rows (P.batch of them used).  blockDim.x = 256 x groups.
 template <int MAXW, int NB>
-__global__ void __launch_bounds__(kT, 3) decode_kernel(const __grid_constant__ DecParams P) {
+__global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_kernel(const __grid_constant__ DecParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t ngroups = blockDim.x / kT;
+  const uint32_t grp = threadIdx.x / kT;
+  const int t = (int)(threadIdx.x % kT), lane = t & 31, warp = t >> 5;
   const uint32_t cap = P.stage_cap;
-  const SmemLayout S = smem_layout(cap, 4 * MAXW, NB);
-  float *acc = reinterpret_cast<float *>(smem + S.acc);  // [NB][kAccRows] row sums
-  const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem + S.tables);
+  const GroupLayout GL = group_layout(cap, 4 * MAXW, NB);
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t lut_a = sbase + S.tables;  // lut is the first member
-  const uint32_t codelen_a = sbase + S.tables + (uint32_t)offsetof(DecodeTables, codelen);
-  const uint32_t bar_stage = sbase + S.bars, bar_sm = sbase + S.bars + 16;
-  uint32_t *meta = reinterpret_cast<uint32_t *>(smem + S.meta);  // [stage][P0, P1, m, u, PM]
-  uint32_t *warp_tot = reinterpret_cast<uint32_t *>(smem + S.warp);
-  const uint32_t lin_a = sbase + S.linear;
-  const uint32_t sm_a = sbase + S.sm;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const uint32_t gofs = kTablesSmem + grp * GL.size;
+  const uint32_t gbase = sbase + gofs;
+  const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem);
+  const uint32_t lut_a = sbase;  // lut is the first member of the tables
+  float *acc = reinterpret_cast<float *>(smem + gofs + GL.acc);  // [NB][kAccRows] row sums
+  const uint32_t bar_stage = gbase + GL.bars, bar_sm = gbase + GL.bars + 16;
+  uint32_t *meta = reinterpret_cast<uint32_t *>(smem + gofs + GL.meta);
+  uint32_t *warp_tot = reinterpret_cast<uint32_t *>(smem + gofs + GL.warp);
+  const uint32_t lin_a = gbase + GL.linear;
+  const uint32_t sm_a = gbase + GL.sm;
   // this lane's column of its warp's interleaved private region
-  const uint32_t col_a = sbase + S.priv + (uint32_t)warp * (MAXW * 128u) + 4u * lane;
+  const uint32_t col_a = gbase + GL.priv + (uint32_t)warp * (MAXW * 128u) + 4u * lane;
+  const uint32_t bar_id = 1 + grp;
 
   const uint64_t total = P.unit_start[P.count];
   const uint64_t g0 = (uint64_t)blockIdx.x * total / gridDim.x;
   const uint64_t g1 = (uint64_t)(blockIdx.x + 1) * total / gridDim.x;
-  if (g0 >= g1) return;
+  if (g0 >= g1) return;  // the same for every thread of the CTA
+#ifdef DF11_CHECKED
+  if (threadIdx.x == 0) s_check_status = P.status;
+  __syncthreads();
+#endif
 
-  // thread 0 fetches the unit after next's positions one iteration early:
-  // its first output P0, the first output of its second block PM (P1 if it
-  // has one block) and the end of its outputs P1
-  uint32_t nxt_p0 = 0, nxt_p1 = 0, nxt_pm = 0, nxt_m = 0;
-  uint32_t hint = 0;
-  auto issue_stream = [&](uint64_t g, uint32_t stage, uint32_t p0, uint32_t p1, uint32_t pm,
-                          uint32_t m) {
-    const DecMat &M = P.m[m];
-    const uint32_t u = (uint32_t)(g - P.unit_start[m]);
-    // the unit's blocks (the last unit of a matrix may hold one) and the
-    // 16 bytes after them; nothing beyond the stream's and gaps' allocations
-    const uint32_t nb = min(kUnitBlocks, M.n_blocks - kUnitBlocks * u);
-    const uint32_t sbytes = nb * kBlockStreamBytes + 16, gbytes = nb * kBlockGapBytes;
-    const uint32_t st = sbase + (stage ? S.stage1 : S.stage0);
-    meta[stage * 8 + 0] = p0;
-    meta[stage * 8 + 1] = p1;
-    meta[stage * 8 + 2] = m;
-    meta[stage * 8 + 3] = u;
-    meta[stage * 8 + 4] = pm;
-    if (NB > 0) {
-      // fused matmul: row and column of output p0 & ~7
-      const uint32_t base8 = p0 & ~7u;
-      meta[stage * 8 + 5] = base8 / M.cols;
-      meta[stage * 8 + 6] = base8 % M.cols;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(bar_stage + 8 * stage, sbytes + gbytes);
-    bulk_g2s(st, M.stream + (uint64_t)u * (8 * kUnitChunks), sbytes, bar_stage + 8 * stage);
-    bulk_g2s(st + kStreamStage, M.gaps + (uint64_t)u * kGapStage, gbytes, bar_stage + 8 * stage);
-  };
-  auto fetch_pos = [&](uint64_t g) {
-    UnitRef r = locate(P, g, hint);
-    hint = r.m;
-    nxt_m = r.m;
-    const DecMat &M = P.m[r.m];
-    const uint32_t b0 = kUnitBlocks * r.u;
-    nxt_p0 = __ldg(M.pos + b0);
-    nxt_p1 = __ldg(M.pos + min(b0 + kUnitBlocks, M.n_blocks));
-    nxt_pm = b0 + 1 < M.n_blocks ? __ldg(M.pos + b0 + 1) : nxt_p1;
-  };
-
-  // the linear row and the private regions start zeroed (the row's words are
-  // OR-ed into; a region holds zeros beyond its codes)
-  for (uint32_t k = t; k < (S.priv - S.linear) / 4; k += kT) sts32(lin_a + 4 * k, 0u);
-#pragma unroll
-  for (int k = 0; k < MAXW; ++k) sts32(col_a + 128 * k, 0u);
+  // the linear rows start zeroed (the words two threads share are OR-ed into)
+  for (uint32_t k = t; k < (GL.priv - GL.linear) / 16; k += kT) sts128_zero(lin_a + 16 * k);
   if (t == 0) {
     mbar_init(bar_stage, 1);
     mbar_init(bar_stage + 8, 1);
     mbar_init(bar_sm, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    fetch_pos(g0);
-    issue_stream(g0, 0, nxt_p0, nxt_p1, nxt_pm, nxt_m);
-    if (g0 + 1 < g1) fetch_pos(g0 + 1);
   }
-  __syncthreads();
-
-  uint32_t cur_m = 0xFFFFFFFFu;
-  bool table_ok = false, table_short = false;
-  Pending prev{0, 0, nullptr, false, 0, 0, 0};
   if constexpr (NB > 0)
     for (uint32_t k = t; k < NB * kAccRows; k += kT) acc[k] = 0.f;
-  for (uint64_t g = g0, it = 0; g < g1; ++g, ++it) {
-    const uint32_t s = (uint32_t)(it & 1);
-    // [A] the previous unit is relocated into the linear row
-    if (it) __syncthreads();
-    const uint32_t *mt = meta + s * 8;
-    const uint32_t P0 = mt[0], P1 = mt[1], m = mt[2], u = mt[3], PM = mt[4];
-    const uint32_t RL = NB > 0 ? mt[5] : 0u, CL = NB > 0 ? mt[6] : 0u;
-    const DecMat &M = P.m[m];
-    // positions are trusted only as far as they stay inside the matrix and
-    // the staging row; anything else is flagged as corrupt after the count
-    const bool sane = P1 >= P0 && P1 <= M.n && P1 - P0 <= cap;
-    if (t == 0 && g + 1 < g1) {
-      issue_stream(g + 1, s ^ 1, nxt_p0, nxt_p1, nxt_pm, nxt_m);
-      if (g + 2 < g1) fetch_pos(g + 2);
-    }
-    if (m != cur_m) {
-      // new matrix: its decode tables into shared memory
-      const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
-      uint4 *dst = reinterpret_cast<uint4 *>(smem + S.tables);
-      for (uint32_t k = t; k < sizeof(DecodeTables) / 16; k += kT) dst[k] = __ldg(src + k);
-      cur_m = m;
-      __syncthreads();
-      // every table entry must spend at least min_len bits per code, so that
-      // no thread can produce more codes than its private region holds
-      bool tbad = false;
-      for (uint32_t k = t; k < (uint32_t)df11i::kLutSize; k += kT) {
-        const uint32_t e = tab.lut[k], used = e >> 28, ns = (e >> 24) & 0x3u;
-        tbad |= used == 0 || used < ns * P.min_len;
-      }
-      table_ok = !__syncthreads_or(tbad);
-      // every code fits the table: the decode loop needs no long-code test
-      table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
-    }
-    const uint32_t st = sbase + (s ? S.stage1 : S.stage0);
-    bool timed_out = !mbar_wait(bar_stage + 8 * s, (uint32_t)((it >> 1) & 1));
 
-    // ---- this thread's two chunks: decoded once into the private region
-    const uint32_t c0 = u * kUnitChunks + kCPT * t;
-    uint32_t cnt = 0;
-    bool bad = false;
-    if (table_ok && c0 < M.n_chunks) {
-      // stream words W0..W3 of the two chunks and the next chunk's first, W4
-      const uint4 a4 = lds128(st + 16 * t);
-      const uint32_t W0 = bswap32(a4.x), W1 = bswap32(a4.y), W2 = bswap32(a4.z),
-                     W3 = bswap32(a4.w), W4 = bswap32(lds32(st + 16 * t + 16));
-      const uint64_t avail = M.total_bits - 64ull * c0;
-      const uint32_t lim = avail < 64u * kCPT ? (uint32_t)avail : 64u * kCPT;
-      // the first chunk's 5-bit gap
-      const uint32_t q = DF11_GAP_BITS * kCPT * t;
-      const uint32_t ga = st + kStreamStage + (q >> 3);
-      const uint32_t two = (lds8(ga) << 8) | lds8(ga + 1);
-      const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
-      uint32_t p = gap, e = 0, nb = 0, cur = 0, row_a = col_a;
-      if (table_short) {
-        // one loop per 32-bit word in which codes start (each loop's window
-        // needs no select): while p < 32(k+1) the window is Wk:Wk+1 << p % 32
-        const uint32_t l1 = min(lim, 32u), l2 = min(lim, 64u), l3 = min(lim, 96u);
-#pragma unroll 1
-        while (p < l1) {
-          const uint32_t w = __funnelshift_l(W1, W0, p);
-          DF11_STEP(w)
-        }
-#pragma unroll 1
-        while (p < l2) {
-          const uint32_t w = __funnelshift_l(W2, W1, p);
-          DF11_STEP(w)
-        }
-#pragma unroll 1
-        while (p < l3) {
-          const uint32_t w = __funnelshift_l(W3, W2, p);
-          DF11_STEP(w)
-        }
-#pragma unroll 1
-        while (p < lim) {
-          const uint32_t w = __funnelshift_l(W4, W3, p);
-          DF11_STEP(w)
-        }
-      } else {
-        // codes longer than the table's reach: per word a table loop; a
-        // flagged entry leaves it, the code is decoded by the length search
-        // (its 32-bit window lies inside Wk:Wk+1 too), and the loop resumes
-#pragma unroll 1
-        while (p < lim) {
-          const uint32_t k = p >> 5;
-          const uint32_t hi = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
-          const uint32_t lo = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
-          const uint32_t seg = min(lim, 32u * (k + 1));
-          bool flagged = false;
-#pragma unroll 1
-          while (p < seg) {
-            const uint32_t w = __funnelshift_l(lo, hi, p);
-            DF11_STEP_FLAG(w, flagged)
-          }
-          if (!flagged) continue;
-          const uint32_t w = __funnelshift_l(lo, hi, p);
-          const uint32_t L = long_code_len(w, tab);
-          if (L == 0) {
-            bad = true;
-            break;
-          }
-          DF11_APPEND(tab.sym[((w >> (32 - L)) + tab.base[L]) & 0xFFu], 1u << 24)
-          p += L;
-          e = 1u << 24;  // one code: nothing to trim below
-        }
-      }
-      sts32(row_a, cur);  // the word being filled (it may have just begun)
-      uint32_t d = nb >> 3;
-      if (d && p > lim) {
-        // the last entry ran past the end of the thread's chunks: keep its
-        // codes that start before lim, clear the others (byte k of the lane
-        // is byte k % 4 of its word k / 4)
-        const uint32_t ns = (e >> 24) & 0x3u;
-        const uint32_t q1 = p - (e >> 28) + lds8(codelen_a + (e & 0xFFu));
-        const uint32_t q2 = q1 + lds8(codelen_a + ((e >> 8) & 0xFFu));
-        const bool drop2 = ns >= 2 && q1 >= lim;
-        const bool drop3 = ns == 3 && q2 >= lim;
-        const uint32_t k2 = d - ns + 1, k3 = d - 1;
-        sts8_if(col_a + ((k2 >> 2) << 7) + (k2 & 3u), 0u, drop2);
-        sts8_if(col_a + ((k3 >> 2) << 7) + (k3 & 3u), 0u, drop3);
-        d -= (uint32_t)drop2 + (uint32_t)drop3;
-      }
-      cnt = d;
-    }
-    // ---- the previous unit's merge (between decode and the count barrier);
-    // its sign/mantissa phase is waited for even if the unit was rejected,
-    // so that the barrier is never re-armed with a copy in flight
-    if (it) {
-      if (!mbar_wait(bar_sm, (uint32_t)((it - 1) & 1))) timed_out = true;
-      else if (prev.ok) {
-        if constexpr (NB == 0) merge_block(prev, lin_a, sm_a, t);
-        else merge_block_matmul<NB>(prev, lin_a, sm_a, t, acc, P.m[prev.m], P.batch);
-      }
-    }
-    // ---- [B] CTA prefix sum of the counts
-    uint32_t incl = cnt;
-#pragma unroll
-    for (int dd = 1; dd < 32; dd <<= 1) {
-      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, dd);
-      if (lane >= dd) incl += o;
-    }
-    const uint32_t wflags = __ballot_sync(0xffffffffu, bad) ? 0x80000000u : 0u;
-    const uint32_t wtime = __ballot_sync(0xffffffffu, timed_out) ? 0x40000000u : 0u;
-    if (lane == 31) warp_tot[warp] = incl | wflags | wtime;
-    __syncthreads();
-    uint32_t wpre = 0, tot = 0, tot_first = 0, flagbits = 0;
+  uint32_t it = 0;  // units this group has started: stage it & 1, phases from it
+  bool timed_out = false;
+  uint32_t m = 0;
+  while (m + 1 < P.count && g0 >= P.unit_start[m + 1]) ++m;
+  for (; m < P.count && P.unit_start[m] < g1; ++m) {
+    // every group is past the previous matrix (and a timeout anywhere ends
+    // the CTA here, with nothing of its own in flight)
+    if (__syncthreads_or(timed_out)) return;
+    const uint64_t s0 = max(g0, P.unit_start[m]), s1 = min(g1, P.unit_start[m + 1]);
+    if (s0 >= s1) continue;
+    const DecMat &M = P.m[m];
     {
-      const uint4 lo4 = reinterpret_cast<const uint4 *>(warp_tot)[0];
-      const uint4 hi4 = reinterpret_cast<const uint4 *>(warp_tot)[1];
-      const uint32_t x[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
-#pragma unroll
-      for (int i = 0; i < kT / 32; ++i) {
-        flagbits |= x[i];
-        const uint32_t v = x[i] & 0x3FFFFFFFu;
-        tot += v;
-        wpre += i < warp ? v : 0u;
-        tot_first += i < kFirstBlockWarps ? v : 0u;
+      const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
+      uint4 *dst = reinterpret_cast<uint4 *>(smem);
+      for (uint32_t k = threadIdx.x; k < sizeof(DecodeTables) / 16; k += blockDim.x)
+        dst[k] = __ldg(src + k);
+    }
+    __syncthreads();
+    bool tbad = false;
+    for (uint32_t k = threadIdx.x; k < (uint32_t)df11i::kLutSize; k += blockDim.x)
+      tbad |= lut_entry_bad(tab.lut[k].y, P.min_len);
+    // a table that could take a decoder past its region is not used: the
+    // matrix's units decode nothing and are reported as corrupt
+    const bool table_ok = !__syncthreads_or(tbad);
+    // every code fits the table: the decode loop needs no long-code test
+    const bool table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
+
+    const uint64_t first = s0 + grp;
+    if (first >= s1) continue;
+    // thread 0 fetches the positions of the unit after next one iteration
+    // early: its first output P0, the first output of its second block PM
+    // (P1 if it has one block) and the end of its outputs P1
+    uint32_t nxt_p0 = 0, nxt_p1 = 0, nxt_pm = 0;
+    auto fetch_pos = [&](uint64_t g) {
+      const uint32_t b0 = kUnitBlocks * (uint32_t)(g - P.unit_start[m]);
+      DF11_GLOBAL_CHECK(b0 < M.n_blocks, return)
+      nxt_p0 = __ldg(M.pos + b0);
+      nxt_p1 = __ldg(M.pos + min(b0 + kUnitBlocks, M.n_blocks));
+      nxt_pm = b0 + 1 < M.n_blocks ? __ldg(M.pos + b0 + 1) : nxt_p1;
+    };
+    auto issue_stream = [&](uint64_t g, uint32_t stage) {
+      const uint32_t u = (uint32_t)(g - P.unit_start[m]);
+      // the unit's blocks (the last unit of a matrix may hold one) and the
+      // 16 bytes after them; nothing beyond the stream's and gaps' allocations
+      const uint32_t nb = min(kUnitBlocks, M.n_blocks - kUnitBlocks * u);
+      const uint32_t sbytes = nb * kBlockStreamBytes + 16, gbytes = nb * kBlockGapBytes;
+      const uint32_t st = gbase + (stage ? GL.stage1 : GL.stage0);
+      uint32_t *mt = meta + stage * 8;
+      mt[0] = nxt_p0;
+      mt[1] = nxt_p1;
+      mt[2] = u;
+      mt[3] = nxt_pm;
+      if (NB > 0) {
+        // fused matmul: row and column of output p0 & ~7
+        const uint32_t base8 = nxt_p0 & ~7u;
+        mt[4] = base8 / M.cols;
+        mt[5] = base8 % M.cols;
       }
-    }
-    if (flagbits & 0x40000000u) {
-      // a bounded wait ran out: leave (uniformly) with the status set, after
-      // a bounded wait for the next unit's copy issued at the top
-      if (t == 0) {
-        set_status(P.status, DF11_ERR_TIMEOUT);
-        if (g + 1 < g1) mbar_wait(bar_stage + 8 * (s ^ 1), (uint32_t)(((it + 1) >> 1) & 1));
-      }
-      return;
-    }
-    // the codes of the whole unit and of its first block must match the
-    // block positions (every stored position is checked)
-    const bool ok =
-        table_ok && sane && !(flagbits >> 31) && tot == P1 - P0 && tot_first == PM - P0;
-    // fused matmul: the previous unit's row sums (merged before the barrier)
-    if constexpr (NB > 0) {
-      if (it && prev.ok) flush_matmul<NB>(prev, acc, P.m[prev.m], P.batch, t);
-    }
-    if (t == 0) {
-      if (!ok) set_status(P.status, DF11_ERR_CORRUPT);
-      // this unit's sign/mantissa bytes (the previous unit's merge is done),
-      // rounded out to 16 B
-      const uint32_t sm_lo = P0 & ~15u;
-      const uint32_t sm_bytes = sane ? (uint32_t)((((uint64_t)P1 + 15u) & ~15ull) - sm_lo) : 0u;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_expect_tx(bar_sm, sm_bytes);
-      if (sm_bytes) bulk_g2s(sm_a, M.sm + sm_lo, sm_bytes, bar_sm);
+      // (checked build: both sources inside the stream's and gaps' allocations)
+      DF11_GLOBAL_CHECK((uint64_t)u * (8 * kUnitChunks) + sbytes <=
+                                (uint64_t)kBlockStreamBytes * M.n_blocks + 16 &&
+                            (uint64_t)u * kGapStage + gbytes <=
+                                (uint64_t)kBlockGapBytes * M.n_blocks + 16,
+                        {
+                          mbar_expect_tx(bar_stage + 8 * stage, 0);
+                          return;
+                        })
+#ifdef DF11_TEST_HOOKS
+      mbar_expect_tx(bar_stage + 8 * stage, sbytes + gbytes + P.starve_tx);
+#else
+      mbar_expect_tx(bar_stage + 8 * stage, sbytes + gbytes);
+#endif
+      bulk_g2s(st, M.stream + (uint64_t)u * (8 * kUnitChunks), sbytes, bar_stage + 8 * stage);
+      bulk_g2s(st + kStreamStage, M.gaps + (uint64_t)u * kGapStage, gbytes, bar_stage + 8 * stage);
+    };
+    if (t == 0) {
+      fetch_pos(first);
+      issue_stream(first, it & 1);
+      if (first + ngroups < s1) fetch_pos(first + ngroups);
     }
-    // ---- move this thread's exponents to its place in the linear row:
-    // 32-bit words realigned with funnel shifts and OR-ed in (the edge words
-    // are shared with the neighbouring threads); the region is cleared
-    // behind the reads
-    if (cnt) {
-      if (ok) {
-        const uint32_t D = (P0 & 7u) + wpre + incl - cnt;
+    group_sync(bar_id);
+
+    Pending prev{0, 0, nullptr, false, 0, 0, 0, 0};
+    bool have_prev = false;
+    for (uint64_t g = first; g < s1; g += ngroups, ++it) {
+      const uint32_t s = it & 1;
+      // [A] the previous unit is relocated into the linear row
+      if (have_prev) group_sync(bar_id);
+      const uint32_t *mt = meta + s * 8;
+      const uint32_t P0 = mt[0], P1 = mt[1], u = mt[2], PM = mt[3];
+      const uint32_t RL = NB > 0 ? mt[4] : 0u, CL = NB > 0 ? mt[5] : 0u;
+      // positions are trusted only as far as they stay inside the matrix and
+      // the staging row; anything else is flagged as corrupt after the count
+      const bool sane = P1 >= P0 && P1 <= M.n && P1 - P0 <= cap;
+      if (t == 0 && g + ngroups < s1) {
+        issue_stream(g + ngroups, s ^ 1);
+        if (g + 2 * ngroups < s1) fetch_pos(g + 2 * ngroups);
+      }
+      bool tmo = !mbar_wait(bar_stage + 8 * s, (it >> 1) & 1);
+
+      // ---- this thread's two chunks: decoded once into the private region
+      const uint32_t c0 = u * kUnitChunks + kCPT * t;
+      uint32_t cnt = 0;
+      bool bad = false;
+      if (table_ok && c0 < M.n_chunks) {
+        const uint32_t st = gbase + (s ? GL.stage1 : GL.stage0);
+        // stream words W0..W3 of the two chunks and the next chunk's first, W4
+        const uint4 a4 = lds128(st + 16 * t);
+        const uint32_t W0 = bswap32(a4.x), W1 = bswap32(a4.y), W2 = bswap32(a4.z),
+                       W3 = bswap32(a4.w), W4 = bswap32(lds32(st + 16 * t + 16));
+        const uint64_t avail = M.total_bits - 64ull * c0;
+        const uint32_t lim = avail < 64u * kCPT ? (uint32_t)avail : 64u * kCPT;
+        // the first chunk's 5-bit gap
+        const uint32_t q = DF11_GAP_BITS * kCPT * t;
+        const uint32_t ga = st + kStreamStage + (q >> 3);
+        const uint32_t two = (lds8(ga) << 8) | lds8(ga + 1);
+        const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
+        uint32_t p = gap, nb = 0, cur = 0, row_a = col_a, ctrl = 0;
+        if (table_short) {
+          // one loop per 32-bit word in which codes start (each loop's window
+          // needs no select): while p < 32(k+1) the window is Wk:Wk+1 << p % 32
+          const uint32_t l1 = min(lim, 32u), l2 = min(lim, 64u), l3 = min(lim, 96u);
+#pragma unroll 1
+          while (p < l1) DF11_STEP(W0, W1)
+#pragma unroll 1
+          while (p < l2) DF11_STEP(W1, W2)
+#pragma unroll 1
+          while (p < l3) DF11_STEP(W2, W3)
+#pragma unroll 1
+          while (p < lim) DF11_STEP(W3, W4)
+        } else {
+          // codes longer than the table's reach: per word a table loop; a
+          // flagged entry leaves it, the code is decoded by the length search
+          // (its 32-bit window lies inside Wk:Wk+1 too), and the loop resumes
+#pragma unroll 1
+          while (p < lim) {
+            const uint32_t k = p >> 5;
+            const uint32_t hw = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
+            const uint32_t lw = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
+            const uint32_t seg = min(lim, 32u * (k + 1));
+            bool flagged = false;
+#pragma unroll 1
+            while (p < seg) {
+              const uint32_t w = __funnelshift_l(lw, hw, p);
+              const uint2 e = lds64(lut_a + ((w >> (32 - df11i::kLutBits)) << 3));
+              if (e.y & df11i::kCtrlLongFlag) {
+                flagged = true;
+                break;
+              }
+              ctrl = e.y;
+              DF11_APPEND(e.x, ctrl)
+              p = madhi(ctrl, 1u << (32 - df11i::kCtrlUsedShift), p);
+            }
+            if (!flagged) continue;
+            const uint32_t w = __funnelshift_l(lw, hw, p);
+            const uint32_t L = long_code_len(w, tab);
+            if (L == 0) {
+              bad = true;
+              break;
+            }
+            const uint32_t x = tab.sym[((w >> (32 - L)) + tab.base[L]) & 0xFFu];
+            ctrl = kLongCodeCtrl;
+            DF11_APPEND(x, ctrl)
+            p += L;
+          }
+        }
+        sts32(row_a, cur);  // the word being filled (it may have just begun)
+        uint32_t d = (nb & 0x7FFu) >> 3;
+        const uint32_t ncodes = (ctrl >> df11i::kCtrlCountShift) & 7u;
+        if (p > lim && ncodes) {
+          // the last entry ran past the end of the thread's chunks: its codes
+          // that start at or after lim belong to the next thread (an absent
+          // code's start field, 15, is past lim too, as lim - pl < 11)
+          const uint32_t pl = p - (ctrl >> df11i::kCtrlUsedShift);
+          const uint32_t past = (uint32_t)(pl + ((ctrl >> 12) & 15u) >= lim) +
+                                (uint32_t)(pl + ((ctrl >> 16) & 15u) >= lim) +
+                                (uint32_t)(pl + ((ctrl >> 20) & 15u) >= lim);
+          d -= past - (df11i::kLutMaxCodes - ncodes);
+        }
+        cnt = d;
+      }
+      // ---- the previous unit's merge (between decode and the count barrier);
+      // its sign/mantissa phase is waited for even if the unit was rejected,
+      // so that the barrier is never re-armed with a copy in flight
+      if (have_prev) {
+        if (!mbar_wait(bar_sm, (it - 1) & 1)) tmo = true;
+        else if (prev.ok) {
+          if constexpr (NB == 0) merge_unit(prev, lin_a, sm_a, t);
+          else merge_unit_matmul<NB>(prev, lin_a, sm_a, t, acc, P.m[prev.m], P.batch);
+        }
+      }
+      // ---- [B] group prefix sum of the counts
+      uint32_t incl = cnt;
+#pragma unroll
+      for (int dd = 1; dd < 32; dd <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, dd);
+        if (lane >= dd) incl += o;
+      }
+      const uint32_t wflags = __ballot_sync(0xffffffffu, bad) ? 0x80000000u : 0u;
+      const uint32_t wtime = __ballot_sync(0xffffffffu, tmo) ? 0x40000000u : 0u;
+      if (lane == 31) warp_tot[warp] = incl | wflags | wtime;
+      group_sync(bar_id);
+      // lane i < 8 holds warp i's total: the group total, the totals of the
+      // warps before this one and of the first block's warps, and the flags,
+      // each one warp reduction
+      const uint32_t xw = lane < kT / 32 ? warp_tot[lane] : 0u;
+      const uint32_t vw = xw & 0x3FFFFFFFu;
+      const uint32_t flagbits = __reduce_or_sync(0xffffffffu, xw);
+      const uint32_t tot = __reduce_add_sync(0xffffffffu, vw);
+      const uint32_t wpre = __reduce_add_sync(0xffffffffu, lane < warp ? vw : 0u);
+      const uint32_t tot_first = __reduce_add_sync(0xffffffffu, lane < kFirstBlockWarps ? vw : 0u);
+      if (flagbits & 0x40000000u) {
+        // a bounded wait ran out: the group stops (uniformly) with the status
+        // set, after a bounded wait for the next unit's copy issued at the top
+        if (t == 0) {
+          set_status(P.status, DF11_ERR_TIMEOUT);
+          if (g + ngroups < s1) mbar_wait(bar_stage + 8 * (s ^ 1), ((it + 1) >> 1) & 1);
+        }
+        timed_out = true;
+        break;
+      }
+      // the codes of the whole unit and of its first block must match the
+      // block positions (every stored position is checked)
+      const bool ok =
+          table_ok && sane && !(flagbits >> 31) && tot == P1 - P0 && tot_first == PM - P0;
+      // fused matmul: the previous unit's row sums (merged before the barrier)
+      if constexpr (NB > 0) {
+        if (have_prev && prev.ok) flush_matmul<NB>(prev, acc, P.m[prev.m], P.batch, t);
+      }
+      if (t == 0) {
+        if (!ok) set_status(P.status, DF11_ERR_CORRUPT);
+        // this unit's sign/mantissa bytes (the previous unit's merge is done),
+        // rounded out to 16 B
+        const uint32_t sm_lo = P0 & ~15u;
+        uint32_t sm_bytes = sane ? (uint32_t)((((uint64_t)P1 + 15u) & ~15ull) - sm_lo) : 0u;
+        DF11_GLOBAL_CHECK((uint64_t)sm_lo + sm_bytes <= ((M.n + 15) & ~15ull) + 16, sm_bytes = 0)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(bar_sm, sm_bytes);
+        if (sm_bytes) bulk_g2s(sm_a, M.sm + sm_lo, sm_bytes, bar_sm);
+      }
+      // ---- move this thread's exponents to its place in the linear row:
+      // destination word i (from D / 4 on) is source words i-1 and i of the
+      // private row, realigned with a funnel shift.  The first and the last
+      // word may hold a neighbour's bytes too: they are OR-ed in (the row is
+      // zero there); the words between belong to this thread alone and are
+      // stored.  Bytes past the thread's count (codes trimmed above) are
+      // masked off the last word.
+      if (cnt && ok) {
+        const uint32_t D = (P0 & 15u) + wpre + incl - cnt;
         const uint32_t sh = (D & 3u) * 8;
         const uint32_t la = lin_a + (D & ~3u);
-        uint32_t prevw = 0;
-        // words past the thread's last target word OR in zeros (the bytes
-        // beyond its codes are zero) and stay inside the row's slack
-#pragma unroll
-        for (int j = 0; j <= MAXW; ++j) {
-          const uint32_t cur = j < MAXW ? lds32(col_a + 128 * j) : 0u;
-          if (j < MAXW) sts32(col_a + 128 * j, 0u);
-          red_or32(la + 4 * j, __funnelshift_l(prevw, cur, sh));
-          prevw = cur;
+        const uint32_t ndw = ((D + cnt - 1) >> 2) - (D >> 2) + 1;  // destination words
+        const uint32_t nsw = (cnt + 3) >> 2;                        // source words
+        const uint32_t lastmask = 0xFFFFFFFFu >> (8 * (3 - ((D + cnt - 1) & 3u)));
+        uint32_t prevw = lds32(col_a);
+        const uint32_t v0 = __funnelshift_l(0u, prevw, sh);
+        red_or32(la, ndw == 1 ? (v0 & lastmask) : v0);
+        uint32_t i = 1;
+#pragma unroll 4
+        for (; i + 1 < ndw; ++i) {
+          const uint32_t cw = lds32(col_a + 128 * i);
+          sts32(la + 4 * i, __funnelshift_l(prevw, cw, sh));
+          prevw = cw;
         }
+        if (ndw > 1) {
+          const uint32_t cw = i < nsw ? lds32(col_a + 128 * i) : 0u;
+          red_or32(la + 4 * i, __funnelshift_l(prevw, cw, sh) & lastmask);
+        }
+      }
+      prev = Pending{P0, P1, M.out, ok, m, RL, CL, (uint32_t)M.n};
+      have_prev = true;
+    }
+    // the group's last unit of this matrix
+    if (!timed_out && have_prev) {
+      group_sync(bar_id);
+      const bool got = mbar_wait(bar_sm, (it - 1) & 1);
+      if (!got) {
+        if (lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
+        timed_out = true;
+      }
+      if constexpr (NB == 0) {
+        if (got && prev.ok) merge_unit(prev, lin_a, sm_a, t);
       } else {
-        // a rejected unit still leaves the private region cleared
-#pragma unroll
-        for (int k = 0; k < MAXW; ++k) sts32(col_a + 128 * k, 0u);
+        if (got && prev.ok) merge_unit_matmul<NB>(prev, lin_a, sm_a, t, acc, P.m[prev.m], P.batch);
+        group_sync(bar_id);
+        if (got && prev.ok) flush_matmul<NB>(prev, acc, P.m[prev.m], P.batch, t);
       }
     }
-    prev = Pending{P0, P1, M.out, ok, m, RL, CL};
-  }
-  // the last unit's merge
-  __syncthreads();
-  const bool got = mbar_wait(bar_sm, (uint32_t)((g1 - g0 - 1) & 1));
-  if (!got && lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
-  if constexpr (NB == 0) {
-    if (got && prev.ok) merge_block(prev, lin_a, sm_a, t);
-  } else {
-    if (got && prev.ok) merge_block_matmul<NB>(prev, lin_a, sm_a, t, acc, P.m[prev.m], P.batch);
-    __syncthreads();
-    if (got && prev.ok) flush_matmul<NB>(prev, acc, P.m[prev.m], P.batch, t);
   }
 }
 
 #undef DF11_APPEND
-#undef DF11_STEP_FLAG
 #undef DF11_STEP
 
 // ============================================================ launch helpers
@@ -1361,13 +1472,14 @@ DecodeKernel decode_kernel_for(bool wide, uint32_t nb) {
 
 struct DeviceInfo {
   int sms = 0;
+  int smem_optin = 0;  // largest dynamic shared memory per decode CTA
   bool configured = false;
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 
-df11_status device_info(int *dev, int *sms) {
+df11_status device_info(int *dev, int *sms, int *smem_optin = nullptr) {
   if (cudaGetDevice(dev) != cudaSuccess) {
     cudaGetLastError();
     return DF11_ERR_NO_DEVICE;
@@ -1378,19 +1490,27 @@ df11_status device_info(int *dev, int *sms) {
   if (!d.configured) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
       return DF11_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, *dev) !=
+        cudaSuccess)
+      return DF11_ERR_CUDA;
+    // the decode kernels' static shared memory (the checked build has some)
+    // comes out of the same per-CTA limit
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, decode_kernel_for(false, 0)) != cudaSuccess) return DF11_ERR_CUDA;
+    d.smem_optin -= (int)fa.sharedSizeBytes;
     if (cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kHistSmem) != cudaSuccess)
       return DF11_ERR_CUDA;
-    // the largest staging: a unit of codes of one bit, 8 activation rows
-    const int max_smem = (int)smem_layout(64 * kCPT * kT, region_bytes_for(1), 8).total;
     for (int wide = 0; wide < 2; ++wide)
       for (uint32_t nb : {0u, 1u, 2u, 4u, 8u})
         if (cudaFuncSetAttribute(decode_kernel_for(wide != 0, nb),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) != cudaSuccess)
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 d.smem_optin) != cudaSuccess)
           return DF11_ERR_CUDA;
     d.configured = true;
   }
   *sms = d.sms;
+  if (smem_optin) *smem_optin = d.smem_optin;
   return DF11_OK;
 }
 
@@ -1542,13 +1662,13 @@ namespace {
 // and df11_decode_matmul_batch (d_outs == nullptr: products added to io[i].y).
 df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const *d_outs,
                           const df11_matmul_io *io, uint32_t batch, uint32_t *d_status,
-                          df11_stream_t stream) {
+                          df11_stream_t stream, uint32_t starve_tx = 0) {
   if (count == 0) return DF11_OK;
   if (!ms || (!d_outs && !io)) return DF11_ERR_INVALID_ARG;
   const uint32_t nb = io ? (batch <= 1 ? 1u : batch <= 2 ? 2u : batch <= 4 ? 4u : 8u) : 0u;
   if (io && (batch < 1 || batch > DF11_MATMUL_MAX_BATCH)) return DF11_ERR_INVALID_ARG;
-  int dev, sms;
-  df11_status st = device_info(&dev, &sms);
+  int dev, sms, smem_optin;
+  df11_status st = device_info(&dev, &sms, &smem_optin);
   if (st != DF11_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   for (uint32_t first = 0; first < count; first += DF11_MAX_BATCH) {
@@ -1557,6 +1677,11 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
     P.count = 0;
     P.status = d_status;
     P.unit_start[0] = 0;
+#ifdef DF11_TEST_HOOKS
+    P.starve_tx = starve_tx;
+#else
+    (void)starve_tx;
+#endif
     uint32_t min_len = DF11_MAX_CODE_LEN;
     uint32_t unit_codes = 0;  // staging size: most codes in one unit of the batch
     for (uint32_t i = 0; i < k; ++i) {
@@ -1613,20 +1738,26 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
     if (P.count == 0) continue;
     for (uint32_t i = P.count + 1; i <= DF11_MAX_BATCH; ++i) P.unit_start[i] = P.unit_start[P.count];
     P.stage_cap = (unit_codes + 15u) & ~15u;
-    P.region_bytes = 4u * (min_len >= 2 ? kMaxWords2 : kMaxWords1);
     P.min_len = min_len;
     P.batch = io ? batch : 0u;
-    const SmemLayout L = smem_layout(P.stage_cap, P.region_bytes, nb);
-    if (!smem_layout_aligned(L)) return DF11_ERR_INVALID_ARG;
-    const uint32_t smem = L.total;
+    const uint32_t region = 4u * (min_len >= 2 ? kMaxWords2 : kMaxWords1);
+    const GroupLayout GL = group_layout(P.stage_cap, region, nb);
+    const uint64_t units = P.unit_start[P.count];
+    // groups per CTA: as many as one CTA's shared memory holds next to the
+    // tables (one CTA per SM), but no more than there are units per SM
+    if (smem_optin < (int)(kTablesSmem + GL.size)) return DF11_ERR_INVALID_ARG;
+    const uint32_t fit = (uint32_t)((smem_optin - (int)kTablesSmem) / (int)GL.size);
+    const uint32_t groups = (uint32_t)std::min<uint64_t>(
+        std::min<uint32_t>(kMaxGroups, fit), std::max<uint64_t>(1, cdiv(units, (uint64_t)sms)));
+    const uint32_t smem = kTablesSmem + groups * GL.size;
     const DecodeKernel kern = decode_kernel_for(min_len < 2, nb);
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kT, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, (int)(groups * kT), smem) !=
+        cudaSuccess)
       return DF11_ERR_CUDA;
     if (occ < 1) return DF11_ERR_CUDA;
-    const uint64_t units = P.unit_start[P.count];
-    const uint64_t grid = std::min<uint64_t>(units, (uint64_t)sms * occ);
-    kern<<<(unsigned)grid, kT, smem, s>>>(P);
+    const uint64_t grid = std::min<uint64_t>(cdiv(units, groups), (uint64_t)sms * occ);
+    kern<<<(unsigned)grid, groups * kT, smem, s>>>(P);
     st = launch_status();
     if (st != DF11_OK) return st;
   }
@@ -1655,6 +1786,20 @@ extern "C" df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32
   return df11_decode_block_batch(m, 1, &d_out, d_status, stream);
 }
 
+#ifdef DF11_TEST_HOOKS
+// Test build only (not in the product library): df11_decode whose stream-stage
+// barriers each expect 16 bytes more than their bulk copies deliver.  Every
+// copy lands, but no stage barrier completes, so each bounded wait runs out
+// and the kernel must end with DF11_ERR_TIMEOUT in *d_status, nothing of its
+// own in flight and nothing written outside d_out.
+extern "C" df11_status df11_test_decode_starved(const df11_matrix *m, uint16_t *d_out,
+                                                uint32_t *d_status, df11_stream_t stream) {
+  if (!m || !d_out) return DF11_ERR_INVALID_ARG;
+  uint16_t *outs[1] = {d_out};
+  return launch_decode(m, 1, outs, nullptr, 0, d_status, stream, 16u);
+}
+#endif
+
 // ============================================================ encode without allocation
 //
 // df11_encode needs a scratch buffer from its caller (the per-tile bit
@@ -1681,7 +1826,9 @@ static __device__ __align__(256) uint64_t g_static_tile_offsets[kStaticTiles];
 std::mutex g_static_mu;
 uint64_t *g_static_ptr[64] = {nullptr};
 
-// Device address of the array on the current device, looked up once per device.
+// Device address of the array on the current device, looked up once per device
+// and kept for the life of the process (a device reset after the first call
+// is not supported: the address would belong to the destroyed context).
 df11_status static_scratch(int dev, uint64_t **ptr) {
   std::lock_guard<std::mutex> lk(g_static_mu);
   if (!g_static_ptr[dev]) {
@@ -1706,7 +1853,8 @@ extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
   if (n > DF11_STATIC_WS_MAX_N) return DF11_ERR_TOO_LARGE;
   df11_status st = check_encode_out(d_w, n, total_bits, out);
   if (st != DF11_OK) return st;
-  if (cdiv(n, df11i::kEncTile) + 1 > kStaticTiles) return DF11_ERR_TOO_LARGE;
+  // (n <= DF11_STATIC_WS_MAX_N gives at most kStaticTiles - 1 tiles plus the
+  // total: the static_assert next to the array ties the two limits together)
   EncCodebook ecb;
   if ((st = host_enc_codebook(cb, &ecb)) != DF11_OK) return st;
   int dev, sms;

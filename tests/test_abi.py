@@ -144,25 +144,39 @@ def tables_of(cb):
     return buf
 
 
-def greedy_window(codes_by_str, bits12):
-    """Up to three whole codes from the left of a 12-bit string."""
-    out, used = [], 0
-    while len(out) < 3:
+TABLE_BITS = df11.TABLE_BITS      # 11: the lookup table's window
+LONG_FLAG = 1 << 26
+
+
+def ror8(e: int) -> int:
+    """The decoder's stored form of an exponent byte: rotated right by one bit."""
+    return ((e >> 1) | (e << 7)) & 0xFF
+
+
+def greedy_window(codes_by_str, bits):
+    """Up to four whole codes from the left of a window string, with their starts."""
+    out, starts, used = [], [], 0
+    while len(out) < 4:
         found = None
-        for L in range(1, 13 - used):
-            s = bits12[used:used + L]
+        for L in range(1, len(bits) + 1 - used):
+            s = bits[used:used + L]
             if s in codes_by_str:
                 found = (codes_by_str[s], L)
                 break
         if found is None:
             break
         out.append(found[0])
+        starts.append(used)
         used += found[1]
-    return out, used
+    return out, starts, used
 
 
 @pytest.mark.parametrize("which", ["workload1", "uniform", "fibonacci34", "two", "skew"])
 def test_decode_table_against_oracle_codes(lib, which):
+    """The library's decode tables describe the oracle's code: every window of
+    the lookup table decodes, greedily, the codes the oracle's canonical code
+    gives for those bits (at most four, with each one's start), and the
+    long-code arrays decode every code canonically."""
     if which == "workload1":
         h = oracle.histogram(oracle.split(workloads.matrix(1, 0))[0])
     elif which == "uniform":
@@ -177,7 +191,8 @@ def test_decode_table_against_oracle_codes(lib, which):
     oln, ocode = oracle.codebook(h)
     codes_by_str = {format(int(ocode[s]), f"0{int(oln[s])}b"): s for s in range(256) if oln[s]}
     tab = tables_of(cb)
-    lut = tab[: 4 * 4096].view(np.uint32)
+    K = TABLE_BITS
+    lut = tab[: 8 << K].view(np.uint32).reshape(-1, 2)
     # the long-code arrays: limit u64[33], base u32[33], codelen u8[256], sym u8[256], then
     # max_len, min_len, n_symbols, lut_bits
     limit = tab[16384:16384 + 264].view(np.uint64)
@@ -187,23 +202,26 @@ def test_decode_table_against_oracle_codes(lib, which):
     max_len, min_len, n_sym, lut_bits = tab[17292:17308].view(np.uint32)
     assert np.array_equal(codelen, oln)
     nz = oln[oln > 0]
-    assert (max_len, min_len, n_sym, lut_bits) == (nz.max(), nz.min(), nz.size, 12)
+    assert (max_len, min_len, n_sym, lut_bits) == (nz.max(), nz.min(), nz.size, K)
     for L in range(1, 33):
         at_L = [s_ for s_ in range(256) if oln[s_] == L]
         for s_ in at_L:   # canonical decoding of a long code: sym[code + base[L]]
-            assert sym[(int(ocode[s_]) + int(base[L])) % 2 ** 32] == s_
+            assert sym[(int(ocode[s_]) + int(base[L])) % 2 ** 32] == ror8(s_)
         if at_L:
             first = min(int(ocode[s_]) for s_ in at_L)
             assert int(limit[L]) == (first + len(at_L)) << (32 - L)
-    for v in range(4096):
-        syms, used = greedy_window(codes_by_str, format(v, "012b"))
-        e = int(lut[v])
+    for v in range(1 << K):
+        syms, starts, used = greedy_window(codes_by_str, format(v, f"0{K}b"))
+        x, c = int(lut[v, 0]), int(lut[v, 1])
         if not syms:
-            assert e == (12 << 28) | (1 << 26), (v, hex(e))  # long-code flag, 12 bits skipped
+            # long-code flag; the window's bits counted as consumed, no codes
+            assert x == 0 and c == (K << 28) | (0xFFF << 12) | LONG_FLAG, (v, hex(c))
             continue
-        assert e >> 28 == used and (e >> 24) & 3 == len(syms) and not e & (1 << 26)
-        assert [(e >> (8 * i)) & 0xFF for i in range(len(syms))] == syms
-        assert e & 0xFFFFFF == sum(s << (8 * i) for i, s in enumerate(syms))
+        n = len(syms)
+        fields = [starts[j] if j < n else 15 for j in (1, 2, 3)]
+        assert c == (used << 28) | (n << 3) | (fields[0] << 12) | (fields[1] << 16) | \
+            (fields[2] << 20), (v, hex(c))
+        assert x == sum(ror8(s) << (8 * i) for i, s in enumerate(syms)), (v, hex(x))
 
 
 def test_validate_accepts_oracle_metadata_and_rejects_corruption(lib):

@@ -56,11 +56,12 @@ class Guarded:
 def _cases():
     return [
         ("fibonacci_cap32", lambda: workloads.fibonacci_exponents(34), 32),
+        ("matrix_4096x4096_cap11", lambda: workloads.matrix(2, 0), 11),
         ("matrix_4096x4096_cap12", lambda: workloads.matrix(2, 0), 12),
-        ("random_1000003_cap12", lambda: workloads.random_bf16(1_000_003, seed=2003), 12),
+        ("random_1000003_cap11", lambda: workloads.random_bf16(1_000_003, seed=2003), 11),
         ("random_1000003_cap32", lambda: workloads.random_bf16(1_000_003, seed=2004), 32),
-        ("single_symbol_65537", lambda: workloads.constant(65_537, 0x3F80), 12),
-        ("seventeen_values", lambda: workloads.random_bf16(17, seed=5), 12),
+        ("single_symbol_65537", lambda: workloads.constant(65_537, 0x3F80), 11),
+        ("seventeen_values", lambda: workloads.random_bf16(17, seed=5), 11),
     ]
 
 

@@ -80,16 +80,17 @@ def histograms():
             h = np.zeros(256, np.uint64)
             h[g.choice(256, m, replace=False)] = g.integers(1, 10 ** int(g.integers(1, 7)), m)
             out.append((f"random_{m}", h, 32))
-            out.append((f"random_{m}_cap12", h, 12))
+            out.append((f"random_{m}_cap11", h, 11))
     fib = np.zeros(256, np.uint64)
     fib[50:50 + 34] = workloads.fibonacci_counts(34)
-    out += [("fibonacci_cap32", fib, 32), ("fibonacci_cap12", fib, 12), ("fibonacci_cap6", fib, 6)]
+    out += [("fibonacci_cap32", fib, 32), ("fibonacci_cap12", fib, 12), ("fibonacci_cap11", fib, 11),
+            ("fibonacci_cap6", fib, 6)]
     one = np.zeros(256, np.uint64)
     one[127] = 1000
-    out += [("one_symbol", one, 12), ("empty", np.zeros(256, np.uint64), 12),
+    out += [("one_symbol", one, 11), ("empty", np.zeros(256, np.uint64), 11),
             ("all_equal_cap8", np.full(256, 9, np.uint64), 8)]
     x = workloads.matrix(2, 0).reshape(-1)
-    out.append(("matrix_4096x4096", oracle.histogram(oracle.split(x)[0]), 12))
+    out.append(("matrix_4096x4096", oracle.histogram(oracle.split(x)[0]), 11))
     return out
 
 
@@ -122,7 +123,7 @@ def test_device_compressor_equals_compress_block(codec):
     xs += [workloads.fibonacci_exponents(30)[:300_000], workloads.constant(5000, 0x3F80),
            workloads.random_bf16(17, seed=3), workloads.all_patterns()]
     ws = [to_dev(x) for x in xs]
-    for cap in (12, 32):
+    for cap in (11, 32):
         a = codec.compress_block(ws, cap=cap)
         b = codec.compress_block_device(ws, cap=cap)
         for ma, mb, x in zip(a, b, xs):

@@ -7,10 +7,10 @@ Expected values come from the oracle only.  Where the expected decode output
 is the input itself, that is the oracle's own result: its round trip is the
 identity (pinned in test_oracle_pins.py) and small cases call it explicitly.
 
-Every case runs under two code-length caps: 12 (the codec default, the decode
-table's reach: the fast path) and 32 (the format's limit: codes longer than
-the table take the length search).  The oracle builds its codebook with the
-same cap."""
+Every case runs under three code-length caps: 11 (the codec default, the
+decode table's reach: the fast path), 12 (codes one bit longer than the
+table: the length search for the rarest values) and 32 (the format's limit).
+The oracle builds its codebook with the same cap."""
 import numpy as np
 import pytest
 import torch
@@ -47,7 +47,7 @@ def assert_encoded_equal(m, enc):
     assert np.array_equal(h["sign_mantissa"], enc.sign_mantissa), "sign/mantissa differ"
 
 
-CAPS = [12, 32]
+CAPS = [11, 12, 32]
 
 
 def full_check(codec, x: np.ndarray, cap: int, call_oracle_decode: bool = True):
@@ -113,17 +113,18 @@ def test_worked_example(codec, cap):
 
 def test_fibonacci_length_cap(codec):
     """14,930,351 values whose exponent counts are Fibonacci numbers: the code
-    needs the 32-bit cap, so 20 of the codes are longer than the 12-bit
+    needs the 32-bit cap, so 21 of the codes are longer than the 11-bit
     decode table and take the length-search path."""
     m, enc = full_check(codec, workloads.fibonacci_exponents(34), 32, call_oracle_decode=False)
     assert int(enc.lengths.max()) == 32
 
 
-def test_fibonacci_at_table_cap(codec):
-    """The same input under the 12-bit cap: package-merge shortens every code
-    to the table's reach."""
-    m, enc = full_check(codec, workloads.fibonacci_exponents(34), 12, call_oracle_decode=False)
-    assert int(enc.lengths.max()) == 12
+@pytest.mark.parametrize("cap", [11, 12])
+def test_fibonacci_at_table_cap(codec, cap):
+    """The same input under the table's 11-bit cap (package-merge shortens
+    every code to the table's reach) and one bit above it."""
+    m, enc = full_check(codec, workloads.fibonacci_exponents(34), cap, call_oracle_decode=False)
+    assert int(enc.lengths.max()) == cap
 
 
 @pytest.mark.parametrize("cap", CAPS)
@@ -134,10 +135,10 @@ def test_workload_single_matrix(codec, wid, cap):
     assert m.stored_bytes == oracle.stored_bytes(enc)
 
 
-@pytest.mark.parametrize("wid,cap", [(3, 12), (3, 32), (5, 12), (5, 32)])
+@pytest.mark.parametrize("wid,cap", [(3, 11), (3, 32), (5, 11), (5, 12), (5, 32)])
 def test_workload_block_batched(codec, wid, cap):
     """A whole transformer block: per-matrix codebooks, one decode launch
-    (the bench configuration, cap 12; and cap 32)."""
+    (the bench configuration, cap 11; and caps 12 and 32)."""
     names = [nm for nm, _ in workloads.WORKLOADS[wid][1]]
     mats, xs = [], []
     for i, _ in enumerate(names):
