@@ -19,10 +19,12 @@ import numpy as np
 import torch
 
 from . import (CODEBOOK_BYTES, MAX_CODE_LEN, TABLE_BITS, DF11Error, check, df11_build_codebook,
-               df11_build_codebook_device, df11_build_tables, df11_codebook, df11_decode,
-               df11_decode_block_batch, df11_decode_matmul_batch, df11_encode,
-               df11_encode_device_codebook, df11_encoded, df11_matmul_io, df11_encoded_sizes,
-               df11_histogram, df11_matrix, df11_sizes, df11_sizes_from_bits, df11_tables_bytes)
+               df11_build_codebook_device, df11_build_tables, df11_codebook,
+               df11_codebook_from_lengths, df11_decode, df11_decode_block_batch,
+               df11_decode_matmul_batch, df11_encode, df11_encode_device_codebook, df11_encoded,
+               df11_encoded_sizes, df11_file_bytes, df11_histogram, df11_host_matrix, df11_matmul_io,
+               df11_matrix, df11_read, df11_sizes, df11_sizes_from_bits, df11_tables_bytes,
+               df11_write)
 
 
 def _stream_handle(stream) -> int:
@@ -359,18 +361,8 @@ def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, st
     """Upload stored arrays (e.g. produced elsewhere) into padded device
     buffers ready for decoding."""
     hist = np.zeros(256, np.uint64)
-    # sizes only depend on n, total_bits and the code lengths' extremes
-    sizes = df11_sizes()
-    C = (total_bits + 63) // 64
-    B = (C + 255) // 256
-    sizes.n, sizes.total_bits, sizes.n_chunks, sizes.n_blocks = n, total_bits, C, B
-    sizes.stream_bytes, sizes.gaps_bytes = 8 * C, (5 * C + 7) // 8
-    sizes.block_pos_bytes, sizes.sign_mantissa_bytes = 4 * (B + 1), n
-    sizes.stored_bytes = sizes.stream_bytes + sizes.gaps_bytes + sizes.block_pos_bytes + n + 256
-    sizes.stream_alloc, sizes.gaps_alloc = 2048 * B + 16, 160 * B + 16
-    sizes.block_pos_alloc = ((4 * (B + 1) + 15) // 16) * 16
-    sizes.sign_mantissa_alloc = ((n + 15) // 16) * 16 + 16
-    sizes.tables_bytes = df11_tables_bytes()
+    st, sizes = df11_sizes_from_bits(n, total_bits)
+    check(st, "df11_sizes_from_bits")
 
     def padded(a, size, dtype=np.uint8):
         buf = np.zeros(size // np.dtype(dtype).itemsize, dtype)
@@ -385,6 +377,71 @@ def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, st
                                        sizes.block_pos_alloc, np.int32),
                       sign_mantissa=padded(sign_mantissa, sizes.sign_mantissa_alloc),
                       tables=build_tables(codebook, device), hist=hist)
+
+
+def serialize(m: DF11Matrix) -> np.ndarray:
+    """The matrix in the .df11 container (include/df11.h), as a uint8 array."""
+    h = m.host_arrays()
+    arrs = {k: np.ascontiguousarray(v) for k, v in h.items()}
+    hm = df11_host_matrix(n=m.n, total_bits=m.total_bits, cap=int(m.codebook.cap),
+                          max_block_codes=int(m.max_block_codes), ndim=len(m.shape))
+    if len(m.shape) > 4:
+        raise ValueError("serialize: at most 4 dimensions")
+    for i, d in enumerate(m.shape):
+        hm.shape[i] = int(d)
+    hm.lengths = arrs["lengths"].ctypes.data
+    hm.gaps = arrs["gaps"].ctypes.data
+    hm.block_pos = arrs["block_pos"].ctypes.data
+    hm.stream = arrs["stream"].ctypes.data
+    hm.sign_mantissa = arrs["sign_mantissa"].ctypes.data
+    size = df11_file_bytes(m.n, m.total_bits)
+    buf = np.empty(size, np.uint8)
+    st, written = df11_write(hm, buf.ctypes.data, size)
+    check(st, "df11_write")
+    assert written == size
+    return buf
+
+
+def deserialize(data, device) -> DF11Matrix:
+    """A matrix read from the .df11 container (bytes or a uint8 array), checked
+    (magic, sizes, CRC-32, metadata) by the library and uploaded to device."""
+    buf = np.frombuffer(data, np.uint8) if not isinstance(data, np.ndarray) else data
+    buf = np.ascontiguousarray(buf, np.uint8)
+    st, hm = df11_read(buf.ctypes.data, buf.size)
+    check(st, "df11_read")
+    base = buf.ctypes.data
+    st, sizes = df11_sizes_from_bits(hm.n, hm.total_bits)
+    check(st, "df11_sizes_from_bits")
+
+    def view(ptr, nbytes):
+        off = int(ptr) - base
+        return buf[off:off + int(nbytes)]
+
+    lengths = view(hm.lengths, 256)
+    st, cb = df11_codebook_from_lengths(lengths.ctypes.data, int(hm.cap) or MAX_CODE_LEN)
+    check(st, "df11_codebook_from_lengths")
+    shape = tuple(int(hm.shape[i]) for i in range(hm.ndim)) if hm.ndim else (int(hm.n),)
+    m = from_host_arrays(shape, int(hm.n), int(hm.total_bits), cb,
+                         view(hm.stream, sizes.stream_bytes), view(hm.gaps, sizes.gaps_bytes),
+                         view(hm.block_pos, sizes.block_pos_bytes).view(np.uint32),
+                         view(hm.sign_mantissa, sizes.sign_mantissa_bytes), device)
+    m.max_block_codes = int(hm.max_block_codes)
+    return m
+
+
+def save(path: str, m: DF11Matrix) -> int:
+    """Write the matrix to a .df11 file; returns the bytes written."""
+    buf = serialize(m)
+    with open(path, "wb") as f:
+        f.write(buf.tobytes())
+    return int(buf.size)
+
+
+def load(path: str, device="cuda") -> DF11Matrix:
+    """Read a .df11 file into device buffers ready for decoding."""
+    with open(path, "rb") as f:
+        data = f.read()
+    return deserialize(data, device)
 
 
 def codebook_from_lengths(lengths, codes) -> df11_codebook:
@@ -403,4 +460,4 @@ def codebook_from_lengths(lengths, codes) -> df11_codebook:
 
 __all__ = ["DF11Matrix", "histogram", "compress", "decompress", "decompress_block",
            "build_tables", "alloc_encoded", "from_host_arrays", "codebook_from_lengths",
-           "ctypes"]
+           "serialize", "deserialize", "save", "load", "ctypes"]
