@@ -10,6 +10,11 @@ block with PyTorch (cuBLAS matmuls, scaled-dot-product attention) and releases
 the buffer, unless the caller passes one to reuse.  The decoded weights are
 bit-identical to the originals, so the forward equals, bit for bit, the same
 forward on resident BF16 weights (forward_reference).
+
+The same page compresses the embedding table and the LM head too, but does not
+batch them with a block: DF11Embedding and DF11LMHead each hold one matrix in
+DF11 form and decode it with one df11_decode launch right before their lookup
+or projection, dropping the BF16 copy after it.
 """
 from __future__ import annotations
 
@@ -124,3 +129,57 @@ class DF11Block:
     def forward_reference(self, x: torch.Tensor, weights: dict[str, torch.Tensor]) -> torch.Tensor:
         """The same forward on resident BF16 weights."""
         return block_forward(x, weights, self.shape)
+
+
+class _DF11Single:
+    """One matrix in DF11 form, decoded by one df11_decode launch on use."""
+
+    def __init__(self, mat: codec.DF11Matrix):
+        if len(mat.shape) != 2:
+            raise ValueError(f"expected a 2-D matrix, got shape {tuple(mat.shape)}")
+        self.mat = mat
+
+    @classmethod
+    def compress(cls, weight: torch.Tensor, cap: int = codec.DEFAULT_CAP):
+        if weight.dim() != 2 or weight.dtype != torch.bfloat16:
+            raise ValueError("expected a 2-D BF16 weight")
+        return cls(codec.compress(weight, cap=cap))
+
+    @property
+    def stored_bytes(self) -> int:
+        return self.mat.stored_bytes
+
+    def decode(self, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """The BF16 matrix (into out when given: a BF16 tensor of its shape)."""
+        return codec.decompress(self.mat, out=out, stream=stream)
+
+
+class DF11Embedding(_DF11Single):
+    """A (vocab, hidden) embedding table in DF11 form."""
+
+    def forward(self, ids: torch.Tensor, scratch: torch.Tensor | None = None) -> torch.Tensor:
+        """Rows of the table for the token ids: the table is decoded, the rows
+        gathered, and the decoded table dropped (unless it is the caller's
+        scratch)."""
+        w = self.decode(scratch)
+        y = F.embedding(ids, w)
+        del w
+        return y
+
+    def forward_reference(self, ids: torch.Tensor, weight: torch.Tensor) -> torch.Tensor:
+        return F.embedding(ids, weight)
+
+
+class DF11LMHead(_DF11Single):
+    """A (vocab, hidden) output projection in DF11 form."""
+
+    def forward(self, x: torch.Tensor, scratch: torch.Tensor | None = None) -> torch.Tensor:
+        """Logits x W^T: W is decoded, used, and dropped (unless it is the
+        caller's scratch)."""
+        w = self.decode(scratch)
+        y = F.linear(x, w)
+        del w
+        return y
+
+    def forward_reference(self, x: torch.Tensor, weight: torch.Tensor) -> torch.Tensor:
+        return F.linear(x, weight)

@@ -62,3 +62,25 @@ def test_shape_mismatch_rejected(blockmod):
     blk = blockmod.DF11Block.compress(w, shape)
     with pytest.raises(ValueError):
         blockmod.DF11Block(blk.mats, blockmod.BlockShape(hidden=512, heads=8, kv_heads=4, ffn=1536))
+
+
+@pytest.mark.parametrize("vocab,hidden", [(1000, 512), (32768, 1024)])
+def test_embedding_and_lm_head_match_resident(blockmod, vocab, hidden):
+    """The embedding lookup and the LM-head projection on a table held in
+    DF11 form equal, bit for bit, the same operations on the resident table;
+    a caller-owned scratch buffer gives the same result."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(vocab)
+    w = (torch.randn(vocab, hidden, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    emb = blockmod.DF11Embedding.compress(w)
+    head = blockmod.DF11LMHead(emb.mat)
+    ids = torch.randint(0, vocab, (3, 17), generator=g, device="cuda")
+    assert torch.equal(emb.forward(ids), emb.forward_reference(ids, w))
+    x = torch.randn(3, 17, hidden, generator=g, device="cuda").to(torch.bfloat16)
+    assert torch.equal(head.forward(x), head.forward_reference(x, w))
+    scratch = torch.empty(vocab, hidden, dtype=torch.bfloat16, device="cuda")
+    assert torch.equal(head.forward(x, scratch=scratch), head.forward_reference(x, w))
+    assert torch.equal(scratch.view(torch.int16), w.view(torch.int16))
+    assert emb.stored_bytes < 0.8 * w.numel() * 2
+    with pytest.raises(ValueError):
+        blockmod.DF11Embedding.compress(w.reshape(-1))
