@@ -93,3 +93,35 @@ def test_static_workspace_encode_rejects_oversized_input(df11):
     st = df11.df11_encode_static_ws(small.data_ptr(), n, cb, n, abi, status.data_ptr(),
                                     torch.cuda.current_stream().cuda_stream)
     assert st == df11.DF11_ERR_TOO_LARGE
+
+
+def test_static_workspace_encode_allocates_no_device_memory(df11):
+    """With every buffer allocated beforehand and one warm-up call made (the
+    first call on a device looks up the array's address and loads the
+    kernels), a further call leaves the device's free memory unchanged."""
+    dev = torch.device("cuda", 0)
+    x = workloads.random_bf16(3_000_001, seed=78)
+    w = torch.from_numpy(x.view(np.int16)).to(dev)
+    n = w.numel()
+    stream = torch.cuda.current_stream().cuda_stream
+    hist = torch.empty(256, dtype=torch.int64, device=dev)
+    df11.check(df11.df11_histogram(w.data_ptr(), n, hist.data_ptr(), stream), "df11_histogram")
+    h = hist.cpu().numpy().view(np.uint64)
+    st, cb = df11.df11_build_codebook(h, 11)
+    df11.check(st, "df11_build_codebook")
+    st, sizes = df11.df11_encoded_sizes(cb, h, n)
+    df11.check(st, "df11_encoded_sizes")
+    bufs, abi = _outputs(df11, sizes, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        df11.check(df11.df11_encode_static_ws(w.data_ptr(), n, cb, sizes.total_bits, abi,
+                                              status.data_ptr(), stream), "df11_encode_static_ws")
+        torch.cuda.synchronize()
+
+    call()
+    free_before, _ = torch.cuda.mem_get_info(dev)
+    call()
+    free_after, _ = torch.cuda.mem_get_info(dev)
+    assert free_after == free_before
+    assert int(status.item()) == 0
