@@ -855,7 +855,7 @@ constexpr uint32_t kLongCodeCtrl =
     sts32(row_a, lo);                                                       \
     const uint32_t nb2 = nb + (add);                                        \
     row_a = col_a + ((nb2 & 0x7E0u) << 2);                                  \
-    cur = __funnelshift_rc(lo, hi, (nb ^ nb2) & 32u);                       \
+    cur = ((nb ^ nb2) & 32u) ? hi : lo;                                     \
     nb = nb2;                                                               \
   }
 

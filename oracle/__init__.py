@@ -76,6 +76,7 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "oracle_total_bits": (c_int, [_u8p, c_u64, _u8p, _u64p]),
         "oracle_encode": (c_int, [_u8p, c_u64, _u8p, _u32p, c_u64, _u8p, _u8p, _u32p]),
         "oracle_pack_gaps": (None, [_u8p, c_u64, _u8p]),
+        "oracle_run_index": (c_int, [_u8p, c_u64, _u8p, c_u64, ctypes.POINTER(ctypes.c_uint16)]),
         "oracle_unpack_gaps": (None, [_u8p, c_u64, _u8p]),
         "oracle_decode_serial": (c_int, [_u8p, c_u64, c_u64, _u8p, _u32p, _u8p]),
         "oracle_decode_chunked": (c_int, [_u8p, _u8p, _u32p, c_u64, c_u64, _u8p, _u32p, _u8p]),
@@ -255,6 +256,21 @@ def encode(w: np.ndarray, cap: int = MAX_CAP, lengths=None, codes=None, lib=None
     return Encoded(n=n, hist=h, lengths=lengths, codes=codes, total_bits=total_bits,
                    stream=stream, gaps=gaps, gaps_packed=pack_gaps(gaps, lib), block_pos=pos,
                    sign_mantissa=sm)
+
+
+def run_index(w: np.ndarray, lengths, total_bits: int, lib=None) -> np.ndarray:
+    """R8: for each 128-bit run of each 256-chunk block, the number of codes
+    that start in the block before the run (uint16, 128 per block)."""
+    lib = lib or load()
+    e, _ = split(w, lib)
+    chunks = (total_bits + CHUNK_BITS - 1) // CHUNK_BITS
+    blocks = (chunks + BLOCK_CHUNKS - 1) // BLOCK_CHUNKS
+    out = np.zeros(blocks * (BLOCK_CHUNKS // 2), np.uint16)
+    r = lib.oracle_run_index(_p(e, _u8p), e.size, _p(np.ascontiguousarray(lengths, np.uint8), _u8p),
+                             total_bits, _p(out, ctypes.POINTER(ctypes.c_uint16)))
+    if r != OK:
+        raise ValueError(f"oracle_run_index failed with {r}")
+    return out
 
 
 def decode_serial_exponents(stream, total_bits: int, n: int, lengths, codes, lib=None) -> np.ndarray:

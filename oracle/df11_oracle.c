@@ -38,6 +38,9 @@
  *      packed 5 bits per chunk, most significant bit first.
  *   R7 block positions: 256 chunks per block; pos[b] = number of codes that
  *      start before bit 64*256*b; pos[B] = n; stored as uint32.
+ *   R8 run index (device-side metadata derived from the stream): for run r
+ *      of block b (chunks 2r and 2r+1 of the block), the number of codes that
+ *      start in the block before the run, as uint16.
  *
  * Parity status: every function here is pinned by a test in
  * tests/test_oracle_pins.py (closed forms, brute force, textbook identities,
@@ -408,6 +411,48 @@ int oracle_encode(const uint8_t *exponent, uint64_t n, const uint8_t len[256],
   pos[blocks] = (uint32_t)n;
   for (uint64_t c = 0; c < chunks; c++)
     if (gap[c] > 31) return OR_ERR_CORRUPT;
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Run index: for each 128-bit run (two consecutive chunks, the part of */
+/* a block one decoding thread takes), the output position of its first */
+/* code within its block.  [Kernel] gives one output position per       */
+/* thread block; this is the same count one level finer.  R8 (reading): */
+/* run_pos[128*b + r] = number of codes that start at bits              */
+/* [16384*b, 16384*b + 128*r); every block has 128 entries (runs past   */
+/* the end of the stream hold the block's total).  Written from the     */
+/* code lengths, one code start at a time.                              */
+/* run_pos must hold 128*B entries, B = ceil(C/256).                    */
+/* ------------------------------------------------------------------ */
+int oracle_run_index(const uint8_t *exponent, uint64_t n, const uint8_t len[256],
+                     uint64_t total_bits, uint16_t *run_pos) {
+  uint64_t chunks = (total_bits + OR_CHUNK_BITS - 1) / OR_CHUNK_BITS;
+  uint64_t blocks = (chunks + OR_BLOCK_CHUNKS - 1) / OR_BLOCK_CHUNKS;
+  uint64_t runs = blocks * (OR_BLOCK_CHUNKS / 2);
+  uint64_t run_bits = 2 * OR_CHUNK_BITS;
+  uint64_t runs_per_block = OR_BLOCK_CHUNKS / 2;
+  uint64_t bit = 0, next_run = 0, block_first = 0;
+  for (uint64_t i = 0; i < n; i++) {
+    unsigned l = len[exponent[i]];
+    if (l == 0) return OR_ERR_SYMBOL;
+    /* every run boundary at or before this code's start: the codes of
+       the boundary's block that started before it are i - (block's first) */
+    while (next_run < runs && next_run * run_bits <= bit) {
+      if (next_run % runs_per_block == 0) block_first = i;
+      uint64_t before = i - block_first;
+      if (before > 0xFFFFu) return OR_ERR_CORRUPT;
+      run_pos[next_run] = (uint16_t)before;
+      next_run++;
+    }
+    bit += l;
+  }
+  if (bit != total_bits) return OR_ERR_ARG;
+  while (next_run < runs) {
+    if (next_run % runs_per_block == 0) block_first = n;
+    run_pos[next_run] = (uint16_t)(n - block_first);
+    next_run++;
+  }
   return OR_OK;
 }
 

@@ -13,7 +13,7 @@ import pytest
 import oracle
 import workloads
 import test_oracle_rans as rp
-from test_oracle_pins import GOLDEN, cost, kraft, textbook_huffman_cost, hist_from
+from test_oracle_pins import GOLDEN, _run_index_by_search, cost, kraft, textbook_huffman_cost, hist_from
 
 MUTATIONS = {
     "lsb_first_bits": [("(uint8_t)(0x80u >> (k & 7u))", "(uint8_t)(0x01u << (k & 7u))"),
@@ -31,6 +31,10 @@ MUTATIONS = {
                         "gap[next_chunk] = (uint8_t)(start - next_chunk * OR_CHUNK_BITS + 1);")],
     "block_pos_counts_inclusive": [("pos[next_block] = (uint32_t)i;",
                                     "pos[next_block] = (uint32_t)(i + 1);")],
+    "run_index_counts_boundary_code": [("    while (next_run < runs && next_run * run_bits <= bit) {",
+                                        "    while (next_run < runs && next_run * run_bits < bit) {")],
+    "run_index_not_reset_per_block": [("      if (next_run % runs_per_block == 0) block_first = i;\n",
+                                       "      if (next_run == 0) block_first = i;\n")],
     "sign_in_bit_0": [("sign_mantissa[i] = (uint8_t)((sign << 7) | mant); /* R1 */",
                        "sign_mantissa[i] = (uint8_t)((mant << 1) | sign); /* R1 */"),
                       ("unsigned sign = (sign_mantissa[i] >> 7) & 1u;\n    unsigned mant = sign_mantissa[i] & 0x7Fu;",
@@ -110,6 +114,17 @@ def _check_round_trip(lib):
         assert np.array_equal(oracle.decode(enc, chunked=True, lib=lib), x)
 
 
+def _check_run_index(lib):
+    x = workloads.all_patterns()
+    enc = oracle.encode(x, lib=lib)
+    ri = oracle.run_index(x, enc.lengths, enc.total_bits, lib)
+    assert np.array_equal(ri, np.tile(np.arange(128, dtype=np.uint16) * 16, 32))
+    x = workloads.random_bf16(100_000, seed=3)
+    enc = oracle.encode(x, cap=11, lib=lib)
+    assert np.array_equal(oracle.run_index(x, enc.lengths, enc.total_bits, lib),
+                          _run_index_by_search(x, enc))
+
+
 def _check_rans(lib):
     f = oracle.rans_freqs(rp.hist_of({0: 1, 1: 1, 2: 1}), lib)
     assert f[:3].tolist() == [1366, 1365, 1365]
@@ -127,7 +142,7 @@ def _check_rans(lib):
 
 
 CHECKS = [_check_uniform, _check_tie, _check_costs, _check_golden, _check_layout, _check_round_trip,
-          _check_rans]
+          _check_run_index, _check_rans]
 
 
 def _failures(lib):

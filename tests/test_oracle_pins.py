@@ -406,3 +406,73 @@ def test_workload1_statistics_band(olib):
     assert 10 <= int((enc.hist > 0).sum()) <= 60
     bits_per_weight = 8 + enc.total_bits / enc.n
     assert 10.3 < bits_per_weight < 11.2
+
+
+# ---------------------------------------------------------------- run index (R8)
+# For run r of block b (its chunks 2r and 2r+1), the number of codes that start
+# in the block before the run.  [Kernel] fixes one output position per thread
+# block; this is the same count for each pair of chunks of a block.
+
+
+def _run_index_by_search(x, enc):
+    """The same quantity by a different route: code starts from the cumulative
+    sum of the code lengths, counted per boundary with a binary search."""
+    e, _ = oracle.split(x)
+    lens = enc.lengths[e].astype(np.uint64)
+    starts = np.cumsum(lens) - lens
+    runs = enc.n_blocks * 128
+    bounds = np.arange(runs, dtype=np.uint64) * 128
+    block_bounds = (np.arange(runs, dtype=np.uint64) // 128) * 16384
+    return (np.searchsorted(starts, bounds, side="left")
+            - np.searchsorted(starts, block_bounds, side="left")).astype(np.uint16)
+
+
+def test_run_index_all_patterns_closed_form(olib):
+    """8-bit codes: 16 codes start in every 128-bit run, so run r of any
+    block starts at output 16 r within it."""
+    x = workloads.all_patterns()
+    enc = oracle.encode(x)
+    ri = oracle.run_index(x, enc.lengths, enc.total_bits)
+    assert ri.size == 32 * 128
+    assert np.array_equal(ri, np.tile(np.arange(128, dtype=np.uint16) * 16, 32))
+
+
+@pytest.mark.parametrize("n", [1, 128, 129, 16384, 16385, 40000])
+def test_run_index_single_symbol_closed_form(olib, n):
+    """One value with a 1-bit code: 128 codes per run, and runs past the end
+    of the stream hold their block's total."""
+    x = workloads.constant(n, 0xBC00)
+    enc = oracle.encode(x)
+    ri = oracle.run_index(x, enc.lengths, enc.total_bits).astype(np.int64)
+    b, r = np.divmod(np.arange(ri.size), 128)
+    in_block = np.minimum(n - 16384 * b, 16384)
+    assert np.array_equal(ri, np.minimum(128 * r, in_block))
+
+
+def test_run_index_hand_example(olib):
+    """64 values of a 1-bit code, then 40 of a 2-bit code: bits 0..63 hold 64
+    codes, the 2-bit codes start at 64, 66, ..., 142.  The run boundary at
+    bit 128 has 64 + 32 code starts before it; every later run of the block
+    (past the end of the 144-bit stream) holds the block total, 104."""
+    lengths = np.zeros(256, np.uint8)
+    codes = np.zeros(256, np.uint32)
+    lengths[10], codes[10] = 1, 0b0
+    lengths[20], codes[20] = 2, 0b10
+    x = np.array([10 << 7] * 64 + [20 << 7] * 40, np.uint16)
+    enc = oracle.encode(x, lengths=lengths, codes=codes)
+    assert enc.total_bits == 144
+    ri = oracle.run_index(x, lengths, 144)
+    assert ri.tolist() == [0, 96] + [104] * 126
+
+
+@pytest.mark.parametrize("n", [7, 4097, 100_000, 300_001])
+def test_run_index_matches_binary_search_and_block_positions(olib, n):
+    x = workloads.random_bf16(n, seed=31 + n)
+    enc = oracle.encode(x, cap=11)
+    ri = oracle.run_index(x, enc.lengths, enc.total_bits)
+    assert np.array_equal(ri, _run_index_by_search(x, enc))
+    per_block = ri.reshape(-1, 128).astype(np.int64)
+    totals = np.diff(enc.block_pos.astype(np.int64))
+    assert (per_block[:, 0] == 0).all()
+    assert (np.diff(per_block, axis=1) >= 0).all()
+    assert (per_block[:, -1] <= totals).all()
