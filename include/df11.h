@@ -102,6 +102,8 @@ typedef struct {
   uint64_t stream_alloc, gaps_alloc, block_pos_alloc, sign_mantissa_alloc;
   uint64_t tables_bytes;       /* df11_build_tables output                      */
   uint64_t workspace_bytes;    /* df11_encode scratch                           */
+  uint64_t run_index_bytes;    /* df11_build_run_index output (128 uint16 per
+                                  block; 16-byte multiple)                      */
 } df11_sizes;
 
 /* One compressed matrix in device memory (non-owning).  Every pointer must be
@@ -120,6 +122,10 @@ typedef struct {
                                   assume the most that min_len allows; sizes
                                   the decoder's staging (a block exceeding it
                                   is reported as corrupt)                       */
+  const uint16_t *run_index;   /* optional (NULL: not used): the matrix's run
+                                  index from df11_build_run_index, 16-byte
+                                  aligned.  With it the decoder places every
+                                  thread's outputs before decoding them       */
 } df11_matrix;
 
 /* Encoder outputs in device memory (sizes from df11_encoded_sizes). */
@@ -293,11 +299,34 @@ df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32_t *d_statu
  * decompressed as one batch just before the block's forward pass.
  *   ms      host array of count matrices, each with its own tables.
  *   d_outs  host array of count device pointers (16-byte aligned).
- * One launch per DF11_MAX_BATCH matrices.
+ * One launch per DF11_MAX_BATCH matrices.  When every matrix of a launch has
+ * a run index (df11_matrix.run_index), the launch takes the indexed decoder;
+ * each thread's decoded count is then also checked against the index.
  */
 df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
                                     uint16_t *const *d_outs, uint32_t *d_status,
                                     df11_stream_t stream);
+
+/*
+ * df11_build_run_index -- the run index of one matrix: for every run of two
+ * consecutive chunks (chunks 2r and 2r+1 of block b, the share of one
+ * decoding thread), the number of codes that start in the block before the
+ * run, as uint16 at d_run_index[128 b + r]; runs past the end of the stream
+ * hold their block's total.  [Kernel] stores one output position per thread
+ * block; this is the same count for every pair of chunks.  It is derived from
+ * the stream (not stored in the format): built once when a matrix is placed
+ * on the device, it costs 2 bytes per 128 stream bits of device memory and of
+ * decode traffic, and lets df11_decode place each thread's outputs before it
+ * decodes them (no per-unit prefix sum, no second pass over the exponents).
+ *   m            the matrix (its run_index field is ignored).
+ *   d_run_index  sizes.run_index_bytes device bytes, 16-byte aligned; written.
+ *   d_status     DF11_ERR_CORRUPT if a block's code count disagrees with its
+ *                stored positions or a code is invalid (the index is then
+ *                unusable).
+ * One kernel launch.
+ */
+df11_status df11_build_run_index(const df11_matrix *m, uint16_t *d_run_index, uint32_t *d_status,
+                                 df11_stream_t stream);
 
 /* Activations and sums of one matrix for df11_decode_matmul_batch.  The
  * matrix W holds rows x cols values in row-major order (the order it was

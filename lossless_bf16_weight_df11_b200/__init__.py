@@ -56,7 +56,7 @@ class df11_sizes(ctypes.Structure):
         "stream_bytes", "gaps_bytes", "block_pos_bytes", "sign_mantissa_bytes",
         "stored_bytes",
         "stream_alloc", "gaps_alloc", "block_pos_alloc", "sign_mantissa_alloc",
-        "tables_bytes", "workspace_bytes")]
+        "tables_bytes", "workspace_bytes", "run_index_bytes")]
 
 
 class df11_matrix(ctypes.Structure):
@@ -64,7 +64,7 @@ class df11_matrix(ctypes.Structure):
                 ("stream", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
                 ("block_pos", ctypes.c_void_p), ("sign_mantissa", ctypes.c_void_p),
                 ("tables", ctypes.c_void_p), ("min_len", ctypes.c_uint32),
-                ("max_block_codes", ctypes.c_uint32)]
+                ("max_block_codes", ctypes.c_uint32), ("run_index", ctypes.c_void_p)]
 
 
 class df11_encoded(ctypes.Structure):
@@ -133,6 +133,7 @@ def _declare(lib):
                                                     _vp, _vp]),
         "df11_sizes_from_bits": (ctypes.c_int, [_u64, _u64, ctypes.POINTER(df11_sizes)]),
         "df11_file_bytes": (_u64, [_u64, _u64]),
+        "df11_build_run_index": (ctypes.c_int, [ctypes.POINTER(df11_matrix), _vp, _vp, _vp]),
         "df11_write": (ctypes.c_int, [ctypes.POINTER(df11_host_matrix), _vp, _u64,
                                       ctypes.POINTER(ctypes.c_uint64)]),
         "df11_read": (ctypes.c_int, [_vp, _u64, ctypes.POINTER(df11_host_matrix)]),
@@ -261,6 +262,12 @@ def df11_sizes_from_bits(n: int, total_bits: int):
     out = df11_sizes()
     st = load().df11_sizes_from_bits(n, total_bits, ctypes.byref(out))
     return st, out
+
+
+def df11_build_run_index(m: df11_matrix, d_run_index: int, d_status: int, stream: int = 0) -> int:
+    """The matrix's run index (per pair of chunks, its first output within its
+    block) into device memory; see include/df11.h."""
+    return load().df11_build_run_index(ctypes.byref(m), d_run_index, d_status, stream)
 
 
 def df11_file_bytes(n: int, total_bits: int) -> int:

@@ -22,7 +22,8 @@ from . import (CODEBOOK_BYTES, MAX_CODE_LEN, TABLE_BITS, DF11Error, check, df11_
                df11_build_codebook_device, df11_build_tables, df11_codebook,
                df11_codebook_from_lengths, df11_decode, df11_decode_block_batch,
                df11_decode_matmul_batch, df11_encode, df11_encode_device_codebook, df11_encoded,
-               df11_encoded_sizes, df11_file_bytes, df11_histogram, df11_host_matrix, df11_matmul_io,
+               df11_build_run_index, df11_encoded_sizes, df11_file_bytes, df11_histogram,
+               df11_host_matrix, df11_matmul_io,
                df11_matrix, df11_read, df11_sizes, df11_sizes_from_bits, df11_tables_bytes,
                df11_write)
 
@@ -57,13 +58,16 @@ class DF11Matrix:
     tables: torch.Tensor         # uint8, df11_tables_bytes()
     hist: np.ndarray = field(repr=False, default=None)
     max_block_codes: int = 0     # most codes in one block (0 = unknown)
+    run_index: torch.Tensor | None = None  # int16 (uint16 bits), df11_build_run_index
 
-    def abi(self) -> df11_matrix:
+    def abi(self, use_run_index: bool = True) -> df11_matrix:
+        ri = self.run_index if (use_run_index and self.run_index is not None) else None
         return df11_matrix(n=self.n, total_bits=self.total_bits, stream=self.stream.data_ptr(),
                            gaps=self.gaps.data_ptr(), block_pos=self.block_pos.data_ptr(),
                            sign_mantissa=self.sign_mantissa.data_ptr(),
                            tables=self.tables.data_ptr(), min_len=max(1, self.codebook.min_len),
-                           max_block_codes=self.max_block_codes)
+                           max_block_codes=self.max_block_codes,
+                           run_index=ri.data_ptr() if ri is not None else None)
 
     @property
     def stored_bytes(self) -> int:
@@ -120,15 +124,33 @@ def alloc_encoded(sizes: df11_sizes, device):
 DEFAULT_CAP = TABLE_BITS
 
 
-def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | None = None,
-             stream=None, check_status: bool = True) -> DF11Matrix:
-    """BF16 tensor on a CUDA device -> DF11Matrix (GPU histogram, host
-    codebook, GPU encode).
+def _run_index_for(n: int, total_bits: int, codebook: df11_codebook, sizes: df11_sizes, bufs,
+                   tables: torch.Tensor, status_ptr: int, sh: int, dev) -> torch.Tensor | None:
+    """Enqueue df11_build_run_index for freshly encoded (or uploaded) buffers;
+    returns the index tensor (None for an empty matrix).  Errors land in the
+    device status word at status_ptr."""
+    if n == 0:
+        return None
+    ri = torch.empty(max(16, int(sizes.run_index_bytes)) // 2, dtype=torch.int16, device=dev)
+    m = df11_matrix(n=n, total_bits=total_bits, stream=bufs["stream"].data_ptr(),
+                    gaps=bufs["gaps"].data_ptr(), block_pos=bufs["block_pos"].data_ptr(),
+                    sign_mantissa=bufs["sign_mantissa"].data_ptr(), tables=tables.data_ptr(),
+                    min_len=max(1, codebook.min_len), max_block_codes=0, run_index=None)
+    with torch.cuda.device(dev):
+        check(df11_build_run_index(m, ri.data_ptr(), status_ptr, sh), "df11_build_run_index")
+    return ri
 
-    cap is the code-length limit.  The default (12, the decode table's
+
+def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | None = None,
+             stream=None, check_status: bool = True, run_index: bool = True) -> DF11Matrix:
+    """BF16 tensor on a CUDA device -> DF11Matrix (GPU histogram, host
+    codebook, GPU encode, and by default the run index the decoder uses to
+    place every thread's outputs).
+
+    cap is the code-length limit.  The default (11, the decode table's
     reach) lets every code decode on the fast path; for the weight
     distributions measured here it costs about 0.2% more exponent bits
-    (0.05% of the compressed size) than the 32-bit limit of the format,
+    (0.06% of the compressed size) than the 32-bit limit of the format,
     which remains fully supported (cap=32)."""
     u = _as_u16(w)
     dev = u.device
@@ -151,16 +173,18 @@ def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | 
     with torch.cuda.device(dev):
         check(df11_encode(u.data_ptr(), u.numel(), codebook, sizes.total_bits, out,
                           ws.data_ptr(), ws.numel(), status.data_ptr(), sh), "df11_encode")
+    ri = (_run_index_for(u.numel(), int(sizes.total_bits), codebook, sizes, bufs, tables,
+                         status.data_ptr(), sh, dev) if run_index else None)
     st_host = status.cpu().numpy()
     if check_status and int(st_host[0]):
         raise DF11Error(int(st_host[0]), "df11_encode (device)")
     return DF11Matrix(shape=tuple(w.shape), n=u.numel(), total_bits=int(sizes.total_bits),
                       codebook=codebook, sizes=sizes, tables=tables, hist=hist,
-                      max_block_codes=int(st_host[1]), **bufs)
+                      max_block_codes=int(st_host[1]), run_index=ri, **bufs)
 
 
 def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
-                   check_status: bool = True) -> list[DF11Matrix]:
+                   check_status: bool = True, run_index: bool = True) -> list[DF11Matrix]:
     """Compress several BF16 tensors (e.g. the matrices of a transformer block
     or a whole model) with two host round trips in all: every histogram is
     computed on the device, copied to the host at once, the codebooks and
@@ -205,6 +229,9 @@ def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
             check(df11_encode(u.data_ptr(), u.numel(), cb, sizes.total_bits, out, wsb.data_ptr(),
                               wsb.numel(), status[i].data_ptr(), sh), "df11_encode")
             mats_bufs.append(bufs)
+    ris = [(_run_index_for(u.numel(), int(sizes.total_bits), cb, sizes, bufs, tables[i],
+                           status[i].data_ptr(), sh, dev) if run_index else None)
+           for i, (u, cb, sizes, bufs) in enumerate(zip(us, cbs, sizes_l, mats_bufs))]
     st_host = status.cpu().numpy()  # round trip 2
     mats = []
     for i, (w, u) in enumerate(zip(ws, us)):
@@ -213,7 +240,8 @@ def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
         mats.append(DF11Matrix(shape=tuple(w.shape), n=u.numel(),
                                total_bits=int(sizes_l[i].total_bits), codebook=cbs[i],
                                sizes=sizes_l[i], tables=tables[i], hist=h_all[i],
-                               max_block_codes=int(st_host[i, 1]), **mats_bufs[i]))
+                               max_block_codes=int(st_host[i, 1]), run_index=ris[i],
+                               **mats_bufs[i]))
     return mats
 
 
@@ -224,7 +252,7 @@ _META_BITS = CODEBOOK_BYTES // 8 * 8
 
 
 def compress_block_device(ws, cap: int = DEFAULT_CAP, stream=None,
-                          check_status: bool = True) -> list[DF11Matrix]:
+                          check_status: bool = True, run_index: bool = True) -> list[DF11Matrix]:
     """compress_block with every step on the device: histograms, codebooks
     and decode tables (df11_build_codebook_device), encodes with the device
     codebooks (df11_encode_device_codebook).  The host only sizes the
@@ -278,6 +306,9 @@ def compress_block_device(ws, cap: int = DEFAULT_CAP, stream=None,
                                               status[i].data_ptr(), sh),
                   "df11_encode_device_codebook")
             mats_bufs.append(bufs)
+    ris = [(_run_index_for(u.numel(), int(sizes.total_bits), cb, sizes, bufs, tables[i],
+                           status[i].data_ptr(), sh, dev) if run_index else None)
+           for i, (u, cb, sizes, bufs) in enumerate(zip(us, cbs, sizes_l, mats_bufs))]
     st_host = status.cpu().numpy()                                   # round trip 2
     mats = []
     for i, (w, u) in enumerate(zip(ws, us)):
@@ -286,12 +317,15 @@ def compress_block_device(ws, cap: int = DEFAULT_CAP, stream=None,
         mats.append(DF11Matrix(shape=tuple(w.shape), n=u.numel(),
                                total_bits=int(sizes_l[i].total_bits), codebook=cbs[i],
                                sizes=sizes_l[i], tables=tables[i], hist=h_all[i].copy(),
-                               max_block_codes=int(st_host[i, 1]), **mats_bufs[i]))
+                               max_block_codes=int(st_host[i, 1]), run_index=ris[i],
+                               **mats_bufs[i]))
     return mats
 
 
 def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
+               stream=None, run_index: bool = True) -> torch.Tensor:
+    """Decode one matrix (with its run index when it has one, unless
+    run_index is False)."""
     dev = m.stream.device
     if out is None:
         out = torch.empty(m.shape, dtype=torch.bfloat16, device=dev)
@@ -299,8 +333,8 @@ def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Ten
     if own_status:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
-        check(df11_decode(m.abi(), out.data_ptr(), status.data_ptr(), _stream_handle(stream)),
-              "df11_decode")
+        check(df11_decode(m.abi(run_index), out.data_ptr(), status.data_ptr(),
+                          _stream_handle(stream)), "df11_decode")
     if own_status:
         s = int(status.item())
         if s:
@@ -308,8 +342,10 @@ def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Ten
     return out
 
 
-def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=None):
-    """Decode every matrix of a block in one launch."""
+def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=None,
+                     run_index: bool = True):
+    """Decode every matrix of a block in one launch (the indexed decoder when
+    every matrix has a run index, unless run_index is False)."""
     dev = ms[0].stream.device
     if outs is None:
         outs = [torch.empty(m.shape, dtype=torch.bfloat16, device=dev) for m in ms]
@@ -317,7 +353,7 @@ def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=N
     if own_status:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
-        check(df11_decode_block_batch([m.abi() for m in ms], [o.data_ptr() for o in outs],
+        check(df11_decode_block_batch([m.abi(run_index) for m in ms], [o.data_ptr() for o in outs],
                                       status.data_ptr(), _stream_handle(stream)),
               "df11_decode_block_batch")
     if own_status:
@@ -357,7 +393,7 @@ def matmul_block(ms, xs, ys=None, status: torch.Tensor | None = None, stream=Non
 
 
 def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, stream, gaps,
-                     block_pos, sign_mantissa, device) -> DF11Matrix:
+                     block_pos, sign_mantissa, device, run_index: bool = True) -> DF11Matrix:
     """Upload stored arrays (e.g. produced elsewhere) into padded device
     buffers ready for decoding."""
     hist = np.zeros(256, np.uint64)
@@ -370,13 +406,24 @@ def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, st
         buf[: a.size] = a
         return torch.from_numpy(buf).to(device)
 
+    bufs = dict(stream=padded(stream, sizes.stream_alloc), gaps=padded(gaps, sizes.gaps_alloc),
+                block_pos=padded(np.asarray(block_pos, np.uint32).view(np.int32),
+                                 sizes.block_pos_alloc, np.int32),
+                sign_mantissa=padded(sign_mantissa, sizes.sign_mantissa_alloc))
+    tables = build_tables(codebook, device)
+    ri = None
+    if run_index and n:
+        # the index of data from elsewhere is built here, on the device; a
+        # stream that does not match its positions is reported
+        dev = bufs["stream"].device
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        ri = _run_index_for(n, total_bits, codebook, sizes, bufs, tables, status.data_ptr(),
+                            _stream_handle(None), dev)
+        st = int(status.item())
+        if st:
+            raise DF11Error(st, "df11_build_run_index (device)")
     return DF11Matrix(shape=tuple(shape), n=n, total_bits=total_bits, codebook=codebook,
-                      sizes=sizes, stream=padded(stream, sizes.stream_alloc),
-                      gaps=padded(gaps, sizes.gaps_alloc),
-                      block_pos=padded(np.asarray(block_pos, np.uint32).view(np.int32),
-                                       sizes.block_pos_alloc, np.int32),
-                      sign_mantissa=padded(sign_mantissa, sizes.sign_mantissa_alloc),
-                      tables=build_tables(codebook, device), hist=hist)
+                      sizes=sizes, tables=tables, hist=hist, run_index=ri, **bufs)
 
 
 def serialize(m: DF11Matrix) -> np.ndarray:

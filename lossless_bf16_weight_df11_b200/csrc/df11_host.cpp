@@ -89,6 +89,7 @@ extern "C" df11_status df11_sizes_from_bits(uint64_t n, uint64_t bits, df11_size
   out->sign_mantissa_alloc = round_up(n, 16) + 16;
   out->tables_bytes = sizeof(DecodeTables);
   out->workspace_bytes = 8 * (ceil_div(n, df11i::kEncTile) + 1) + 16;
+  out->run_index_bytes = 2 * (DF11_BLOCK_CHUNKS / 2) * B;
   return DF11_OK;
 }
 

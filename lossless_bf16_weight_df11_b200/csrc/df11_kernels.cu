@@ -614,6 +614,7 @@ struct DecMat {
   const uint8_t *gaps;
   const uint32_t *pos;
   const uint8_t *sm;
+  const uint16_t *run_index;  // indexed decoder only
   const DecodeTables *tables;
   uint16_t *out;
   uint64_t n;
@@ -1448,6 +1449,483 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_kernel(const __grid_
 #undef DF11_APPEND
 #undef DF11_STEP
 
+// ============================================================ decode with a run index
+//
+// The same work unit, group and pipeline as decode_kernel, with the run index
+// (df11_build_run_index) fetched with the unit's stream bytes: thread t of a
+// unit reads the first output of its run within its block, so it knows where
+// its exponents go before it decodes them.  It decodes straight into the
+// group's linear row at that place: the write-through store of each step is an
+// OR (the row is zero where nothing was written, a word that only gains bits
+// can be OR-ed again, and the words at a thread's two ends, shared with its
+// neighbours, come out right in any order).  The steps whose codes may start
+// past the thread's chunks (the last 11 bits of them) keep only the codes that
+// start inside.  No private rows, no prefix sum and no relocation; two linear
+// rows let the previous unit's merge overlap this unit's decode.
+
+constexpr uint32_t kRunIndexStage = 2 * kUnitChunks / kCPT;          // 512 B: 256 uint16
+constexpr uint32_t kStageBytesIdx = kStreamStage + kGapStage + kRunIndexStage + 16;
+static_assert(kStageBytesIdx % 16 == 0, "stage alignment");
+// a thread can write this far past its first output: 128 codes (1-bit codes
+// over 128 bits) and the word holding the last of them
+constexpr uint32_t kIdxRowSlack = 128 + 48;
+
+// One group's shared memory for the indexed decoder (offsets from the group's
+// base): two stages (stream + gaps + run index), the sign/mantissa bytes, two
+// linear rows, mbarriers, positions, per-warp flags.
+struct GroupLayoutIdx {
+  uint32_t stage0, stage1, sm, lin0, lin1, bars, meta, flags, size;
+};
+
+__host__ __device__ inline GroupLayoutIdx group_layout_idx(uint32_t cap) {
+  GroupLayoutIdx G;
+  G.stage0 = 0;
+  G.stage1 = kStageBytesIdx;
+  G.sm = 2 * kStageBytesIdx;
+  G.lin0 = round16(G.sm + cap + 32);
+  G.lin1 = round16(G.lin0 + cap + kIdxRowSlack);
+  G.bars = round16(G.lin1 + cap + kIdxRowSlack);
+  G.meta = G.bars + 32;
+  G.flags = G.meta + 64;
+  G.size = (G.flags + 64 + 127u) & ~127u;
+  return G;
+}
+
+// a * b + c (low word), kept on the multiply pipe
+__device__ __forceinline__ uint32_t madlo(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// Append to the linear row through OR-ed write-through stores (see
+// DF11_APPEND for the register side; here the row is contiguous).  The
+// word's address, (nb2 bits 5..10) * 4 past row0, and the table address are
+// computed with multiply-adds: the integer logic pipe is this loop's busiest.
+#define DF11_APPEND_OR(xs, add)                                             \
+  {                                                                         \
+    const uint32_t lo = cur | __funnelshift_l(0u, (xs), nb);                \
+    const uint32_t hi = __funnelshift_l((xs), 0u, nb);                      \
+    red_or32(row_a, lo);                                                    \
+    const uint32_t nb2 = nb + (add);                                        \
+    row_a = madlo(madhi(nb2 << 21, 1u << 6, 0u), 4u, row0);                 \
+    cur = ((nb ^ nb2) & 32u) ? hi : lo;                                     \
+    nb = nb2;                                                               \
+  }
+
+#define DF11_LUT_ADDR(w) madlo(madhi((w), 1u << df11i::kLutBits, 0u), 8u, lut_a)
+
+#define DF11_STEP_OR(hw, lw)                                                \
+  {                                                                         \
+    const uint32_t w = __funnelshift_l((lw), (hw), p);                      \
+    const uint2 e = lds64(DF11_LUT_ADDR(w));                                \
+    DF11_APPEND_OR(e.x, e.y)                                                \
+    p = madhi(e.y, 1u << (32 - df11i::kCtrlUsedShift), p);                  \
+  }
+
+// A table step that keeps only the entry's codes starting before lim (room =
+// lim - p <= kLutBits bits ahead): the first code always, each further one if
+// its start field is below room (an absent code's field, 15, never is).
+#define DF11_STEP_MASKED(hw, lw)                                            \
+  {                                                                         \
+    const uint32_t w = __funnelshift_l((lw), (hw), p);                      \
+    const uint2 e = lds64(DF11_LUT_ADDR(w));                                \
+    const uint32_t room = lim - p;                                          \
+    const uint32_t nc = (e.y >> df11i::kCtrlCountShift) & 7u;               \
+    uint32_t keep = 1u + (((e.y >> 12) & 15u) < room) +                     \
+                    (((e.y >> 16) & 15u) < room) + (((e.y >> 20) & 15u) < room); \
+    keep = min(keep, nc);                                                   \
+    const uint32_t mask = keep >= 4u ? 0xFFFFFFFFu : ((1u << (8u * keep)) - 1u); \
+    DF11_APPEND_OR(e.x & mask, 8u * keep)                                   \
+    p = madhi(e.y, 1u << (32 - df11i::kCtrlUsedShift), p);                  \
+  }
+
+__global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_idx_kernel(const __grid_constant__ DecParams P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t ngroups = blockDim.x / kT;
+  const uint32_t grp = threadIdx.x / kT;
+  const int t = (int)(threadIdx.x % kT), lane = t & 31, warp = t >> 5;
+  const uint32_t cap = P.stage_cap;
+  const GroupLayoutIdx GL = group_layout_idx(cap);
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t gofs = kTablesSmem + grp * GL.size;
+  const uint32_t gbase = sbase + gofs;
+  const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem);
+  const uint32_t lut_a = sbase;  // lut is the first member of the tables
+  const uint32_t bar_stage = gbase + GL.bars, bar_sm = gbase + GL.bars + 16;
+  uint32_t *meta = reinterpret_cast<uint32_t *>(smem + gofs + GL.meta);
+  uint32_t *wflags = reinterpret_cast<uint32_t *>(smem + gofs + GL.flags);
+  const uint32_t sm_a = gbase + GL.sm;
+  const uint32_t bar_id = 1 + grp;
+
+  const uint64_t total = P.unit_start[P.count];
+  const uint64_t g0 = (uint64_t)blockIdx.x * total / gridDim.x;
+  const uint64_t g1 = (uint64_t)(blockIdx.x + 1) * total / gridDim.x;
+  if (g0 >= g1) return;  // the same for every thread of the CTA
+#ifdef DF11_CHECKED
+  if (threadIdx.x == 0) s_check_status = P.status;
+  __syncthreads();
+#endif
+
+  // both linear rows start zeroed
+  for (uint32_t k = t; k < (GL.bars - GL.lin0) / 16; k += kT) sts128_zero(gbase + GL.lin0 + 16 * k);
+  if (t == 0) {
+    mbar_init(bar_stage, 1);
+    mbar_init(bar_stage + 8, 1);
+    mbar_init(bar_sm, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+
+  uint32_t it = 0;
+  bool timed_out = false;
+  uint32_t m = 0;
+  while (m + 1 < P.count && g0 >= P.unit_start[m + 1]) ++m;
+  for (; m < P.count && P.unit_start[m] < g1; ++m) {
+    if (__syncthreads_or(timed_out)) return;
+    const uint64_t s0 = max(g0, P.unit_start[m]), s1 = min(g1, P.unit_start[m + 1]);
+    if (s0 >= s1) continue;
+    const DecMat &M = P.m[m];
+    {
+      const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
+      uint4 *dst = reinterpret_cast<uint4 *>(smem);
+      for (uint32_t k = threadIdx.x; k < sizeof(DecodeTables) / 16; k += blockDim.x)
+        dst[k] = __ldg(src + k);
+    }
+    __syncthreads();
+    bool tbad = false;
+    for (uint32_t k = threadIdx.x; k < (uint32_t)df11i::kLutSize; k += blockDim.x)
+      tbad |= lut_entry_bad(tab.lut[k].y, P.min_len);
+    const bool table_ok = !__syncthreads_or(tbad);
+    const bool table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
+
+    const uint64_t first = s0 + grp;
+    if (first >= s1) continue;
+    uint32_t nxt_p0 = 0, nxt_p1 = 0, nxt_pm = 0;
+    auto fetch_pos = [&](uint64_t g) {
+      const uint32_t b0 = kUnitBlocks * (uint32_t)(g - P.unit_start[m]);
+      DF11_GLOBAL_CHECK(b0 < M.n_blocks, return)
+      nxt_p0 = __ldg(M.pos + b0);
+      nxt_p1 = __ldg(M.pos + min(b0 + kUnitBlocks, M.n_blocks));
+      nxt_pm = b0 + 1 < M.n_blocks ? __ldg(M.pos + b0 + 1) : nxt_p1;
+    };
+    auto issue_stream = [&](uint64_t g, uint32_t stage) {
+      const uint32_t u = (uint32_t)(g - P.unit_start[m]);
+      const uint32_t nb = min(kUnitBlocks, M.n_blocks - kUnitBlocks * u);
+      const uint32_t sbytes = nb * kBlockStreamBytes + 16, gbytes = nb * kBlockGapBytes;
+      const uint32_t ibytes = nb * (kRunIndexStage / kUnitBlocks);
+      const uint32_t st = gbase + (stage ? GL.stage1 : GL.stage0);
+      uint32_t *mt = meta + stage * 8;
+      mt[0] = nxt_p0;
+      mt[1] = nxt_p1;
+      mt[2] = u;
+      mt[3] = nxt_pm;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      DF11_GLOBAL_CHECK((uint64_t)u * (8 * kUnitChunks) + sbytes <=
+                                (uint64_t)kBlockStreamBytes * M.n_blocks + 16 &&
+                            (uint64_t)u * kGapStage + gbytes <=
+                                (uint64_t)kBlockGapBytes * M.n_blocks + 16,
+                        {
+                          mbar_expect_tx(bar_stage + 8 * stage, 0);
+                          return;
+                        })
+#ifdef DF11_TEST_HOOKS
+      mbar_expect_tx(bar_stage + 8 * stage, sbytes + gbytes + ibytes + P.starve_tx);
+#else
+      mbar_expect_tx(bar_stage + 8 * stage, sbytes + gbytes + ibytes);
+#endif
+      bulk_g2s(st, M.stream + (uint64_t)u * (8 * kUnitChunks), sbytes, bar_stage + 8 * stage);
+      bulk_g2s(st + kStreamStage, M.gaps + (uint64_t)u * kGapStage, gbytes, bar_stage + 8 * stage);
+      bulk_g2s(st + kStreamStage + kGapStage, M.run_index + (uint64_t)u * (kRunIndexStage / 2),
+               ibytes, bar_stage + 8 * stage);
+    };
+    if (t == 0) {
+      fetch_pos(first);
+      issue_stream(first, it & 1);
+      if (first + ngroups < s1) fetch_pos(first + ngroups);
+    }
+    group_sync(bar_id);
+
+    // One group barrier per unit, at its end ([B]).  Everything a unit
+    // reuses was last touched before the previous [B]: the stage and meta
+    // slot the next copy goes to (read while decoding the unit before),
+    // the linear row this unit decodes into (merged and cleared in the
+    // previous iteration, or cleared after its [B] when rejected), and the
+    // flag words (two sets, by the stage's parity).
+    Pending prev{0, 0, nullptr, false, 0, 0, 0, 0};
+    bool have_prev = false;
+    for (uint64_t g = first; g < s1; g += ngroups, ++it) {
+      const uint32_t s = it & 1;
+      const uint32_t *mt = meta + s * 8;
+      const uint32_t P0 = mt[0], P1 = mt[1], u = mt[2], PM = mt[3];
+      const bool sane = P1 >= P0 && P1 <= M.n && P1 - P0 <= cap && PM >= P0 && PM <= P1;
+      if (t == 0 && g + ngroups < s1) {
+        issue_stream(g + ngroups, s ^ 1);
+        if (g + 2 * ngroups < s1) fetch_pos(g + 2 * ngroups);
+      }
+      bool tmo = !mbar_wait(bar_stage + 8 * s, (it >> 1) & 1);
+      const uint32_t lin_s = gbase + (s ? GL.lin1 : GL.lin0);
+
+      // ---- this thread's two chunks, decoded straight into the linear row
+      const uint32_t c0 = u * kUnitChunks + kCPT * t;
+      bool bad = false;
+      if (table_ok && sane && c0 < M.n_chunks) {
+        const uint32_t st = gbase + (s ? GL.stage1 : GL.stage0);
+        // the run's first output within its block and the next run's (or the
+        // block's total after its last run)
+        const uint32_t ia = st + kStreamStage + kGapStage + 2 * t;
+        const uint32_t r = (uint32_t)t & 127u;
+        const uint32_t btot = t < 128 ? PM - P0 : P1 - PM;
+        const uint32_t two_idx = lds32(ia & ~3u);
+        const uint32_t off = (t & 1) ? two_idx >> 16 : two_idx & 0xFFFFu;
+        const uint32_t nxt = r == 127u ? btot : ((t & 1) ? lds32(ia + 2) & 0xFFFFu : two_idx >> 16);
+        bad = off > nxt || nxt > btot || (r == 0u && off != 0u);
+        if (!bad) {
+          const uint32_t D = (P0 & 15u) + (t < 128 ? 0u : PM - P0) + off;
+          const uint4 a4 = lds128(st + 16 * t);
+          const uint32_t W0 = bswap32(a4.x), W1 = bswap32(a4.y), W2 = bswap32(a4.z),
+                         W3 = bswap32(a4.w), W4 = bswap32(lds32(st + 16 * t + 16));
+          const uint64_t avail = M.total_bits - 64ull * c0;
+          const uint32_t lim = avail < 64u * kCPT ? (uint32_t)avail : 64u * kCPT;
+          const uint32_t q = DF11_GAP_BITS * kCPT * t;
+          const uint32_t ga = st + kStreamStage + (q >> 3);
+          const uint32_t two = (lds8(ga) << 8) | lds8(ga + 1);
+          const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
+          const uint32_t row0 = lin_s + (D & ~3u);
+          const uint32_t nb0 = 8u * (D & 3u);
+          uint32_t p = gap, nb = nb0, cur = 0, row_a = row0;
+          if (table_short) {
+            // steps whose codes all start before lim, one loop per word; then
+            // the last few steps, masked
+            const uint32_t safe = lim > (uint32_t)df11i::kLutBits ? lim - df11i::kLutBits : 0u;
+            const uint32_t l1 = min(safe, 32u), l2 = min(safe, 64u), l3 = min(safe, 96u);
+#pragma unroll 1
+            while (p < l1) DF11_STEP_OR(W0, W1)
+#pragma unroll 1
+            while (p < l2) DF11_STEP_OR(W1, W2)
+#pragma unroll 1
+            while (p < l3) DF11_STEP_OR(W2, W3)
+#pragma unroll 1
+            while (p < safe) DF11_STEP_OR(W3, W4)
+#pragma unroll 1
+            while (p < lim) {
+              const uint32_t k = p >> 5;
+              const uint32_t hw = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
+              const uint32_t lw = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
+              DF11_STEP_MASKED(hw, lw)
+            }
+          } else {
+            // codes longer than the table's reach: per word a table loop that
+            // leaves on a flagged entry, whose code the length search decodes
+            // (a code starting before lim is the thread's whatever its
+            // length); the last steps masked as above
+            const uint32_t safe = lim > (uint32_t)df11i::kLutBits ? lim - df11i::kLutBits : 0u;
+#pragma unroll 1
+            while (p < lim) {
+              const uint32_t k = p >> 5;
+              const uint32_t hw = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
+              const uint32_t lw = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
+              if (p < safe) {
+                // steps of word k whose codes all start before lim
+                const uint32_t seg = min(safe, 32u * (k + 1));
+                bool flagged = false;
+#pragma unroll 1
+                while (p < seg) {
+                  const uint32_t w = __funnelshift_l(lw, hw, p);
+                  const uint2 e = lds64(DF11_LUT_ADDR(w));
+                  if (e.y & df11i::kCtrlLongFlag) {
+                    flagged = true;
+                    break;
+                  }
+                  DF11_APPEND_OR(e.x, e.y)
+                  p = madhi(e.y, 1u << (32 - df11i::kCtrlUsedShift), p);
+                }
+                if (!flagged) continue;  // the next word's loop (words re-picked)
+              } else {
+                // p in [safe, lim): a table entry may hold the next thread's codes
+                const uint32_t w = __funnelshift_l(lw, hw, p);
+                const uint32_t ey = lds32(DF11_LUT_ADDR(w) + 4);
+                if (!(ey & df11i::kCtrlLongFlag)) {
+                  DF11_STEP_MASKED(hw, lw)
+                  continue;
+                }
+              }
+              // a flagged entry at p (inside word k): the length search
+              const uint32_t w = __funnelshift_l(lw, hw, p);
+              const uint32_t L = long_code_len(w, tab);
+              if (L == 0) {
+                bad = true;
+                break;
+              }
+              const uint32_t x = tab.sym[((w >> (32 - L)) + tab.base[L]) & 0xFFu];
+              DF11_APPEND_OR(x, 8u)
+              p += L;
+            }
+          }
+          red_or32(row_a, cur);  // the word being filled
+          const uint32_t d = ((nb & 0x7FFu) - nb0) >> 3;
+          bad |= d != nxt - off;
+        }
+      }
+      // ---- the previous unit's merge (its row is the other one)
+      if (have_prev) {
+        if (!mbar_wait(bar_sm, (it - 1) & 1)) tmo = true;
+        else if (prev.ok) merge_unit(prev, gbase + (s ? GL.lin0 : GL.lin1), sm_a, t);
+      }
+      // ---- [B] the group's flags
+      const uint32_t wf = (__ballot_sync(0xffffffffu, bad) ? 1u : 0u) |
+                          (__ballot_sync(0xffffffffu, tmo) ? 2u : 0u);
+      uint32_t *wfl = wflags + 8 * s;
+      if (lane == 0) wfl[warp] = wf;
+      group_sync(bar_id);
+      const uint32_t flagbits = __reduce_or_sync(0xffffffffu, lane < kT / 32 ? wfl[lane] : 0u);
+      if (flagbits & 2u) {
+        if (t == 0) {
+          set_status(P.status, DF11_ERR_TIMEOUT);
+          if (g + ngroups < s1) mbar_wait(bar_stage + 8 * (s ^ 1), ((it + 1) >> 1) & 1);
+        }
+        timed_out = true;
+        break;
+      }
+      // every thread's count matched its run's share of the block positions
+      const bool ok = table_ok && sane && !(flagbits & 1u);
+      if (t == 0) {
+        if (!ok) set_status(P.status, DF11_ERR_CORRUPT);
+        const uint32_t sm_lo = P0 & ~15u;
+        uint32_t sm_bytes = sane ? (uint32_t)((((uint64_t)P1 + 15u) & ~15ull) - sm_lo) : 0u;
+        DF11_GLOBAL_CHECK((uint64_t)sm_lo + sm_bytes <= ((M.n + 15) & ~15ull) + 16, sm_bytes = 0)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(bar_sm, sm_bytes);
+        if (sm_bytes) bulk_g2s(sm_a, M.sm + sm_lo, sm_bytes, bar_sm);
+      }
+      // a rejected unit is not merged: its row is cleared here instead
+      if (!ok)
+        for (uint32_t k = t; k < (cap + kIdxRowSlack) / 16; k += kT) sts128_zero(lin_s + 16 * k);
+      prev = Pending{P0, P1, M.out, ok, m, 0, 0, (uint32_t)M.n};
+      have_prev = true;
+    }
+    if (!timed_out && have_prev) {
+      group_sync(bar_id);
+      const bool got = mbar_wait(bar_sm, (it - 1) & 1);
+      if (!got) {
+        if (lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
+        timed_out = true;
+      }
+      if (got && prev.ok) merge_unit(prev, gbase + (((it - 1) & 1) ? GL.lin1 : GL.lin0), sm_a, t);
+    }
+  }
+}
+
+#undef DF11_APPEND_OR
+#undef DF11_LUT_ADDR
+#undef DF11_STEP_OR
+#undef DF11_STEP_MASKED
+
+// ============================================================ run index
+//
+// One CTA of 128 threads per block of 256 chunks at a time (persistent over a
+// contiguous range of blocks, decode tables loaded once): thread r counts the
+// codes that start in chunks 2r and 2r+1 (the decode steps without appends,
+// the last entry trimmed at the end of the run), the CTA's exclusive prefix
+// sum gives each run's first output within the block, and the block's total
+// is checked against its stored positions.
+constexpr int kRiThreads = DF11_BLOCK_CHUNKS / kCPT;  // 128
+
+__global__ void __launch_bounds__(kRiThreads) run_index_kernel(const __grid_constant__ DecParams P,
+                                                              uint16_t *__restrict__ out) {
+  __shared__ __align__(16) DecodeTables tab;
+  __shared__ uint32_t s_warp[kRiThreads / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const DecMat &M = P.m[0];
+  const uint32_t B = M.n_blocks;
+  const uint32_t b0 = (uint32_t)((uint64_t)blockIdx.x * B / gridDim.x);
+  const uint32_t b1 = (uint32_t)((uint64_t)(blockIdx.x + 1) * B / gridDim.x);
+  if (b0 >= b1) return;
+  {
+    const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
+    uint4 *dst = reinterpret_cast<uint4 *>(&tab);
+    for (uint32_t k = t; k < sizeof(DecodeTables) / 16; k += kRiThreads) dst[k] = __ldg(src + k);
+  }
+  __syncthreads();
+  bool tbad = false;
+  for (uint32_t k = t; k < (uint32_t)df11i::kLutSize; k += kRiThreads)
+    tbad |= lut_entry_bad(tab.lut[k].y, P.min_len);
+  if (__syncthreads_or(tbad)) {
+    if (t == 0) set_status(P.status, DF11_ERR_CORRUPT);
+    return;
+  }
+  const bool table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
+  const uint32_t lut_a = smem_addr(&tab);
+  for (uint32_t b = b0; b < b1; ++b) {
+    const uint32_t c0 = b * DF11_BLOCK_CHUNKS + kCPT * t;
+    uint32_t cnt = 0;
+    bool bad = false;
+    if (c0 < M.n_chunks) {
+      // the run's 16 stream bytes and the next 4 (inside the stream's
+      // allocation: whole blocks plus 16 bytes)
+      const uint4 a4 = __ldg(reinterpret_cast<const uint4 *>(M.stream + 8ull * c0));
+      const uint32_t W0 = bswap32(a4.x), W1 = bswap32(a4.y), W2 = bswap32(a4.z),
+                     W3 = bswap32(a4.w),
+                     W4 = bswap32(__ldg(reinterpret_cast<const uint32_t *>(M.stream + 8ull * c0 + 16)));
+      const uint64_t avail = M.total_bits - 64ull * c0;
+      const uint32_t lim = avail < 64u * kCPT ? (uint32_t)avail : 64u * kCPT;
+      const uint64_t q = (uint64_t)DF11_GAP_BITS * c0;
+      const uint32_t two = ((uint32_t)__ldg(M.gaps + (q >> 3)) << 8) | __ldg(M.gaps + (q >> 3) + 1);
+      const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
+      uint32_t p = gap, acc = 0, ctrl = 0;
+#pragma unroll 1
+      while (p < lim) {
+        const uint32_t k = p >> 5;
+        const uint32_t hw = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
+        const uint32_t lw = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
+        const uint32_t w = __funnelshift_l(lw, hw, p);
+        const uint32_t ey = lds32(lut_a + ((w >> (32 - df11i::kLutBits)) << 3) + 4);
+        if (!table_short && (ey & df11i::kCtrlLongFlag)) {
+          const uint32_t L = long_code_len(w, tab);
+          if (L == 0) {
+            bad = true;
+            break;
+          }
+          acc += 8u;
+          ctrl = kLongCodeCtrl;
+          p += L;
+        } else {
+          acc += ey;  // bits 0..10: 8 x the codes (the rest is never read)
+          ctrl = ey;
+          p = madhi(ey, 1u << (32 - df11i::kCtrlUsedShift), p);
+        }
+      }
+      cnt = (acc & 0x7FFu) >> 3;
+      const uint32_t ncodes = (ctrl >> df11i::kCtrlCountShift) & 7u;
+      if (p > lim && ncodes) {
+        const uint32_t pl = p - (ctrl >> df11i::kCtrlUsedShift);
+        const uint32_t past = (uint32_t)(pl + ((ctrl >> 12) & 15u) >= lim) +
+                              (uint32_t)(pl + ((ctrl >> 16) & 15u) >= lim) +
+                              (uint32_t)(pl + ((ctrl >> 20) & 15u) >= lim);
+        cnt -= past - (df11i::kLutMaxCodes - ncodes);
+      }
+    }
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int dd = 1; dd < 32; dd <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, dd);
+      if (lane >= dd) incl += o;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    const bool any_bad = __syncthreads_or(bad);
+    uint32_t pre = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < kRiThreads / 32; ++i) {
+      pre += i < warp ? s_warp[i] : 0u;
+      tot += s_warp[i];
+    }
+    const uint32_t excl = pre + incl - cnt;
+    out[(uint64_t)b * kRiThreads + t] = (uint16_t)excl;
+    if (t == 0 && (any_bad || tot != __ldg(M.pos + b + 1) - __ldg(M.pos + b) || tot > 0xFFFFu))
+      set_status(P.status, DF11_ERR_CORRUPT);
+    __syncthreads();  // s_warp is reused by the next block
+  }
+}
+
 // ============================================================ launch helpers
 
 // decode_kernel instantiations: regions of codes >= 2 bits and >= 1 bit
@@ -1507,6 +1985,9 @@ df11_status device_info(int *dev, int *sms, int *smem_optin = nullptr) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  d.smem_optin) != cudaSuccess)
           return DF11_ERR_CUDA;
+    if (cudaFuncSetAttribute(decode_idx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess)
+      return DF11_ERR_CUDA;
     d.configured = true;
   }
   *sms = d.sms;
@@ -1684,6 +2165,7 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
 #endif
     uint32_t min_len = DF11_MAX_CODE_LEN;
     uint32_t unit_codes = 0;  // staging size: most codes in one unit of the batch
+    bool indexed = io == nullptr;  // every matrix has a run index (plain decode only)
     for (uint32_t i = 0; i < k; ++i) {
       const df11_matrix &m = ms[first + i];
       if (m.n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
@@ -1691,8 +2173,9 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
       if (!m.stream || !m.gaps || !m.block_pos || !m.sign_mantissa || !m.tables)
         return DF11_ERR_INVALID_ARG;
       if (!aligned16(m.stream) || !aligned16(m.gaps) || !aligned16(m.sign_mantissa) ||
-          !aligned16(m.tables) || ((uintptr_t)m.block_pos & 3u))
+          !aligned16(m.tables) || ((uintptr_t)m.block_pos & 3u) || !aligned16(m.run_index))
         return DF11_ERR_INVALID_ARG;
+      indexed = indexed && m.run_index != nullptr;
       if (io) {
         // the matrix is rows x cols; activations and sums 16-byte aligned
         const df11_matmul_io &q = io[first + i];
@@ -1722,6 +2205,7 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
       d.pos = m.block_pos;
       d.sm = m.sign_mantissa;
       d.tables = reinterpret_cast<const DecodeTables *>(m.tables);
+      d.run_index = m.run_index;
       d.out = io ? nullptr : d_outs[first + i];
       d.rows = io ? io[first + i].rows : 0u;
       d.cols = io ? io[first + i].cols : 1u;
@@ -1741,16 +2225,17 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
     P.min_len = min_len;
     P.batch = io ? batch : 0u;
     const uint32_t region = 4u * (min_len >= 2 ? kMaxWords2 : kMaxWords1);
-    const GroupLayout GL = group_layout(P.stage_cap, region, nb);
+    const uint32_t group_bytes =
+        indexed ? group_layout_idx(P.stage_cap).size : group_layout(P.stage_cap, region, nb).size;
     const uint64_t units = P.unit_start[P.count];
     // groups per CTA: as many as one CTA's shared memory holds next to the
     // tables (one CTA per SM), but no more than there are units per SM
-    if (smem_optin < (int)(kTablesSmem + GL.size)) return DF11_ERR_INVALID_ARG;
-    const uint32_t fit = (uint32_t)((smem_optin - (int)kTablesSmem) / (int)GL.size);
+    if (smem_optin < (int)(kTablesSmem + group_bytes)) return DF11_ERR_INVALID_ARG;
+    const uint32_t fit = (uint32_t)((smem_optin - (int)kTablesSmem) / (int)group_bytes);
     const uint32_t groups = (uint32_t)std::min<uint64_t>(
         std::min<uint32_t>(kMaxGroups, fit), std::max<uint64_t>(1, cdiv(units, (uint64_t)sms)));
-    const uint32_t smem = kTablesSmem + groups * GL.size;
-    const DecodeKernel kern = decode_kernel_for(min_len < 2, nb);
+    const uint32_t smem = kTablesSmem + groups * group_bytes;
+    const DecodeKernel kern = indexed ? decode_idx_kernel : decode_kernel_for(min_len < 2, nb);
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, (int)(groups * kT), smem) !=
         cudaSuccess)
@@ -1784,6 +2269,43 @@ extern "C" df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32
                                    df11_stream_t stream) {
   if (!m) return DF11_ERR_INVALID_ARG;
   return df11_decode_block_batch(m, 1, &d_out, d_status, stream);
+}
+
+extern "C" df11_status df11_build_run_index(const df11_matrix *m, uint16_t *d_run_index,
+                                            uint32_t *d_status, df11_stream_t stream) {
+  if (!m || !d_status) return DF11_ERR_INVALID_ARG;
+  if (m->n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
+  if (m->n == 0) return DF11_OK;
+  if (!d_run_index || !aligned16(d_run_index) || !m->stream || !m->gaps || !m->block_pos ||
+      !m->tables || !aligned16(m->stream) || !aligned16(m->tables) ||
+      ((uintptr_t)m->block_pos & 3u))
+    return DF11_ERR_INVALID_ARG;
+  if (m->min_len < 1 || m->min_len > 8) return DF11_ERR_INVALID_ARG;
+  if (m->total_bits < m->n * (uint64_t)m->min_len || m->total_bits > m->n * 32ull)
+    return DF11_ERR_INVALID_ARG;
+  int dev, sms;
+  df11_status st = device_info(&dev, &sms);
+  if (st != DF11_OK) return st;
+  const uint64_t C = cdiv(m->total_bits, 64);
+  const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
+  if (C >= (1ull << 31)) return DF11_ERR_TOO_LARGE;
+  DecParams P{};
+  DecMat &d = P.m[0];
+  d.stream = m->stream;
+  d.gaps = m->gaps;
+  d.pos = m->block_pos;
+  d.tables = reinterpret_cast<const DecodeTables *>(m->tables);
+  d.n = m->n;
+  d.total_bits = m->total_bits;
+  d.n_chunks = (uint32_t)C;
+  d.n_blocks = (uint32_t)B;
+  P.count = 1;
+  P.min_len = m->min_len;
+  P.status = d_status;
+  const uint64_t grid = std::min<uint64_t>(B, (uint64_t)sms * 8);
+  run_index_kernel<<<(unsigned)grid, kRiThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      P, d_run_index);
+  return launch_status();
 }
 
 #ifdef DF11_TEST_HOOKS

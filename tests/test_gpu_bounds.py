@@ -125,20 +125,35 @@ def test_encode_and_decode_stay_inside_their_buffers(df11, name, gen, cap, stati
     before = {k: g.full.clone() for k, g in bufs.items()}
     before["tables"] = tables.full.clone()
     n = x.size
-    out = Guarded(max(2 * n, 16), dev, fill=0x00)
+    sh = torch.cuda.current_stream().cuda_stream
     m = df11.df11_matrix(n=n, total_bits=sizes.total_bits, stream=bufs["stream"].ptr,
                          gaps=bufs["gaps"].ptr, block_pos=bufs["block_pos"].ptr,
                          sign_mantissa=bufs["sign_mantissa"].ptr, tables=tables.ptr,
                          min_len=max(1, cb.min_len), max_block_codes=block_max)
-    status = Guarded(16, dev, fill=0)
-    df11.check(df11.df11_decode_block_batch([m], [out.ptr], status.ptr,
-                                            torch.cuda.current_stream().cuda_stream),
-               "df11_decode_block_batch")
+    # the run index, built into its own guarded buffer
+    ri = Guarded(max(16, sizes.run_index_bytes), dev)
+    ri_status = Guarded(16, dev, fill=0)
+    df11.check(df11.df11_build_run_index(m, ri.ptr, ri_status.ptr, sh), "df11_build_run_index")
     torch.cuda.synchronize()
-    assert int(status.inner.cpu().numpy().view(np.uint32)[0]) == 0, "decode status"
-    assert out.margins_intact(), "decode wrote outside its output"
-    assert status.margins_intact(), "decode wrote outside its status word"
+    assert int(ri_status.inner.cpu().numpy().view(np.uint32)[0]) == 0, "run index status"
+    assert ri.margins_intact() and ri_status.margins_intact(), "run index wrote outside its buffers"
     for k, g in list(bufs.items()) + [("tables", tables)]:
-        assert torch.equal(g.full, before[k]), f"decode modified its input {k}"
-    got = out.inner[: 2 * n].cpu().numpy().view(np.uint16)
-    assert np.array_equal(got, x)
+        assert torch.equal(g.full, before[k]), f"the run index modified its input {k}"
+    if n:
+        want = oracle.run_index(x, enc.lengths, enc.total_bits)
+        assert np.array_equal(ri.inner[: 2 * want.size].cpu().numpy().view(np.uint16), want)
+    before["run_index"] = ri.full.clone()
+    for use_index in (False, True):
+        m.run_index = ri.ptr if use_index else None
+        out = Guarded(max(2 * n, 16), dev, fill=0x00)
+        status = Guarded(16, dev, fill=0)
+        df11.check(df11.df11_decode_block_batch([m], [out.ptr], status.ptr, sh),
+                   "df11_decode_block_batch")
+        torch.cuda.synchronize()
+        assert int(status.inner.cpu().numpy().view(np.uint32)[0]) == 0, "decode status"
+        assert out.margins_intact(), "decode wrote outside its output"
+        assert status.margins_intact(), "decode wrote outside its status word"
+        for k, g in list(bufs.items()) + [("tables", tables), ("run_index", ri)]:
+            assert torch.equal(g.full, before[k]), f"decode modified its input {k}"
+        got = out.inner[: 2 * n].cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, x)

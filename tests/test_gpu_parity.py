@@ -50,6 +50,15 @@ def assert_encoded_equal(m, enc):
 CAPS = [11, 12, 32]
 
 
+def assert_run_index_equal(m, x, enc):
+    if enc.n == 0:
+        assert m.run_index is None
+        return
+    want = oracle.run_index(x, enc.lengths, enc.total_bits)
+    got = m.run_index[: want.size].cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, want), "run index differs"
+
+
 def full_check(codec, x: np.ndarray, cap: int, call_oracle_decode: bool = True):
     x = np.ascontiguousarray(x, np.uint16).reshape(-1)
     enc = oracle.encode(x, cap=cap)
@@ -58,13 +67,17 @@ def full_check(codec, x: np.ndarray, cap: int, call_oracle_decode: bool = True):
     assert np.array_equal(hist, enc.hist), "histogram differs"
     m = codec.compress(w, cap=cap)
     assert_encoded_equal(m, enc)
+    assert_run_index_equal(m, x, enc)
     expected = oracle.decode(enc, chunked=True) if call_oracle_decode else x
     out = codec.decompress(m)
+    assert np.array_equal(bits_of(out), expected), "decode (run index) of GPU-encoded data differs"
+    out = codec.decompress(m, run_index=False)
     assert np.array_equal(bits_of(out), expected), "decode of GPU-encoded data differs"
     # decode of the oracle's own buffers (independent of the GPU encoder)
     cb = codec.codebook_from_lengths(enc.lengths, enc.codes)
     mo = codec.from_host_arrays(x.shape, enc.n, enc.total_bits, cb, enc.stream, enc.gaps_packed,
                                 enc.block_pos, enc.sign_mantissa, w.device)
+    assert_run_index_equal(mo, x, enc)
     out2 = codec.decompress(mo)
     assert np.array_equal(bits_of(out2), expected), "decode of oracle-encoded data differs"
     return m, enc
@@ -146,16 +159,20 @@ def test_workload_block_batched(codec, wid, cap):
         enc = oracle.encode(x, cap=cap)
         m = codec.compress(to_dev(x), cap=cap)
         assert_encoded_equal(m, enc)
+        assert_run_index_equal(m, x, enc)
         mats.append(m)
         xs.append(x)
         del enc
-    outs = codec.decompress_block(mats)
-    for x, o in zip(xs, outs):
-        assert np.array_equal(bits_of(o), x)
+    for use_index in (True, False):
+        outs = codec.decompress_block(mats, run_index=use_index)
+        for x, o in zip(xs, outs):
+            assert np.array_equal(bits_of(o), x)
+        del outs
 
 
+@pytest.mark.parametrize("use_index", [True, False])
 @pytest.mark.parametrize("cap", CAPS)
-def test_decode_reports_corrupt_positions_without_fault(codec, cap):
+def test_decode_reports_corrupt_positions_without_fault(codec, cap, use_index):
     x = workloads.random_bf16(2_000_000, seed=9)
     m = codec.compress(to_dev(x), cap=cap)
     pos = m.block_pos.clone()
@@ -163,20 +180,39 @@ def test_decode_reports_corrupt_positions_without_fault(codec, cap):
     for b in (3, 4):  # a position inside a decode unit and one between two units
         m.block_pos[b] += 5
         status.zero_()
-        codec.decompress(m, status=status)
+        codec.decompress(m, status=status, run_index=use_index)
         assert int(status.item()) == 4  # DF11_ERR_CORRUPT
         m.block_pos.copy_(pos)
     m.block_pos[5] = int(m.n) + 100  # beyond the matrix: must not be dereferenced
     status.zero_()
-    codec.decompress(m, status=status)
+    codec.decompress(m, status=status, run_index=use_index)
     assert int(status.item()) == 4
     m.block_pos.copy_(pos)
     m.stream[1000:1010] ^= 0x5A  # flipped stream bits change the counts
     status.zero_()
-    out = codec.decompress(m, status=status)
+    out = codec.decompress(m, status=status, run_index=use_index)
     torch.cuda.synchronize()
     assert int(status.item()) in (0, 4)
     m.stream[1000:1010] ^= 0x5A
+    status.zero_()
+    out = codec.decompress(m, status=status, run_index=use_index)
+    assert int(status.item()) == 0 and np.array_equal(bits_of(out), x)
+
+
+def test_decode_reports_corrupt_run_index_without_fault(codec):
+    """Run-index entries that disagree with the stream, or point past their
+    block, are reported as corrupt; the decode of the intact index after
+    them is exact (rejected units leave nothing behind)."""
+    x = workloads.random_bf16(2_000_000, seed=10)
+    m = codec.compress(to_dev(x))
+    ri = m.run_index.clone()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for k, v in ((5, 1), (128, 3), (300, -7), (129, 30000), (255, 32767)):
+        m.run_index[k] += v
+        status.zero_()
+        codec.decompress(m, status=status)
+        assert int(status.item()) == 4, (k, v)
+        m.run_index.copy_(ri)
     status.zero_()
     out = codec.decompress(m, status=status)
     assert int(status.item()) == 0 and np.array_equal(bits_of(out), x)
