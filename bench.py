@@ -37,10 +37,11 @@ import workloads  # noqa: E402
 
 METRIC = "DF11 decode output BF16 GB/s & % of HBM roofline (bit-exact); ratio"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_idx_kernel_traffic.txt")
 KERNEL_SOURCE = os.path.join(ROOT, "lossless_bf16_weight_df11_b200", "csrc", "df11_kernels.cu")
 ORACLE_SAMPLE = ("q", "o", "k", "v", "gate")
-CAP = 12  # code-length cap of the benchmarked codebooks (the decode table's reach)
+CAP = 11  # code-length cap of the benchmarked codebooks: DF11_TABLE_BITS, the decode table's reach
+L2_FLUSH_BYTES = 256 << 20  # written between timed launches of inputs that fit the 126 MB L2
 
 
 def parse():
@@ -62,6 +63,8 @@ def parse():
                     help="decode launches of the block coded with the rANS variant (0: skip)")
     ap.add_argument("--block-steps", type=int, default=5,
                     help="steps of the DF11 transformer-block forward timing (0: skip)")
+    ap.add_argument("--config-steps", type=int, default=10,
+                    help="decode launches timed on each of the other workloads (0: skip)")
     return ap.parse_args()
 
 
@@ -193,6 +196,124 @@ def oracle_decode_rate(mats_np, names):
     return 2 * n / dt / 1e9, dt, n
 
 
+def cpu_info():
+    """Host cores this process may use and the CPU model."""
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except Exception:
+        usable = os.cpu_count() or 1
+    model = None
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    return {"nproc": usable, "cpu_model": model}
+
+
+CPU_SAMPLE = 1 << 23  # weights per matrix sample of the oracle's per-config timings
+
+
+def cpu_baseline_plan(samples):
+    """The oracle (plain C, bit-serial, one thread per call) on bounded samples
+    of every workload: encode (histogram, codebook, bitstream) and decode on
+    one core, and, for the two transformer blocks, one matrix per thread on
+    min(7, nproc) cores.  samples: {workload id: [uint16 arrays]}, at most
+    CPU_SAMPLE weights each.  Rates in GB/s of BF16 (input for encode,
+    output for decode)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    info = cpu_info()
+    out = {"cores_available": info["nproc"], "cpu_model": info["cpu_model"], "configs": {}}
+    for wid, mats in samples.items():
+        x = mats[0]
+        t0 = time.perf_counter()
+        enc = oracle.encode(x, cap=CAP)
+        t1 = time.perf_counter()
+        y = oracle.decode(enc)
+        t2 = time.perf_counter()
+        assert np.array_equal(y, x)
+        row = {"sample": f"{x.size} weights of {workloads.workload_name(wid)}",
+               "encode_GBps_1core": 2 * x.size / (t1 - t0) / 1e9,
+               "decode_GBps_1core": 2 * x.size / (t2 - t1) / 1e9}
+        if len(mats) > 1:
+            threads = max(1, min(7, info["nproc"], len(mats)))
+
+            def one(m):
+                e = oracle.encode(m, cap=CAP)
+                return oracle.decode(e).size
+
+            t0 = time.perf_counter()
+            with ThreadPoolExecutor(threads) as ex:
+                done = sum(ex.map(one, mats[:threads]))
+            dt = time.perf_counter() - t0
+            row["multicore"] = {"threads": threads, "weights": done,
+                                "encode_plus_decode_s": dt,
+                                "decode_side_GBps": 2 * done / dt / 1e9,
+                                "what": "one matrix sample per thread, each encoded then decoded"}
+        out["configs"][workloads.workload_name(wid)] = row
+    return out
+
+
+def time_configs(torch, df11, codec, dev, steps, warmup, peak, peak_kind, skip_wid, skip_xs):
+    """Decode of every other workload in one launch per step: median launch
+    time over `steps` launches, each preceded by a write of L2_FLUSH_BYTES (so
+    inputs that fit the 126 MB L2 are read from HBM), with its roofline and
+    compression ratio.  Returns ({workload: line}, {workload id: CPU samples})."""
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lines, samples = {}, {}
+    for wid in (1, 2, 3, 4, 5):
+        if wid == skip_wid:  # the main workload: timed already, its matrices at hand
+            samples[wid] = [x.reshape(-1)[:CPU_SAMPLE] for x in skip_xs]
+            continue
+        mats_def = workloads.WORKLOADS[wid][1]
+        xs = [workloads.matrix(wid, i).reshape(-1) for i in range(len(mats_def))]
+        samples[wid] = [x[:CPU_SAMPLE] for x in xs]
+        n = sum(x.size for x in xs)
+        ws = [torch.from_numpy(x.view(np.int16)).to(dev) for x in xs]
+        cms = codec.compress_block(ws, cap=CAP)
+        outs = [torch.empty(x.size, dtype=torch.bfloat16, device=dev) for x in xs]
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        abis, ptrs = [m.abi() for m in cms], [o.data_ptr() for o in outs]
+        stream = torch.cuda.current_stream(dev)
+        sh = int(stream.cuda_stream)
+
+        def step():
+            df11.check(df11.df11_decode_block_batch(abis, ptrs, status.data_ptr(), sh),
+                       "df11_decode_block_batch")
+
+        for _ in range(max(3, warmup)):
+            step()
+        torch.cuda.synchronize()
+        exact = int(status.item()) == 0 and all(
+            torch.equal(o.view(torch.int16), w) for o, w in zip(outs, ws))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for i, (a, b) in enumerate(evs):
+            flush.fill_(i & 0xFF)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        algo = sum(m.read_bytes + m.index_bytes for m in cms) + 2 * n
+        lines[workloads.workload_name(wid)] = {
+            "weights": n, "matrices": len(xs), "ms_per_launch": ms,
+            "value": 2 * n / (ms / 1e3) / 1e9, "unit": "GB/s", "weights_per_s": n / (ms / 1e3),
+            "ratio": sum(m.stored_bytes for m in cms) / (2 * n), "bit_exact": exact,
+            "max_code_len": max(int(m.codebook.max_len) for m in cms),
+            "l2": f"{L2_FLUSH_BYTES >> 20} MiB written before each timed launch",
+            "roofline": {"bound": "hbm", "achieved": algo / (ms / 1e3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": algo / (ms / 1e3) / 1e9 / peak,
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": algo}}
+        del cms, outs, ws
+        torch.cuda.empty_cache()
+    del flush
+    return lines, samples
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -289,9 +410,11 @@ def run_df11(args):
                       and torch.equal(a.tables, b.tables) for a, b in zip(cms, cms_d))
     del cms_d
     read_bytes = sum(m.read_bytes for m in cms)
+    index_bytes = sum(m.index_bytes for m in cms)
     stored = sum(m.stored_bytes for m in cms)
     ratio = stored / (2 * n_total)
-    algo_bytes = read_bytes + 2 * n_total  # compressed bytes read + BF16 written
+    # compressed bytes read (the format's arrays and the run index) + BF16 written
+    algo_bytes = read_bytes + index_bytes + 2 * n_total
 
     outs = [torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in xs]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -341,6 +464,54 @@ def run_df11(args):
     if int(status.item()) != 0:
         raise df11.DF11Error(int(status.item()), "decode (device)")
 
+    # ---- the same block without its run index (the decoder that places the
+    # exponents after a prefix sum of the per-thread counts), and the time to
+    # build the index (once, when a matrix is placed on the device)
+    no_index = None
+    if args.cap32:
+        abis_ni = [m.abi(False) for m in cms]
+
+        def step_ni():
+            st = df11.df11_decode_block_batch(abis_ni, out_ptrs, status.data_ptr(), sh)
+            if st:
+                raise df11.DF11Error(st, "df11_decode_block_batch")
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                step_ni()
+        torch.cuda.synchronize()
+        ok_ni = all(torch.equal(o.reshape(-1).view(torch.int16), w) for o, w in zip(outs, ws))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step_ni()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms_ni = e0.elapsed_time(e1) / args.steps
+        ri_status = torch.zeros(1, dtype=torch.int32, device=dev)
+        tmp_ri = [torch.empty_like(m.run_index) for m in cms]
+
+        def build_index():
+            for m, r in zip(cms, tmp_ri):
+                df11.check(df11.df11_build_run_index(m.abi(False), r.data_ptr(), ri_status.data_ptr(),
+                                                     sh), "df11_build_run_index")
+
+        with torch.cuda.stream(stream):
+            build_index()
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            build_index()
+            b1.record(stream)
+        torch.cuda.synchronize()
+        same_index = all(torch.equal(a, m.run_index) for a, m in zip(tmp_ri, cms))
+        del tmp_ri
+        no_index = {"ms_per_step": ms_ni, "value": 2 * n_total / (ms_ni / 1e3) / 1e9, "unit": "GB/s",
+                    "roofline_frac": (read_bytes + 2 * n_total) / (ms_ni / 1e3) / 1e9 / measured_peak()[0],
+                    "bit_exact": ok_ni, "kernel": "decode_kernel",
+                    "run_index_build_ms": b0.elapsed_time(b1), "run_index_bytes": index_bytes,
+                    "run_index_rebuilt_identical": same_index and int(ri_status.item()) == 0}
+
     # ---- the rANS variant of the exponent coding on the same block: its
     # ratio and decode time beside the Huffman format's, launches alternated
     rans_line = None
@@ -360,7 +531,7 @@ def run_df11(args):
     if args.cap32:
         cms32 = [codec.compress(w, cap=32) for w in ws]
         abis32 = [m.abi() for m in cms32]
-        algo32 = sum(m.read_bytes for m in cms32) + 2 * n_total
+        algo32 = sum(m.read_bytes + m.index_bytes for m in cms32) + 2 * n_total
 
         def step32():
             st = df11.df11_decode_block_batch(abis32, out_ptrs, status.data_ptr(), sh)
@@ -406,12 +577,22 @@ def run_df11(args):
         fused = [time_fused_matmul(torch, df11, cms, abis, outs, out_ptrs, status, xs_shapes(mats_def),
                                    dev, b, args.matmul_steps, peak, peak_kind) for b in (1, 8)]
 
+    configs, cpu_plan = None, None
+    if args.config_steps > 0:
+        peak_c, peak_kind_c = measured_peak()
+        configs, samples = time_configs(torch, df11, codec, dev, args.config_steps, args.warmup,
+                                        peak_c, peak_kind_c, wid, xs)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cpu_plan = cpu_baseline_plan(samples)
+        del samples
+
     avg_launch_ms = statistics.mean(per_launch_ms)
     achieved = algo_bytes / (avg_launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": profiled_traffic(name),
-                "peak_kind": peak_kind, "kernel": "decode_kernel",
+                "peak_kind": peak_kind, "kernel": "decode_idx_kernel",
                 "algorithmic_bytes_per_launch": algo_bytes,
+                "run_index_bytes_per_launch": index_bytes,
                 "frac_of_8TBps": achieved / 8000.0,
                 "median_launch_ms": statistics.median(per_launch_ms)}
 
@@ -419,7 +600,7 @@ def run_df11(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sample = [xs[i] for i, (nm, _) in enumerate(mats_def) if nm in ORACLE_SAMPLE] or xs[:1]
         gbs, dt, ns = oracle_decode_rate(sample, ORACLE_SAMPLE)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", **cpu_info(),
                "sample": f"{'+'.join(nm for nm, _ in mats_def if nm in ORACLE_SAMPLE) or 'first matrix'}"
                          f" of {name}: {ns} weights decoded bit-serially in {dt:.1f} s"}
 
@@ -455,6 +636,7 @@ def run_df11(args):
             "code_len_cap": CAP,
             "max_code_len": max(int(m.codebook.max_len) for m in cms),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "cap32": cap32,
+            "configs": configs, "cpu_baseline_plan": cpu_plan, "no_run_index": no_index,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -83,6 +83,11 @@ class DF11Matrix:
         """Compressed bytes one decode reads (everything but the lengths)."""
         return int(self.sizes.stored_bytes) - 256
 
+    @property
+    def index_bytes(self) -> int:
+        """Bytes of the run index (0 without one): read by the indexed decoder."""
+        return int(self.sizes.run_index_bytes) if self.run_index is not None else 0
+
     def host_arrays(self):
         """Stored arrays copied to the host (for checks and serialisation)."""
         s = self.sizes
