@@ -77,6 +77,7 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "oracle_encode": (c_int, [_u8p, c_u64, _u8p, _u32p, c_u64, _u8p, _u8p, _u32p]),
         "oracle_pack_gaps": (None, [_u8p, c_u64, _u8p]),
         "oracle_run_index": (c_int, [_u8p, c_u64, _u8p, c_u64, ctypes.POINTER(ctypes.c_uint16)]),
+        "oracle_segment_index": (c_int, [_u8p, c_u64, _u8p, c_u64, _u32p]),
         "oracle_unpack_gaps": (None, [_u8p, c_u64, _u8p]),
         "oracle_decode_serial": (c_int, [_u8p, c_u64, c_u64, _u8p, _u32p, _u8p]),
         "oracle_decode_chunked": (c_int, [_u8p, _u8p, _u32p, c_u64, c_u64, _u8p, _u32p, _u8p]),
@@ -259,7 +260,7 @@ def encode(w: np.ndarray, cap: int = MAX_CAP, lengths=None, codes=None, lib=None
 
 
 def run_index(w: np.ndarray, lengths, total_bits: int, lib=None) -> np.ndarray:
-    """R8: for each 128-bit run of each 256-chunk block, the number of codes
+    """R12: for each 128-bit run of each 256-chunk block, the number of codes
     that start in the block before the run (uint16, 128 per block)."""
     lib = lib or load()
     e, _ = split(w, lib)
@@ -270,6 +271,23 @@ def run_index(w: np.ndarray, lengths, total_bits: int, lib=None) -> np.ndarray:
                              total_bits, _p(out, ctypes.POINTER(ctypes.c_uint16)))
     if r != OK:
         raise ValueError(f"oracle_run_index failed with {r}")
+    return out
+
+
+SEGMENT = 64  # outputs per segment of the segment index
+
+
+def segment_index(w: np.ndarray, lengths, total_bits: int, lib=None) -> np.ndarray:
+    """R13: the stream bit at which the code of value 64j starts, for
+    j < ceil(n/64), then total_bits (uint32, ceil(n/64) + 1 entries)."""
+    lib = lib or load()
+    e, _ = split(w, lib)
+    out = np.zeros((e.size + SEGMENT - 1) // SEGMENT + 1, np.uint32)
+    r = lib.oracle_segment_index(_p(e, _u8p), e.size,
+                                 _p(np.ascontiguousarray(lengths, np.uint8), _u8p), total_bits,
+                                 _p(out, _u32p))
+    if r != OK:
+        raise ValueError(f"oracle_segment_index failed with {r}")
     return out
 
 

@@ -34,13 +34,16 @@
  *   R5 bit order: code bits are written most significant first; stream bit k
  *      is bit (7 - k%8) of byte k/8; the stream is zero-padded to whole
  *      64-bit chunks.
- *   R6 gaps: gap[c] = (first code start >= 64c, or total_bits if none) - 64c,
- *      packed 5 bits per chunk, most significant bit first.
+ *   R6 gaps: gap[c] = (first code start >= 64c, or total_bits if none) - 64c.
+ *   R8 gap packing: 5 bits per chunk, most significant bit first.
  *   R7 block positions: 256 chunks per block; pos[b] = number of codes that
  *      start before bit 64*256*b; pos[B] = n; stored as uint32.
- *   R8 run index (device-side metadata derived from the stream): for run r
+ *   R12 run index (device-side metadata derived from the stream): for run r
  *      of block b (chunks 2r and 2r+1 of the block), the number of codes that
  *      start in the block before the run, as uint16.
+ *   R13 segment index (device-side metadata derived from the stream): for
+ *      every 64th value, the stream bit at which its code starts, then
+ *      total_bits; uint32.
  *
  * Parity status: every function here is pinned by a test in
  * tests/test_oracle_pins.py (closed forms, brute force, textbook identities,
@@ -418,7 +421,7 @@ int oracle_encode(const uint8_t *exponent, uint64_t n, const uint8_t len[256],
 /* Run index: for each 128-bit run (two consecutive chunks, the part of */
 /* a block one decoding thread takes), the output position of its first */
 /* code within its block.  [Kernel] gives one output position per       */
-/* thread block; this is the same count one level finer.  R8 (reading): */
+/* thread block; this is the same count one level finer.  R12 (reading):*/
 /* run_pos[128*b + r] = number of codes that start at bits              */
 /* [16384*b, 16384*b + 128*r); every block has 128 entries (runs past   */
 /* the end of the stream hold the block's total).  Written from the     */
@@ -456,7 +459,33 @@ int oracle_run_index(const uint8_t *exponent, uint64_t n, const uint8_t len[256]
   return OR_OK;
 }
 
-/* Gaps packed as 5-bit fields, most significant bit first (R6).
+/* ------------------------------------------------------------------ */
+/* Segment index: the stream bit at which every 64th code starts.       */
+/* [Kernel] ties threads to chunks of the stream and finds output       */
+/* positions by counting; this is the converse map, from an output      */
+/* position to a stream position, at a fixed output step.  R13          */
+/* (reading): seg[j] = sum of the code lengths of values 0..64j-1 for   */
+/* j = 0..S-1, S = ceil(n/64), and seg[S] = total_bits; uint32, so the  */
+/* stream must hold fewer than 2^32 bits.  Written from the code        */
+/* lengths, one value at a time.  seg must hold S+1 entries.            */
+/* ------------------------------------------------------------------ */
+int oracle_segment_index(const uint8_t *exponent, uint64_t n, const uint8_t len[256],
+                         uint64_t total_bits, uint32_t *seg) {
+  uint64_t segments = (n + 63) / 64;
+  uint64_t bit = 0;
+  if (total_bits > 0xFFFFFFFFull) return OR_ERR_ARG;
+  for (uint64_t i = 0; i < n; i++) {
+    unsigned l = len[exponent[i]];
+    if (l == 0) return OR_ERR_SYMBOL;
+    if (i % 64 == 0) seg[i / 64] = (uint32_t)bit; /* code i starts here */
+    bit += l;
+  }
+  if (bit != total_bits) return OR_ERR_ARG;
+  seg[segments] = (uint32_t)total_bits;
+  return OR_OK;
+}
+
+/* Gaps packed as 5-bit fields, most significant bit first (R8).
  * packed must hold ceil(5*C/8) zeroed bytes. */
 void oracle_pack_gaps(const uint8_t *gap, uint64_t chunks, uint8_t *packed) {
   uint64_t k = 0;

@@ -35,6 +35,11 @@ MUTATIONS = {
                                         "    while (next_run < runs && next_run * run_bits < bit) {")],
     "run_index_not_reset_per_block": [("      if (next_run % runs_per_block == 0) block_first = i;\n",
                                        "      if (next_run == 0) block_first = i;\n")],
+    "segment_index_after_the_code": [("    if (i % 64 == 0) seg[i / 64] = (uint32_t)bit; /* code i starts here */\n    bit += l;",
+                                      "    bit += l;\n    if (i % 64 == 0) seg[i / 64] = (uint32_t)bit; /* code i starts here */")],
+    "segment_index_one_value_early": [("    if (i % 64 == 0) seg[i / 64] = (uint32_t)bit;",
+                                       "    if (i % 64 == 63) seg[i / 64] = (uint32_t)bit;")],
+    "segment_index_ends_with_n": [("  seg[segments] = (uint32_t)total_bits;", "  seg[segments] = (uint32_t)n;")],
     "sign_in_bit_0": [("sign_mantissa[i] = (uint8_t)((sign << 7) | mant); /* R1 */",
                        "sign_mantissa[i] = (uint8_t)((mant << 1) | sign); /* R1 */"),
                       ("unsigned sign = (sign_mantissa[i] >> 7) & 1u;\n    unsigned mant = sign_mantissa[i] & 0x7Fu;",
@@ -125,6 +130,19 @@ def _check_run_index(lib):
                           _run_index_by_search(x, enc))
 
 
+def _check_segment_index(lib):
+    x = workloads.all_patterns()
+    enc = oracle.encode(x, lib=lib)
+    assert np.array_equal(oracle.segment_index(x, enc.lengths, enc.total_bits, lib),
+                          512 * np.arange(1025, dtype=np.uint32))
+    x = workloads.random_bf16(100_003, seed=5)
+    enc = oracle.encode(x, cap=11, lib=lib)
+    seg = oracle.segment_index(x, enc.lengths, enc.total_bits, lib).astype(np.int64)
+    assert seg[-1] == enc.total_bits
+    for b in range(enc.block_pos.size):
+        assert int((seg[:-1] < 16384 * b).sum()) == (int(enc.block_pos[b]) + 63) // 64
+
+
 def _check_rans(lib):
     f = oracle.rans_freqs(rp.hist_of({0: 1, 1: 1, 2: 1}), lib)
     assert f[:3].tolist() == [1366, 1365, 1365]
@@ -142,7 +160,7 @@ def _check_rans(lib):
 
 
 CHECKS = [_check_uniform, _check_tie, _check_costs, _check_golden, _check_layout, _check_round_trip,
-          _check_run_index, _check_rans]
+          _check_run_index, _check_segment_index, _check_rans]
 
 
 def _failures(lib):

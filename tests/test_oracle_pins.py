@@ -408,7 +408,7 @@ def test_workload1_statistics_band(olib):
     assert 10.3 < bits_per_weight < 11.2
 
 
-# ---------------------------------------------------------------- run index (R8)
+# --------------------------------------------------------------- run index (R12)
 # For run r of block b (its chunks 2r and 2r+1), the number of codes that start
 # in the block before the run.  [Kernel] fixes one output position per thread
 # block; this is the same count for each pair of chunks of a block.
@@ -476,3 +476,75 @@ def test_run_index_matches_binary_search_and_block_positions(olib, n):
     assert (per_block[:, 0] == 0).all()
     assert (np.diff(per_block, axis=1) >= 0).all()
     assert (per_block[:, -1] <= totals).all()
+
+
+# ----------------------------------------------------------- segment index (R13)
+# For every 64th value, the stream bit at which its code starts; then
+# total_bits.  The converse of the block positions: output -> stream bit.
+
+
+def _code_at(stream, bit, length):
+    """The length bits of the stream starting at bit, MSB first (R5), read
+    bit by bit from the bytes."""
+    v = 0
+    for k in range(bit, bit + length):
+        v = (v << 1) | ((int(stream[k >> 3]) >> (7 - (k & 7))) & 1)
+    return v
+
+
+def test_segment_index_all_patterns_closed_form(olib):
+    """8-bit codes: value 64j starts at bit 512j; 1024 segments, then 2^19."""
+    x = workloads.all_patterns()
+    enc = oracle.encode(x)
+    seg = oracle.segment_index(x, enc.lengths, enc.total_bits)
+    assert np.array_equal(seg, 512 * np.arange(1025, dtype=np.uint32))
+
+
+@pytest.mark.parametrize("n", [1, 63, 64, 65, 4096, 40001])
+def test_segment_index_single_symbol_closed_form(olib, n):
+    """One value with a 1-bit code: value 64j starts at bit 64j; the last
+    entry is n (= total_bits)."""
+    x = workloads.constant(n, 0xBC00)
+    enc = oracle.encode(x)
+    seg = oracle.segment_index(x, enc.lengths, enc.total_bits).astype(np.int64)
+    S = (n + 63) // 64
+    assert seg.size == S + 1
+    assert np.array_equal(seg[:S], 64 * np.arange(S)) and seg[S] == n
+
+
+def test_segment_index_hand_example(olib):
+    """64 values of a 1-bit code, then 40 of a 2-bit code (144 bits): value
+    0 starts at bit 0, value 64 (the first 2-bit code) at bit 64."""
+    lengths = np.zeros(256, np.uint8)
+    codes = np.zeros(256, np.uint32)
+    lengths[10], codes[10] = 1, 0b0
+    lengths[20], codes[20] = 2, 0b10
+    x = np.array([10 << 7] * 64 + [20 << 7] * 40, np.uint16)
+    enc = oracle.encode(x, lengths=lengths, codes=codes)
+    assert oracle.segment_index(x, lengths, 144).tolist() == [0, 64, 144]
+    assert oracle.segment_index(x[:64], lengths, 64).tolist() == [0, 64]
+
+
+@pytest.mark.parametrize("n,cap", [(7, 11), (4097, 11), (100_000, 11), (300_001, 11), (70_001, 32)])
+def test_segment_index_against_stream_and_block_positions(olib, n, cap):
+    """Against the encoder's own arrays: the stream holds value 64j's code at
+    bit seg[j]; segments use between 64 x the shortest and 64 x the longest
+    code; and the segment starts before block b's first bit are exactly the
+    multiples of 64 below block_pos[b] (the codes that start before it)."""
+    x = workloads.random_bf16(n, seed=77 + n) if cap == 11 else workloads.fibonacci_exponents(26)[:n]
+    enc = oracle.encode(x, cap=cap)
+    seg = oracle.segment_index(x, enc.lengths, enc.total_bits).astype(np.int64)
+    e, _ = oracle.split(x)
+    S = (n + 63) // 64
+    assert seg.size == S + 1 and seg[0] == 0 and seg[S] == enc.total_bits
+    for j in range(0, S, max(1, S // 200)):
+        v = int(e[64 * j])
+        L = int(enc.lengths[v])
+        assert _code_at(enc.stream, int(seg[j]), L) == int(enc.codes[v]), j
+    used = enc.lengths[enc.lengths > 0]
+    d = np.diff(seg)
+    full = np.minimum(64, n - 64 * np.arange(S))
+    assert (d >= full * int(used.min())).all() and (d <= full * int(used.max())).all()
+    for b in range(enc.block_pos.size):
+        below = int((seg[:S] < 16384 * b).sum())
+        assert below == (int(enc.block_pos[b]) + 63) // 64, b
