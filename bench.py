@@ -37,7 +37,8 @@ import workloads  # noqa: E402
 
 METRIC = "DF11 decode output BF16 GB/s & % of HBM roofline (bit-exact); ratio"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_idx_kernel_traffic.txt")
+FALLBACK_BF16_TFLOPS = 1590.0  # the fallback dense BF16 figure (burst)
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_seg_kernel_traffic.txt")
 KERNEL_SOURCE = os.path.join(ROOT, "lossless_bf16_weight_df11_b200", "csrc", "df11_kernels.cu")
 ORACLE_SAMPLE = ("q", "o", "k", "v", "gate")
 CAP = 11  # code-length cap of the benchmarked codebooks: DF11_TABLE_BITS, the decode table's reach
@@ -96,12 +97,24 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-DECODE_BEGIN = "// ============================================================ decode"
+def measured_tensor_peak():
+    """Dense BF16 tensor-core peak (TFLOP/s) of this machine's B200s: the burst
+    figure, for a kernel timed alone."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+DECODE_BEGIN = "// ============================================================ segment decoder"
 DECODE_END = "// ============================================================ launch helpers"
 
 
 def kernel_hash() -> str:
-    """Fingerprint of the decode kernel's code (the decode section of
+    """Fingerprint of the segment decoder's code (its section of
     df11_kernels.cu without comments), so that a stored traffic figure is
     used only for the kernel it was measured on."""
     with open(KERNEL_SOURCE, encoding="utf-8") as f:
@@ -298,7 +311,7 @@ def time_configs(torch, df11, codec, dev, steps, warmup, peak, peak_kind, skip_w
             b.record(stream)
         torch.cuda.synchronize()
         ms = statistics.median(a.elapsed_time(b) for a, b in evs)
-        algo = sum(m.read_bytes + m.index_bytes for m in cms) + 2 * n
+        algo = sum(m.seg_read_bytes for m in cms) + 2 * n
         lines[workloads.workload_name(wid)] = {
             "weights": n, "matrices": len(xs), "ms_per_launch": ms,
             "value": 2 * n / (ms / 1e3) / 1e9, "unit": "GB/s", "weights_per_s": n / (ms / 1e3),
@@ -411,10 +424,13 @@ def run_df11(args):
     del cms_d
     read_bytes = sum(m.read_bytes for m in cms)
     index_bytes = sum(m.index_bytes for m in cms)
+    seg_read = sum(m.seg_read_bytes for m in cms)
+    seg_index_bytes = sum(4 * (-(-m.n // df11.SEGMENT) + 1) for m in cms)
     stored = sum(m.stored_bytes for m in cms)
     ratio = stored / (2 * n_total)
-    # compressed bytes read (the format's arrays and the run index) + BF16 written
-    algo_bytes = read_bytes + index_bytes + 2 * n_total
+    # the segment decoder's bytes: the stream, the sign/mantissa plane and the
+    # segment index read, the BF16 written
+    algo_bytes = seg_read + 2 * n_total
 
     outs = [torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in xs]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -464,53 +480,75 @@ def run_df11(args):
     if int(status.item()) != 0:
         raise df11.DF11Error(int(status.item()), "decode (device)")
 
-    # ---- the same block without its run index (the decoder that places the
-    # exponents after a prefix sum of the per-thread counts), and the time to
-    # build the index (once, when a matrix is placed on the device)
-    no_index = None
+    # ---- the same block through the two other decoders: with the run index
+    # (each thread's first output known, exponents placed directly) and with
+    # no index (per-unit prefix sums of the threads' counts); and the time to
+    # build each index (once, when a matrix is placed on the device)
+    other = None
     if args.cap32:
-        abis_ni = [m.abi(False) for m in cms]
+        other = {}
+        for name, kw, kern, algo in (
+                ("run_index", (True, False), "decode_idx_kernel", read_bytes + index_bytes + 2 * n_total),
+                ("no_index", (False, False), "decode_kernel", read_bytes + 2 * n_total)):
+            abis_o = [m.abi(*kw) for m in cms]
 
-        def step_ni():
-            st = df11.df11_decode_block_batch(abis_ni, out_ptrs, status.data_ptr(), sh)
-            if st:
-                raise df11.DF11Error(st, "df11_decode_block_batch")
+            def step_o():
+                st = df11.df11_decode_block_batch(abis_o, out_ptrs, status.data_ptr(), sh)
+                if st:
+                    raise df11.DF11Error(st, "df11_decode_block_batch")
 
-        with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                step_ni()
-        torch.cuda.synchronize()
-        ok_ni = all(torch.equal(o.reshape(-1).view(torch.int16), w) for o, w in zip(outs, ws))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.steps):
-                step_ni()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        ms_ni = e0.elapsed_time(e1) / args.steps
+            for o in outs:
+                o.zero_()
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    step_o()
+            torch.cuda.synchronize()
+            ok_o = int(status.item()) == 0 and all(
+                torch.equal(o.reshape(-1).view(torch.int16), w) for o, w in zip(outs, ws))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(args.steps):
+                    step_o()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            ms_o = e0.elapsed_time(e1) / args.steps
+            other[name] = {"ms_per_step": ms_o, "value": 2 * n_total / (ms_o / 1e3) / 1e9,
+                           "unit": "GB/s", "kernel": kern, "algorithmic_bytes_per_launch": algo,
+                           "roofline_frac": algo / (ms_o / 1e3) / 1e9 / measured_peak()[0],
+                           "bit_exact": ok_o}
         ri_status = torch.zeros(1, dtype=torch.int32, device=dev)
         tmp_ri = [torch.empty_like(m.run_index) for m in cms]
+        tmp_si = [torch.empty_like(m.seg_index) for m in cms]
 
-        def build_index():
+        def build_run_index():
             for m, r in zip(cms, tmp_ri):
-                df11.check(df11.df11_build_run_index(m.abi(False), r.data_ptr(), ri_status.data_ptr(),
-                                                     sh), "df11_build_run_index")
+                df11.check(df11.df11_build_run_index(m.abi(False, False), r.data_ptr(),
+                                                     ri_status.data_ptr(), sh), "df11_build_run_index")
 
-        with torch.cuda.stream(stream):
-            build_index()
-            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            b0.record(stream)
-            build_index()
-            b1.record(stream)
-        torch.cuda.synchronize()
-        same_index = all(torch.equal(a, m.run_index) for a, m in zip(tmp_ri, cms))
-        del tmp_ri
-        no_index = {"ms_per_step": ms_ni, "value": 2 * n_total / (ms_ni / 1e3) / 1e9, "unit": "GB/s",
-                    "roofline_frac": (read_bytes + 2 * n_total) / (ms_ni / 1e3) / 1e9 / measured_peak()[0],
-                    "bit_exact": ok_ni, "kernel": "decode_kernel",
-                    "run_index_build_ms": b0.elapsed_time(b1), "run_index_bytes": index_bytes,
-                    "run_index_rebuilt_identical": same_index and int(ri_status.item()) == 0}
+        def build_seg_index():
+            for m, r in zip(cms, tmp_si):
+                df11.check(df11.df11_build_segment_index(m.abi(False, False), r.data_ptr(),
+                                                         ri_status.data_ptr(), sh),
+                           "df11_build_segment_index")
+
+        build_ms = {}
+        for nm, fn in (("run_index", build_run_index), ("seg_index", build_seg_index)):
+            with torch.cuda.stream(stream):
+                fn()
+                b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                b0.record(stream)
+                fn()
+                b1.record(stream)
+            torch.cuda.synchronize()
+            build_ms[nm] = b0.elapsed_time(b1)
+        same_index = (all(torch.equal(a, m.run_index) for a, m in zip(tmp_ri, cms)) and
+                      all(torch.equal(a, m.seg_index) for a, m in zip(tmp_si, cms)))
+        del tmp_ri, tmp_si
+        other["index_build"] = {"run_index_ms": build_ms["run_index"],
+                                "seg_index_ms": build_ms["seg_index"],
+                                "run_index_bytes": index_bytes, "seg_index_bytes": seg_index_bytes,
+                                "rebuilt_identical": same_index and int(ri_status.item()) == 0}
 
     # ---- the rANS variant of the exponent coding on the same block: its
     # ratio and decode time beside the Huffman format's, launches alternated
@@ -531,7 +569,7 @@ def run_df11(args):
     if args.cap32:
         cms32 = [codec.compress(w, cap=32) for w in ws]
         abis32 = [m.abi() for m in cms32]
-        algo32 = sum(m.read_bytes + m.index_bytes for m in cms32) + 2 * n_total
+        algo32 = sum(m.seg_read_bytes for m in cms32) + 2 * n_total
 
         def step32():
             st = df11.df11_decode_block_batch(abis32, out_ptrs, status.data_ptr(), sh)
@@ -573,9 +611,16 @@ def run_df11(args):
     if args.block_steps > 0 and wid in BLOCK_SHAPES:
         blockfw = time_block_forward(torch, cms, ws, mats_def, wid, dev, args.block_steps)
     fused = None
+    tc_gemm = None
     if args.matmul_steps > 0:
         fused = [time_fused_matmul(torch, df11, cms, abis, outs, out_ptrs, status, xs_shapes(mats_def),
                                    dev, b, args.matmul_steps, peak, peak_kind) for b in (1, 8)]
+        tf, tf_kind = measured_tensor_peak()
+        tc_gemm = []
+        for b in (16, 64, 256, 1024, 2048):
+            tc_gemm.append(time_tc_gemm(torch, df11, cms, out_ptrs, outs, status, xs_shapes(mats_def),
+                                        dev, b, args.matmul_steps, tf, tf_kind, peak))
+            torch.cuda.empty_cache()
 
     configs, cpu_plan = None, None
     if args.config_steps > 0:
@@ -590,9 +635,9 @@ def run_df11(args):
     achieved = algo_bytes / (avg_launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": profiled_traffic(name),
-                "peak_kind": peak_kind, "kernel": "decode_idx_kernel",
+                "peak_kind": peak_kind, "kernel": "decode_seg_kernel",
                 "algorithmic_bytes_per_launch": algo_bytes,
-                "run_index_bytes_per_launch": index_bytes,
+                "seg_index_bytes_per_launch": seg_index_bytes,
                 "frac_of_8TBps": achieved / 8000.0,
                 "median_launch_ms": statistics.median(per_launch_ms)}
 
@@ -631,12 +676,13 @@ def run_df11(args):
                                                   "host, all encodes, one copy of the status words"},
             "encode": encode,
             "fused_matmul": fused,
+            "tc_gemm": tc_gemm,
             "block_forward": blockfw,
             "rans": rans_line,
             "code_len_cap": CAP,
             "max_code_len": max(int(m.codebook.max_len) for m in cms),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "cap32": cap32,
-            "configs": configs, "cpu_baseline_plan": cpu_plan, "no_run_index": no_index,
+            "configs": configs, "cpu_baseline_plan": cpu_plan, "other_decoders": other,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -871,13 +917,93 @@ def time_fused_matmul(torch, df11, cms, abis, outs, out_ptrs, status, shapes, de
                          "peak_kind": peak_kind, "algorithmic_bytes": algo}}
 
 
+def time_tc_gemm(torch, df11, cms, out_ptrs, outs, status, shapes, dev, batch, steps, peak_tf,
+                 peak_tf_kind, hbm_peak):
+    """Per step, for all matrices W_i (rows x cols) of the block and BF16
+    activations x_i (batch x cols): y_i += x_i W_i^T.  Three ways: the
+    tensor-core fused kernel (df11_decode_gemm_batch: W decoded into the MMA's
+    operand tiles, one pass per 256 activation rows); decode into BF16 then
+    torch.matmul (cuBLAS); the matmul alone with the BF16 weights resident."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(4321 + batch)
+    xs = [torch.randn(batch, c, generator=g, device=dev).to(torch.bfloat16) for _, c in shapes]
+    ys = [torch.zeros(batch, r, dtype=torch.float32, device=dev) for r, _ in shapes]
+    ios = [df11.df11_matmul_io(rows=r, cols=c, x=x.data_ptr(), y=y.data_ptr())
+           for (r, c), x, y in zip(shapes, xs, ys)]
+    abis = [m.abi() for m in cms]
+    stream = torch.cuda.current_stream(dev)
+    sh = int(stream.cuda_stream)
+    ws_bf16 = [o.view(r, c) for o, (r, c) in zip(outs, shapes)]
+
+    def fused():
+        df11.check(df11.df11_decode_gemm_batch(abis, ios, batch, status.data_ptr(), sh),
+                   "df11_decode_gemm_batch")
+
+    def decode_then_matmul():
+        df11.check(df11.df11_decode_block_batch(abis, out_ptrs, status.data_ptr(), sh),
+                   "df11_decode_block_batch")
+        for x, w, y in zip(xs, ws_bf16, ys):
+            y.add_(torch.matmul(x, w.t()).float())
+
+    def matmul_only():
+        for x, w, y in zip(xs, ws_bf16, ys):
+            y.add_(torch.matmul(x, w.t()).float())
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    t_fused = timed(fused)
+    # one step from zero, checked on 16 sampled rows of every W against a
+    # float64 product, within (cols + 8) ulps of the sum of |w x|
+    for y in ys:
+        y.zero_()
+    fused()
+    decode_then_matmul()  # fills the BF16 weights (and adds the cuBLAS product to y)
+    for y in ys:
+        y.zero_()
+    fused()
+    ok = int(status.item()) == 0
+    for x, w, y in zip(xs, ws_bf16, ys):
+        rows = torch.randperm(w.shape[0], generator=torch.Generator().manual_seed(batch))[:16].to(dev)
+        wr = w[rows].double()
+        ref = x.double() @ wr.t()
+        bound = (x.double().abs() @ wr.abs().t()) * (w.shape[1] + 8) * 2.0 ** -23 * 1.01
+        ok = ok and bool(((y[:, rows].double() - ref).abs() <= bound).all())
+    t_unfused = timed(decode_then_matmul)
+    t_mm = timed(matmul_only)
+    if int(status.item()) != 0:
+        raise df11.DF11Error(int(status.item()), "tensor-core fused GEMM (device)")
+    flops = 2.0 * batch * sum(r * c for r, c in shapes)
+    passes = -(-batch // df11.GEMM_MAX_BATCH)
+    algo = (passes * sum(m.seg_read_bytes for m in cms) + sum(2 * x.numel() for x in xs)
+            + sum(8 * y.numel() for y in ys))  # compressed W per pass, x, y read and written
+    return {"batch": batch, "fused_ms": t_fused, "decode_then_matmul_ms": t_unfused,
+            "matmul_only_ms": t_mm, "speedup_vs_decode_then_matmul": t_unfused / t_fused,
+            "passes": passes, "within_fp32_bound_sampled": ok, "kernel": "decode_gemm_tc_kernel",
+            "roofline": {"bound": "tensor", "achieved": flops / (t_fused / 1e3) / 1e12,
+                         "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": flops / (t_fused / 1e3) / 1e12 / peak_tf, "peak_kind": peak_tf_kind,
+                         "flops": flops},
+            "hbm_view": {"achieved": algo / (t_fused / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": algo / (t_fused / 1e3) / 1e9 / hbm_peak, "bytes": algo}}
+
+
 def end_to_end(torch, df11, codec, cms, xs, dev, steps, dist, world):
     """Host-resident compressed block -> device (pinned H2D), one decode
     launch, decoded BF16 -> host (D2H), every step, all timed."""
     host_parts, dev_parts = [], []
     h2d = 0
     for m in cms:
-        for buf in (m.stream, m.gaps, m.block_pos, m.sign_mantissa, m.tables):
+        for buf in (m.stream, m.gaps, m.block_pos, m.sign_mantissa, m.tables, m.seg_index):
             h = torch.empty(buf.shape, dtype=buf.dtype, pin_memory=True)
             h.copy_(buf)
             d = torch.empty_like(buf)
@@ -892,11 +1018,11 @@ def end_to_end(torch, df11, codec, cms, xs, dev, steps, dist, world):
     abis = []
     k = 0
     for m in cms:
-        d_stream, d_gaps, d_pos, d_sm, d_tab = dev_parts[k:k + 5]
-        k += 5
-        a = m.abi()
+        d_stream, d_gaps, d_pos, d_sm, d_tab, d_seg = dev_parts[k:k + 6]
+        k += 6
+        a = m.abi(False, True)
         a.stream, a.gaps, a.block_pos = d_stream.data_ptr(), d_gaps.data_ptr(), d_pos.data_ptr()
-        a.sign_mantissa, a.tables = d_sm.data_ptr(), d_tab.data_ptr()
+        a.sign_mantissa, a.tables, a.seg_index = d_sm.data_ptr(), d_tab.data_ptr(), d_seg.data_ptr()
         abis.append(a)
     stream = torch.cuda.Stream(device=dev)
     sh = int(stream.cuda_stream)

@@ -104,6 +104,9 @@ typedef struct {
   uint64_t workspace_bytes;    /* df11_encode scratch                           */
   uint64_t run_index_bytes;    /* df11_build_run_index output (128 uint16 per
                                   block; 16-byte multiple)                      */
+  uint64_t seg_index_bytes;    /* df11_build_segment_index output (uint32 per
+                                  DF11_SEGMENT values, plus one; rounded up to
+                                  16 bytes)                                     */
 } df11_sizes;
 
 /* One compressed matrix in device memory (non-owning).  Every pointer must be
@@ -126,6 +129,11 @@ typedef struct {
                                   index from df11_build_run_index, 16-byte
                                   aligned.  With it the decoder places every
                                   thread's outputs before decoding them       */
+  const uint32_t *seg_index;   /* optional (NULL: not used): the matrix's
+                                  segment index from df11_build_segment_index,
+                                  4-byte aligned.  With it every decoding lane
+                                  starts at a known stream bit and decodes a
+                                  known number of values                       */
 } df11_matrix;
 
 /* Encoder outputs in device memory (sizes from df11_encoded_sizes). */
@@ -300,8 +308,12 @@ df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32_t *d_statu
  *   ms      host array of count matrices, each with its own tables.
  *   d_outs  host array of count device pointers (16-byte aligned).
  * One launch per DF11_MAX_BATCH matrices.  When every matrix of a launch has
- * a run index (df11_matrix.run_index), the launch takes the indexed decoder;
- * each thread's decoded count is then also checked against the index.
+ * a segment index (df11_matrix.seg_index; total_bits < 2^32), the launch
+ * takes the segment decoder: each segment's decode must end exactly where the
+ * next segment starts.  Otherwise, when every matrix has a run index
+ * (df11_matrix.run_index), the launch takes the indexed decoder, and each
+ * thread's decoded count is also checked against the index.  Without either
+ * index every block's count is checked against its stored position.
  */
 df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
                                     uint16_t *const *d_outs, uint32_t *d_status,
@@ -327,6 +339,32 @@ df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
  */
 df11_status df11_build_run_index(const df11_matrix *m, uint16_t *d_run_index, uint32_t *d_status,
                                  df11_stream_t stream);
+
+/*
+ * df11_build_segment_index -- the segment index of one matrix: for every
+ * segment of DF11_SEGMENT consecutive values, the stream bit at which the
+ * code of its first value starts, as uint32 at d_seg_index[j] (value
+ * DF11_SEGMENT * j), j < S = ceil(n / DF11_SEGMENT); d_seg_index[S] =
+ * total_bits.  [Kernel] stores, per thread block, where in the output a
+ * block's codes go; this is the converse map (where in the stream an output
+ * position's code is) at a fixed step of outputs.  It is derived from the
+ * stream (not stored in the format): built once when a matrix is placed on
+ * the device, it costs 4 bytes per 64 values (0.0625 B per weight) of device
+ * memory and of decode traffic, and lets df11_decode give every lane exactly
+ * DF11_SEGMENT values to decode from a known stream bit: no counting pass, no
+ * prefix sum and no relocation of the exponents.
+ *   m            the matrix (its run_index and seg_index fields are ignored).
+ *   d_seg_index  sizes.seg_index_bytes device bytes, 4-byte aligned; written.
+ *   d_status     DF11_ERR_CORRUPT if a block's code count disagrees with its
+ *                stored positions or a code is invalid (the index is then
+ *                unusable).
+ * Returns DF11_ERR_TOO_LARGE when total_bits >= 2^32 (the entries are 32-bit;
+ * such a matrix decodes without this index).  One kernel launch (a memset for
+ * n = 0).
+ */
+#define DF11_SEGMENT 64u
+df11_status df11_build_segment_index(const df11_matrix *m, uint32_t *d_seg_index,
+                                     uint32_t *d_status, df11_stream_t stream);
 
 /* Activations and sums of one matrix for df11_decode_matmul_batch.  The
  * matrix W holds rows x cols values in row-major order (the order it was
@@ -363,6 +401,35 @@ typedef struct {
 df11_status df11_decode_matmul_batch(const df11_matrix *ms, const df11_matmul_io *io,
                                      uint32_t count, uint32_t batch, uint32_t *d_status,
                                      df11_stream_t stream);
+
+/*
+ * df11_decode_gemm_batch -- the same product for larger batches, on the
+ * tensor cores:  y[j][r] += sum_c W[r][c] * x[j][c]  (j < batch), with W
+ * decoded through its segment index straight into the B operand of
+ * tcgen05.mma (never written to device memory) and FP32 accumulators in
+ * tensor memory.  [GPU]: decompression right before the matmul, discarded
+ * after; each weight is decoded once per DF11_GEMM_MAX_BATCH activation rows.
+ *   ms, io   host arrays of count matrices and their activations and sums;
+ *            every matrix needs its segment index (df11_matrix.seg_index),
+ *            cols a multiple of DF11_SEGMENT and total_bits < 2^32; x 16-byte
+ *            and y 4-byte aligned.  Nothing else of the matrix is read but
+ *            the stream, the sign/mantissa plane and the tables.
+ *   batch    activation rows, >= 1; one pass per DF11_GEMM_MAX_BATCH rows
+ *            (W is decoded again for each pass).
+ *   d_status DF11_ERR_CORRUPT when a segment does not decode to exactly
+ *            DF11_SEGMENT values ending where the next one starts (its
+ *            weights then count as zero); DF11_ERR_TIMEOUT when a bounded
+ *            wait inside the kernel ran out (y is then left unchanged for the
+ *            tiles concerned).
+ * Products are exact in FP32 and summed in FP32 in the tensor cores' order,
+ * so the result agrees with an exact sum within cols * 2^-23 * sum |w x| per
+ * entry (the same bound as df11_decode_matmul_batch's).
+ * One launch per DF11_MAX_BATCH matrices and pass; one CTA per 128 rows of W.
+ */
+#define DF11_GEMM_MAX_BATCH 256u
+df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_matmul_io *io,
+                                   uint32_t count, uint32_t batch, uint32_t *d_status,
+                                   df11_stream_t stream);
 
 /*
  * df11_validate -- host.  Checks stored metadata before it is trusted:

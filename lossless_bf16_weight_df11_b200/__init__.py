@@ -32,6 +32,7 @@ MAX_CODE_LEN = 32
 MAX_N = 0xFFFFFFFF
 MAX_BATCH = 32
 TABLE_BITS = 11  # decode-table reach; the codec's default length cap
+SEGMENT = 64     # DF11_SEGMENT: values per entry of the segment index
 
 DF11_OK = 0
 DF11_ERR_INVALID_ARG = 1
@@ -56,7 +57,7 @@ class df11_sizes(ctypes.Structure):
         "stream_bytes", "gaps_bytes", "block_pos_bytes", "sign_mantissa_bytes",
         "stored_bytes",
         "stream_alloc", "gaps_alloc", "block_pos_alloc", "sign_mantissa_alloc",
-        "tables_bytes", "workspace_bytes", "run_index_bytes")]
+        "tables_bytes", "workspace_bytes", "run_index_bytes", "seg_index_bytes")]
 
 
 class df11_matrix(ctypes.Structure):
@@ -64,7 +65,8 @@ class df11_matrix(ctypes.Structure):
                 ("stream", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
                 ("block_pos", ctypes.c_void_p), ("sign_mantissa", ctypes.c_void_p),
                 ("tables", ctypes.c_void_p), ("min_len", ctypes.c_uint32),
-                ("max_block_codes", ctypes.c_uint32), ("run_index", ctypes.c_void_p)]
+                ("max_block_codes", ctypes.c_uint32), ("run_index", ctypes.c_void_p),
+                ("seg_index", ctypes.c_void_p)]
 
 
 class df11_encoded(ctypes.Structure):
@@ -131,9 +133,13 @@ def _declare(lib):
         "df11_decode_matmul_batch": (ctypes.c_int, [ctypes.POINTER(df11_matrix),
                                                     ctypes.POINTER(df11_matmul_io), _u32, _u32,
                                                     _vp, _vp]),
+        "df11_decode_gemm_batch": (ctypes.c_int, [ctypes.POINTER(df11_matrix),
+                                                  ctypes.POINTER(df11_matmul_io), _u32, _u32,
+                                                  _vp, _vp]),
         "df11_sizes_from_bits": (ctypes.c_int, [_u64, _u64, ctypes.POINTER(df11_sizes)]),
         "df11_file_bytes": (_u64, [_u64, _u64]),
         "df11_build_run_index": (ctypes.c_int, [ctypes.POINTER(df11_matrix), _vp, _vp, _vp]),
+        "df11_build_segment_index": (ctypes.c_int, [ctypes.POINTER(df11_matrix), _vp, _vp, _vp]),
         "df11_write": (ctypes.c_int, [ctypes.POINTER(df11_host_matrix), _vp, _u64,
                                       ctypes.POINTER(ctypes.c_uint64)]),
         "df11_read": (ctypes.c_int, [_vp, _u64, ctypes.POINTER(df11_host_matrix)]),
@@ -242,6 +248,7 @@ def df11_decode_block_batch(ms, d_outs, d_status: int, stream: int = 0) -> int:
 
 MATMUL_MAX_BATCH = 8      # DF11_MATMUL_MAX_BATCH
 MATMUL_MIN_COLS = 256     # DF11_MATMUL_MIN_COLS
+GEMM_MAX_BATCH = 256      # DF11_GEMM_MAX_BATCH: activation rows per pass of the tensor-core path
 
 
 def df11_decode_matmul_batch(ms, ios, batch: int, d_status: int, stream: int = 0) -> int:
@@ -250,6 +257,14 @@ def df11_decode_matmul_batch(ms, ios, batch: int, d_status: int, stream: int = 0
     arr = (df11_matrix * len(ms))(*ms)
     io = (df11_matmul_io * len(ios))(*ios)
     return load().df11_decode_matmul_batch(arr, io, len(ms), batch, d_status, stream)
+
+
+def df11_decode_gemm_batch(ms, ios, batch: int, d_status: int, stream: int = 0) -> int:
+    """y += x W^T on the tensor cores, W decoded through its segment index;
+    see include/df11.h."""
+    arr = (df11_matrix * len(ms))(*ms)
+    io = (df11_matmul_io * len(ios))(*ios)
+    return load().df11_decode_gemm_batch(arr, io, len(ms), batch, d_status, stream)
 
 
 def df11_validate(n: int, total_bits: int, min_len: int, h_gaps: int, gaps_bytes: int,
@@ -268,6 +283,13 @@ def df11_build_run_index(m: df11_matrix, d_run_index: int, d_status: int, stream
     """The matrix's run index (per pair of chunks, its first output within its
     block) into device memory; see include/df11.h."""
     return load().df11_build_run_index(ctypes.byref(m), d_run_index, d_status, stream)
+
+
+def df11_build_segment_index(m: df11_matrix, d_seg_index: int, d_status: int,
+                             stream: int = 0) -> int:
+    """The matrix's segment index (the stream bit of every 64th code, then
+    total_bits) into device memory; see include/df11.h."""
+    return load().df11_build_segment_index(ctypes.byref(m), d_seg_index, d_status, stream)
 
 
 def df11_file_bytes(n: int, total_bits: int) -> int:

@@ -18,10 +18,11 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-from . import (CODEBOOK_BYTES, MAX_CODE_LEN, TABLE_BITS, DF11Error, check, df11_build_codebook,
+from . import (CODEBOOK_BYTES, MAX_CODE_LEN, SEGMENT, TABLE_BITS, DF11Error, check,
+               df11_build_codebook, df11_build_segment_index,
                df11_build_codebook_device, df11_build_tables, df11_codebook,
                df11_codebook_from_lengths, df11_decode, df11_decode_block_batch,
-               df11_decode_matmul_batch, df11_encode, df11_encode_device_codebook, df11_encoded,
+               df11_decode_matmul_batch, df11_decode_gemm_batch, df11_encode, df11_encode_device_codebook, df11_encoded,
                df11_build_run_index, df11_encoded_sizes, df11_file_bytes, df11_histogram,
                df11_host_matrix, df11_matmul_io,
                df11_matrix, df11_read, df11_sizes, df11_sizes_from_bits, df11_tables_bytes,
@@ -59,15 +60,20 @@ class DF11Matrix:
     hist: np.ndarray = field(repr=False, default=None)
     max_block_codes: int = 0     # most codes in one block (0 = unknown)
     run_index: torch.Tensor | None = None  # int16 (uint16 bits), df11_build_run_index
+    seg_index: torch.Tensor | None = None  # int32 (uint32 bits), df11_build_segment_index
 
-    def abi(self, use_run_index: bool = True) -> df11_matrix:
+    def abi(self, use_run_index: bool = True, use_seg_index: bool = True) -> df11_matrix:
+        """The C-ABI view.  The decoder takes the segment index when every
+        matrix of a launch passes one, else the run index, else neither."""
         ri = self.run_index if (use_run_index and self.run_index is not None) else None
+        si = self.seg_index if (use_seg_index and self.seg_index is not None) else None
         return df11_matrix(n=self.n, total_bits=self.total_bits, stream=self.stream.data_ptr(),
                            gaps=self.gaps.data_ptr(), block_pos=self.block_pos.data_ptr(),
                            sign_mantissa=self.sign_mantissa.data_ptr(),
                            tables=self.tables.data_ptr(), min_len=max(1, self.codebook.min_len),
                            max_block_codes=self.max_block_codes,
-                           run_index=ri.data_ptr() if ri is not None else None)
+                           run_index=ri.data_ptr() if ri is not None else None,
+                           seg_index=si.data_ptr() if si is not None else None)
 
     @property
     def stored_bytes(self) -> int:
@@ -87,6 +93,13 @@ class DF11Matrix:
     def index_bytes(self) -> int:
         """Bytes of the run index (0 without one): read by the indexed decoder."""
         return int(self.sizes.run_index_bytes) if self.run_index is not None else 0
+
+    @property
+    def seg_read_bytes(self) -> int:
+        """Bytes the segment decoder reads: the stream, the sign/mantissa plane
+        and the segment index (not the gaps or block positions)."""
+        s = self.sizes
+        return int(s.stream_bytes) + int(s.sign_mantissa_bytes) + 4 * (-(-self.n // SEGMENT) + 1)
 
     def host_arrays(self):
         """Stored arrays copied to the host (for checks and serialisation)."""
@@ -131,19 +144,25 @@ DEFAULT_CAP = TABLE_BITS
 
 def _run_index_for(n: int, total_bits: int, codebook: df11_codebook, sizes: df11_sizes, bufs,
                    tables: torch.Tensor, status_ptr: int, sh: int, dev) -> torch.Tensor | None:
-    """Enqueue df11_build_run_index for freshly encoded (or uploaded) buffers;
-    returns the index tensor (None for an empty matrix).  Errors land in the
-    device status word at status_ptr."""
+    """Enqueue df11_build_run_index and df11_build_segment_index for freshly
+    encoded (or uploaded) buffers; returns the two index tensors (None for an
+    empty matrix, and no segment index for a stream of 2^32 bits or more).
+    Errors land in the device status word at status_ptr."""
     if n == 0:
-        return None
+        return None, None
     ri = torch.empty(max(16, int(sizes.run_index_bytes)) // 2, dtype=torch.int16, device=dev)
+    si = (torch.empty(int(sizes.seg_index_bytes) // 4, dtype=torch.int32, device=dev)
+          if total_bits < (1 << 32) else None)
     m = df11_matrix(n=n, total_bits=total_bits, stream=bufs["stream"].data_ptr(),
                     gaps=bufs["gaps"].data_ptr(), block_pos=bufs["block_pos"].data_ptr(),
                     sign_mantissa=bufs["sign_mantissa"].data_ptr(), tables=tables.data_ptr(),
                     min_len=max(1, codebook.min_len), max_block_codes=0, run_index=None)
     with torch.cuda.device(dev):
         check(df11_build_run_index(m, ri.data_ptr(), status_ptr, sh), "df11_build_run_index")
-    return ri
+        if si is not None:
+            check(df11_build_segment_index(m, si.data_ptr(), status_ptr, sh),
+                  "df11_build_segment_index")
+    return ri, si
 
 
 def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | None = None,
@@ -178,14 +197,14 @@ def compress(w: torch.Tensor, cap: int = DEFAULT_CAP, codebook: df11_codebook | 
     with torch.cuda.device(dev):
         check(df11_encode(u.data_ptr(), u.numel(), codebook, sizes.total_bits, out,
                           ws.data_ptr(), ws.numel(), status.data_ptr(), sh), "df11_encode")
-    ri = (_run_index_for(u.numel(), int(sizes.total_bits), codebook, sizes, bufs, tables,
-                         status.data_ptr(), sh, dev) if run_index else None)
+    ri, si = (_run_index_for(u.numel(), int(sizes.total_bits), codebook, sizes, bufs, tables,
+                             status.data_ptr(), sh, dev) if run_index else (None, None))
     st_host = status.cpu().numpy()
     if check_status and int(st_host[0]):
         raise DF11Error(int(st_host[0]), "df11_encode (device)")
     return DF11Matrix(shape=tuple(w.shape), n=u.numel(), total_bits=int(sizes.total_bits),
                       codebook=codebook, sizes=sizes, tables=tables, hist=hist,
-                      max_block_codes=int(st_host[1]), run_index=ri, **bufs)
+                      max_block_codes=int(st_host[1]), run_index=ri, seg_index=si, **bufs)
 
 
 def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
@@ -235,7 +254,7 @@ def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
                               wsb.numel(), status[i].data_ptr(), sh), "df11_encode")
             mats_bufs.append(bufs)
     ris = [(_run_index_for(u.numel(), int(sizes.total_bits), cb, sizes, bufs, tables[i],
-                           status[i].data_ptr(), sh, dev) if run_index else None)
+                           status[i].data_ptr(), sh, dev) if run_index else (None, None))
            for i, (u, cb, sizes, bufs) in enumerate(zip(us, cbs, sizes_l, mats_bufs))]
     st_host = status.cpu().numpy()  # round trip 2
     mats = []
@@ -245,8 +264,8 @@ def compress_block(ws, cap: int = DEFAULT_CAP, stream=None,
         mats.append(DF11Matrix(shape=tuple(w.shape), n=u.numel(),
                                total_bits=int(sizes_l[i].total_bits), codebook=cbs[i],
                                sizes=sizes_l[i], tables=tables[i], hist=h_all[i],
-                               max_block_codes=int(st_host[i, 1]), run_index=ris[i],
-                               **mats_bufs[i]))
+                               max_block_codes=int(st_host[i, 1]), run_index=ris[i][0],
+                               seg_index=ris[i][1], **mats_bufs[i]))
     return mats
 
 
@@ -312,7 +331,7 @@ def compress_block_device(ws, cap: int = DEFAULT_CAP, stream=None,
                   "df11_encode_device_codebook")
             mats_bufs.append(bufs)
     ris = [(_run_index_for(u.numel(), int(sizes.total_bits), cb, sizes, bufs, tables[i],
-                           status[i].data_ptr(), sh, dev) if run_index else None)
+                           status[i].data_ptr(), sh, dev) if run_index else (None, None))
            for i, (u, cb, sizes, bufs) in enumerate(zip(us, cbs, sizes_l, mats_bufs))]
     st_host = status.cpu().numpy()                                   # round trip 2
     mats = []
@@ -322,15 +341,15 @@ def compress_block_device(ws, cap: int = DEFAULT_CAP, stream=None,
         mats.append(DF11Matrix(shape=tuple(w.shape), n=u.numel(),
                                total_bits=int(sizes_l[i].total_bits), codebook=cbs[i],
                                sizes=sizes_l[i], tables=tables[i], hist=h_all[i].copy(),
-                               max_block_codes=int(st_host[i, 1]), run_index=ris[i],
-                               **mats_bufs[i]))
+                               max_block_codes=int(st_host[i, 1]), run_index=ris[i][0],
+                               seg_index=ris[i][1], **mats_bufs[i]))
     return mats
 
 
 def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
-               stream=None, run_index: bool = True) -> torch.Tensor:
-    """Decode one matrix (with its run index when it has one, unless
-    run_index is False)."""
+               stream=None, run_index: bool = True, seg_index: bool = True) -> torch.Tensor:
+    """Decode one matrix: with its segment index when it has one, else with
+    its run index; seg_index / run_index False leave the index out."""
     dev = m.stream.device
     if out is None:
         out = torch.empty(m.shape, dtype=torch.bfloat16, device=dev)
@@ -338,7 +357,7 @@ def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Ten
     if own_status:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
-        check(df11_decode(m.abi(run_index), out.data_ptr(), status.data_ptr(),
+        check(df11_decode(m.abi(run_index, seg_index), out.data_ptr(), status.data_ptr(),
                           _stream_handle(stream)), "df11_decode")
     if own_status:
         s = int(status.item())
@@ -348,9 +367,10 @@ def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Ten
 
 
 def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=None,
-                     run_index: bool = True):
-    """Decode every matrix of a block in one launch (the indexed decoder when
-    every matrix has a run index, unless run_index is False)."""
+                     run_index: bool = True, seg_index: bool = True):
+    """Decode every matrix of a block in one launch (the segment decoder when
+    every matrix has a segment index, else the indexed decoder when every
+    matrix has a run index; seg_index / run_index False leave them out)."""
     dev = ms[0].stream.device
     if outs is None:
         outs = [torch.empty(m.shape, dtype=torch.bfloat16, device=dev) for m in ms]
@@ -358,7 +378,8 @@ def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=N
     if own_status:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
-        check(df11_decode_block_batch([m.abi(run_index) for m in ms], [o.data_ptr() for o in outs],
+        check(df11_decode_block_batch([m.abi(run_index, seg_index) for m in ms],
+                                      [o.data_ptr() for o in outs],
                                       status.data_ptr(), _stream_handle(stream)),
               "df11_decode_block_batch")
     if own_status:
@@ -397,6 +418,38 @@ def matmul_block(ms, xs, ys=None, status: torch.Tensor | None = None, stream=Non
     return ys
 
 
+def gemm_block(ms, xs, ys=None, status: torch.Tensor | None = None, stream=None):
+    """y_i = x_i W_i^T for every matrix W_i of a block on the tensor cores
+    (df11_decode_gemm_batch): W_i decoded through its segment index into the
+    MMA's operand tiles, never written to device memory.  xs: BF16 tensors of
+    shape (batch, cols_i) with cols_i a multiple of SEGMENT, any batch; ys:
+    FP32 (batch, rows_i), zeroed here when not given (the products are
+    added)."""
+    dev = ms[0].stream.device
+    batch = int(xs[0].shape[0])
+    for m, x in zip(ms, xs):
+        if len(m.shape) != 2 or x.dtype != torch.bfloat16 or x.shape != (batch, m.shape[1]):
+            raise ValueError("gemm_block: x must be BF16 (batch, cols) for a rows x cols matrix")
+        if m.seg_index is None:
+            raise ValueError("gemm_block: the matrix has no segment index")
+    xs = [x.contiguous() for x in xs]
+    if ys is None:
+        ys = [torch.zeros(batch, m.shape[0], dtype=torch.float32, device=dev) for m in ms]
+    ios = [df11_matmul_io(rows=m.shape[0], cols=m.shape[1], x=x.data_ptr(), y=y.data_ptr())
+           for m, x, y in zip(ms, xs, ys)]
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        check(df11_decode_gemm_batch([m.abi() for m in ms], ios, batch, status.data_ptr(),
+                                     _stream_handle(stream)), "df11_decode_gemm_batch")
+    if own_status:
+        s = int(status.item())
+        if s:
+            raise DF11Error(s, "df11_decode_gemm_batch (device)")
+    return ys
+
+
 def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, stream, gaps,
                      block_pos, sign_mantissa, device, run_index: bool = True) -> DF11Matrix:
     """Upload stored arrays (e.g. produced elsewhere) into padded device
@@ -416,19 +469,19 @@ def from_host_arrays(shape, n: int, total_bits: int, codebook: df11_codebook, st
                                  sizes.block_pos_alloc, np.int32),
                 sign_mantissa=padded(sign_mantissa, sizes.sign_mantissa_alloc))
     tables = build_tables(codebook, device)
-    ri = None
+    ri = si = None
     if run_index and n:
         # the index of data from elsewhere is built here, on the device; a
         # stream that does not match its positions is reported
         dev = bufs["stream"].device
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        ri = _run_index_for(n, total_bits, codebook, sizes, bufs, tables, status.data_ptr(),
-                            _stream_handle(None), dev)
+        ri, si = _run_index_for(n, total_bits, codebook, sizes, bufs, tables, status.data_ptr(),
+                                _stream_handle(None), dev)
         st = int(status.item())
         if st:
-            raise DF11Error(st, "df11_build_run_index (device)")
+            raise DF11Error(st, "df11_build_run_index / df11_build_segment_index (device)")
     return DF11Matrix(shape=tuple(shape), n=n, total_bits=total_bits, codebook=codebook,
-                      sizes=sizes, tables=tables, hist=hist, run_index=ri, **bufs)
+                      sizes=sizes, tables=tables, hist=hist, run_index=ri, seg_index=si, **bufs)
 
 
 def serialize(m: DF11Matrix) -> np.ndarray:

@@ -90,6 +90,7 @@ extern "C" df11_status df11_sizes_from_bits(uint64_t n, uint64_t bits, df11_size
   out->tables_bytes = sizeof(DecodeTables);
   out->workspace_bytes = 8 * (ceil_div(n, df11i::kEncTile) + 1) + 16;
   out->run_index_bytes = 2 * (DF11_BLOCK_CHUNKS / 2) * B;
+  out->seg_index_bytes = round_up(4 * (ceil_div(n, DF11_SEGMENT) + 1), 16);
   return DF11_OK;
 }
 

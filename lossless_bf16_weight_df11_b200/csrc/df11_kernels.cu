@@ -615,12 +615,14 @@ struct DecMat {
   const uint32_t *pos;
   const uint8_t *sm;
   const uint16_t *run_index;  // indexed decoder only
+  const uint32_t *seg;        // segment decoder only: the segment index
   const DecodeTables *tables;
   uint16_t *out;
   uint64_t n;
   uint64_t total_bits;
   uint32_t n_chunks;  // C = ceil(total_bits / 64) (< 2^31 for n < 2^32)
   uint32_t n_blocks;  // B = ceil(C / 256); pos holds B + 1 entries
+  uint32_t n_segs;    // segment decoder: S = ceil(n / 64); seg holds S + 1 entries
   // fused matmul only: the matrix is rows x cols (row-major), x holds
   // `batch` rows of cols BF16 activations, y `batch` rows of rows FP32 sums
   uint32_t rows, cols;
@@ -736,8 +738,13 @@ __device__ __forceinline__ bool smem_ok(uint32_t a, uint32_t bytes) {
 #define DF11_GLOBAL_CHECK(cond, on_fail)
 #endif
 
+// (A failed check in the checked build skips the access.  A load then
+// returns a value whose top four bits are set: read as a table entry's
+// control word it consumes 15 bits and decodes nothing, so every decode loop
+// still advances to its end.)
+constexpr uint32_t kCheckFailValue = 0xF0000000u;
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  DF11_SMEM_CHECK(a, 4, return 0u)
+  DF11_SMEM_CHECK(a, 4, return kCheckFailValue)
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
   return v;
@@ -749,7 +756,7 @@ __device__ __forceinline__ uint32_t lds8(uint32_t a) {
   return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t a) {
-  DF11_SMEM_CHECK(a, 8, return make_uint2(0u, 0u))
+  DF11_SMEM_CHECK(a, 8, return make_uint2(0u, kCheckFailValue))
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
   return v;
@@ -1829,9 +1836,18 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_idx_kernel(const __g
 // sum gives each run's first output within the block, and the block's total
 // is checked against its stored positions.
 constexpr int kRiThreads = DF11_BLOCK_CHUNKS / kCPT;  // 128
+constexpr uint32_t kSegOut = DF11_SEGMENT;  // outputs per segment of the segment index
+static_assert(kSegOut == 64, "segment index: code index >> 6 is its segment");
 
+// kSeg = false: the run index (one uint16 per run).  kSeg = true: the
+// segment index instead -- after the count pass and the block's scan each
+// thread knows the output index of its run's first code, and a second pass
+// over the run records the start bit of every code whose index is a
+// multiple of 64 (the start of a segment).
+template <bool kSeg>
 __global__ void __launch_bounds__(kRiThreads) run_index_kernel(const __grid_constant__ DecParams P,
-                                                              uint16_t *__restrict__ out) {
+                                                              uint16_t *__restrict__ out,
+                                                              uint32_t *__restrict__ seg) {
   __shared__ __align__(16) DecodeTables tab;
   __shared__ uint32_t s_warp[kRiThreads / 32];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -1854,23 +1870,24 @@ __global__ void __launch_bounds__(kRiThreads) run_index_kernel(const __grid_cons
     return;
   }
   const bool table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
-  const uint32_t lut_a = smem_addr(&tab);
+  const uint64_t n_segs = (M.n + kSegOut - 1) / kSegOut;
+  if (kSeg && blockIdx.x == 0 && t == 0) seg[n_segs] = (uint32_t)M.total_bits;
   for (uint32_t b = b0; b < b1; ++b) {
     const uint32_t c0 = b * DF11_BLOCK_CHUNKS + kCPT * t;
     uint32_t cnt = 0;
     bool bad = false;
+    uint32_t W0 = 0, W1 = 0, W2 = 0, W3 = 0, W4 = 0, lim = 0, gap = 0;
     if (c0 < M.n_chunks) {
       // the run's 16 stream bytes and the next 4 (inside the stream's
       // allocation: whole blocks plus 16 bytes)
       const uint4 a4 = __ldg(reinterpret_cast<const uint4 *>(M.stream + 8ull * c0));
-      const uint32_t W0 = bswap32(a4.x), W1 = bswap32(a4.y), W2 = bswap32(a4.z),
-                     W3 = bswap32(a4.w),
-                     W4 = bswap32(__ldg(reinterpret_cast<const uint32_t *>(M.stream + 8ull * c0 + 16)));
+      W0 = bswap32(a4.x), W1 = bswap32(a4.y), W2 = bswap32(a4.z), W3 = bswap32(a4.w);
+      W4 = bswap32(__ldg(reinterpret_cast<const uint32_t *>(M.stream + 8ull * c0 + 16)));
       const uint64_t avail = M.total_bits - 64ull * c0;
-      const uint32_t lim = avail < 64u * kCPT ? (uint32_t)avail : 64u * kCPT;
+      lim = avail < 64u * kCPT ? (uint32_t)avail : 64u * kCPT;
       const uint64_t q = (uint64_t)DF11_GAP_BITS * c0;
       const uint32_t two = ((uint32_t)__ldg(M.gaps + (q >> 3)) << 8) | __ldg(M.gaps + (q >> 3) + 1);
-      const uint32_t gap = (two >> (11 - (q & 7u))) & 31u;
+      gap = (two >> (11 - (q & 7u))) & 31u;
       uint32_t p = gap, acc = 0, ctrl = 0;
 #pragma unroll 1
       while (p < lim) {
@@ -1878,7 +1895,7 @@ __global__ void __launch_bounds__(kRiThreads) run_index_kernel(const __grid_cons
         const uint32_t hw = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
         const uint32_t lw = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
         const uint32_t w = __funnelshift_l(lw, hw, p);
-        const uint32_t ey = lds32(lut_a + ((w >> (32 - df11i::kLutBits)) << 3) + 4);
+        const uint32_t ey = tab.lut[w >> (32 - df11i::kLutBits)].y;  // (static shared memory)
         if (!table_short && (ey & df11i::kCtrlLongFlag)) {
           const uint32_t L = long_code_len(w, tab);
           if (L == 0) {
@@ -1919,12 +1936,303 @@ __global__ void __launch_bounds__(kRiThreads) run_index_kernel(const __grid_cons
       tot += s_warp[i];
     }
     const uint32_t excl = pre + incl - cnt;
-    out[(uint64_t)b * kRiThreads + t] = (uint16_t)excl;
-    if (t == 0 && (any_bad || tot != __ldg(M.pos + b + 1) - __ldg(M.pos + b) || tot > 0xFFFFu))
-      set_status(P.status, DF11_ERR_CORRUPT);
+    const uint32_t pb = __ldg(M.pos + b);
+    const bool block_bad = any_bad || tot != __ldg(M.pos + b + 1) - pb || tot > 0xFFFFu;
+    if (!kSeg) out[(uint64_t)b * kRiThreads + t] = (uint16_t)excl;
+    if (t == 0 && block_bad) set_status(P.status, DF11_ERR_CORRUPT);
+    if (kSeg && !block_bad && c0 < M.n_chunks) {
+      // second pass: the codes that start in this run, with their output
+      // indices; a LUT entry holds at most 4 codes, so at most one of them
+      // starts a segment
+      uint64_t i = (uint64_t)pb + excl;
+      uint32_t p = gap;
+#pragma unroll 1
+      while (p < lim) {
+        const uint32_t k = p >> 5;
+        const uint32_t hw = k == 0 ? W0 : k == 1 ? W1 : k == 2 ? W2 : W3;
+        const uint32_t lw = k == 0 ? W1 : k == 1 ? W2 : k == 2 ? W3 : W4;
+        const uint32_t w = __funnelshift_l(lw, hw, p);
+        const uint32_t ey = tab.lut[w >> (32 - df11i::kLutBits)].y;
+        uint32_t nc, adv;
+        if (!table_short && (ey & df11i::kCtrlLongFlag)) {
+          nc = 1u;
+          adv = long_code_len(w, tab);
+          if (adv == 0) break;  // reported by the count pass
+        } else {
+          nc = (ey >> df11i::kCtrlCountShift) & 7u;
+          adv = ey >> df11i::kCtrlUsedShift;
+        }
+        const uint32_t j = (uint32_t)(-i) & (kSegOut - 1);  // first code here at a multiple of 64
+        if (j < nc) {
+          const uint32_t st = j == 0 ? 0u : (ey >> (8 + 4 * j)) & 15u;  // its start in the window
+          if (p + st < lim && ((i + j) >> 6) < n_segs)
+            seg[(i + j) >> 6] = (uint32_t)(64ull * c0) + p + st;
+        }
+        i += nc;
+        p += adv;
+      }
+    }
     __syncthreads();  // s_warp is reused by the next block
   }
 }
+
+// ============================================================ segment decoder
+//
+// With the segment index (the stream bit at which every 64th code starts),
+// each lane of a warp decodes one segment -- exactly 64 codes, or the
+// matrix's last few -- into its own exponent row, checks that it ended
+// where the next segment begins, and merges the row with the segment's
+// sign/mantissa bytes into 128 bytes of BF16.  A warp takes a unit of 32
+// consecutive segments (2048 outputs): their stream bits are one contiguous
+// range, copied into the warp's shared memory (cp.async) while the warp
+// decodes the unit before; the unit's sign/mantissa bytes are copied while
+// it decodes.  Nothing is counted, scanned or relocated, and the warps of a
+// CTA meet only when the CTA moves on to another matrix (its tables).
+constexpr uint32_t kSegWarps = 32;
+constexpr uint32_t kSegThreads = 32 * kSegWarps;
+constexpr uint32_t kSegUnit = 32 * kSegOut;          // outputs per warp unit
+constexpr uint32_t kSegRowWords = kSegOut / 4 + 1;   // exponent words per lane, + 1 spare
+constexpr uint32_t kSegStage = 1024;                 // stream bytes per stage
+constexpr uint32_t kSegWarpBytes = 128 * kSegRowWords + kSegUnit + 2 * kSegStage;
+constexpr uint32_t kSegSmem = kTablesSmem + kSegWarps * kSegWarpBytes;
+static_assert(kSegWarpBytes % 16 == 0, "segment decoder layout");
+
+__device__ __forceinline__ void seg_cp16(uint32_t dst, const void *src) {
+  DF11_SMEM_CHECK(dst, 16, return)
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void seg_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void seg_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void seg_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+#define DF11_LUT_ADDR(w) madlo(madhi((w), 1u << df11i::kLutBits, 0u), 8u, lut_a)
+
+// Append `add` bits (whole exponent bytes, low byte first) of xs at bit nb of
+// the lane's exponent row (word w at row_a + row_stride * w); the word being
+// filled is kept in cur and stored whole at every step.
+#define DF11_SEG_APPEND(xs, add)                                            \
+  {                                                                         \
+    const uint32_t lo4 = cur | __funnelshift_l(0u, (xs), nb);               \
+    const uint32_t hi4 = __funnelshift_l((xs), 0u, nb);                     \
+    sts32(row_a + (nb >> 5) * row_stride, lo4);                             \
+    const uint32_t nb2 = nb + (add);                                        \
+    cur = ((nb ^ nb2) & 32u) ? hi4 : lo4;                                   \
+    nb = nb2;                                                               \
+  }
+
+// Advance the window to bit pn; a step moves at most 32 bits, so at most one
+// word boundary is crossed.
+#define DF11_SEG_ADVANCE(pn)                                                \
+  {                                                                         \
+    if (((pn) >> 5) != (p >> 5)) {                                          \
+      hw = lw;                                                              \
+      lw = nxt;                                                             \
+      nxt = word(((pn) >> 5) + 2u);                                         \
+    }                                                                       \
+    p = (pn);                                                               \
+  }
+
+// One lane's segment: cnt (<= 64) codes from stream bit p (relative to the
+// words word(k) returns, byte-swapped to MSB-first), exponents into the
+// lane's row.  True when exactly cnt codes were decoded and the last one
+// ended at pend (where the next segment starts).
+template <class WordFn>
+__device__ __forceinline__ bool seg_decode_lane(uint32_t p, uint32_t pend, uint32_t cnt,
+                                                bool table_short, const DecodeTables &tab,
+                                                uint32_t lut_a, uint32_t row_a, uint32_t row_stride,
+                                                WordFn word) {
+  uint32_t hw = word(p >> 5), lw = word((p >> 5) + 1u), nxt = word((p >> 5) + 2u);
+  uint32_t nb = 0, cur = 0;
+  const uint32_t nb_end = 8u * cnt;
+  if (table_short) {
+    // whole table entries while at least 4 codes remain
+    const int32_t nb_fast = 8 * ((int32_t)cnt - 4);
+#pragma unroll 1
+    while ((int32_t)nb <= nb_fast && p < pend) {
+      const uint32_t w = __funnelshift_l(lw, hw, p);
+      const uint2 en = lds64(DF11_LUT_ADDR(w));
+      DF11_SEG_APPEND(en.x, en.y & 0x38u)
+      const uint32_t pn = madhi(en.y, 1u << (32 - df11i::kCtrlUsedShift), p);
+      DF11_SEG_ADVANCE(pn)
+    }
+  }
+  // the last codes (and codes longer than the table's reach): keep only as
+  // many of an entry's codes as remain
+#pragma unroll 1
+  while (nb < nb_end && p < pend) {
+    const uint32_t w = __funnelshift_l(lw, hw, p);
+    const uint2 en = lds64(DF11_LUT_ADDR(w));
+    uint32_t adv;
+    if (!table_short && (en.y & df11i::kCtrlLongFlag)) {
+      const uint32_t L = long_code_len(w, tab);
+      if (L == 0) break;  // no code: reported (nb short of nb_end)
+      const uint32_t x = tab.sym[((w >> (32 - L)) + tab.base[L]) & 0xFFu];
+      DF11_SEG_APPEND(x, 8u)
+      adv = L;
+    } else {
+      const uint32_t nc = (en.y >> df11i::kCtrlCountShift) & 7u;
+      const uint32_t keep = min(nc, (nb_end - nb) >> 3);
+      const uint32_t mask = keep >= 4u ? 0xFFFFFFFFu : ((1u << (8u * keep)) - 1u);
+      DF11_SEG_APPEND(en.x & mask, 8u * keep)
+      adv = keep < nc ? (en.y >> (8u + 4u * keep)) & 15u : en.y >> df11i::kCtrlUsedShift;
+    }
+    const uint32_t pn = p + adv;
+    DF11_SEG_ADVANCE(pn)
+  }
+  sts32(row_a + (nb >> 5) * row_stride, cur);  // the word being filled
+  return nb == nb_end && p == pend;
+}
+
+__global__ void __launch_bounds__(kSegThreads, 1) decode_seg_kernel(const __grid_constant__ DecParams P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+  const uint32_t sbase = smem_addr(smem);
+  const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem);
+  const uint32_t lut_a = sbase;  // lut is the first member of the tables
+  const uint32_t wb = sbase + kTablesSmem + warp * kSegWarpBytes;
+  const uint32_t row_a = wb + 4u * lane;                // exponent word w: row_a + 128 w
+  const uint32_t sm_a = wb + 128u * kSegRowWords;       // sign/mantissa piece q of lane l:
+                                                        // sm_a + 16 (32 q + l)
+  const uint32_t stage_a = sm_a + kSegUnit;             // stream stages 0 and 1
+
+  const uint64_t total = P.unit_start[P.count];
+  const uint64_t g0 = (uint64_t)blockIdx.x * total / gridDim.x;
+  const uint64_t g1 = (uint64_t)(blockIdx.x + 1) * total / gridDim.x;
+  if (g0 >= g1) return;  // the same for every thread of the CTA
+#ifdef DF11_CHECKED
+  if (threadIdx.x == 0) s_check_status = P.status;
+  __syncthreads();
+#endif
+  uint32_t m = 0;
+  while (m + 1 < P.count && g0 >= P.unit_start[m + 1]) ++m;
+  for (; m < P.count && P.unit_start[m] < g1; ++m) {
+    const uint64_t s0 = max(g0, P.unit_start[m]), s1 = min(g1, P.unit_start[m + 1]);
+    __syncthreads();  // every warp is done with the previous matrix's tables
+    if (s0 >= s1) continue;
+    const DecMat &M = P.m[m];
+    {
+      const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
+      uint4 *dst = reinterpret_cast<uint4 *>(smem);
+      for (uint32_t k = threadIdx.x; k < sizeof(DecodeTables) / 16; k += blockDim.x)
+        dst[k] = __ldg(src + k);
+    }
+    __syncthreads();
+    bool tbad = false;
+    for (uint32_t k = threadIdx.x; k < (uint32_t)df11i::kLutSize; k += blockDim.x)
+      tbad |= lut_entry_bad(tab.lut[k].y, P.min_len);
+    const bool table_ok = !__syncthreads_or(tbad);
+    const bool table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
+
+    const uint64_t ubase = P.unit_start[m];
+    const uint64_t first = s0 + warp;
+    if (first >= s1) continue;
+    const uint32_t S = M.n_segs;
+    const uint64_t alloc = 2048ull * M.n_blocks + 16;  // the stream's allocation (bytes)
+    // this lane's segment start and the unit's end (the next unit's first
+    // segment start, or total_bits), as absolute stream bits
+    auto bounds = [&](uint64_t g, uint32_t &a, uint32_t &E) {
+      const uint64_t j0 = (uint64_t)kSegWarps * (g - ubase);
+      a = __ldg(M.seg + min(j0 + lane, (uint64_t)S));
+      E = __ldg(M.seg + min(j0 + 32, (uint64_t)S));
+    };
+    // the unit's stream bytes [lo, hi) into a stage, when they fit; staged
+    // is false otherwise (the unit then reads the stream from global memory)
+    auto stage_in = [&](uint32_t a, uint32_t E, uint32_t st, uint32_t &lo, bool &staged) {
+      const uint32_t a0 = __shfl_sync(0xffffffffu, a, 0);
+      const bool sane = a0 <= E && E <= M.total_bits;
+      lo = sane ? (a0 >> 3) & ~15u : 0u;
+      const uint64_t hi = min((uint64_t)((4ull * ((E >> 5) + 3u) + 15u) & ~15ull), alloc);
+      const uint32_t size = sane && hi > lo ? (uint32_t)(hi - lo) : 0u;
+      staged = size <= kSegStage;
+      if (staged)
+        for (uint32_t q = lane; 16u * q < size; q += 32u) seg_cp16(st + 16u * q, M.stream + lo + 16u * q);
+    };
+
+    uint64_t g = first;
+    uint32_t a, E, lo;
+    bool staged;
+    bounds(g, a, E);
+    stage_in(a, E, stage_a, lo, staged);
+    seg_commit();
+    uint32_t an = 0, En = 0;
+    if (g + kSegWarps < s1) bounds(g + kSegWarps, an, En);
+    for (uint32_t it = 0; g < s1; g += kSegWarps, ++it) {
+      const uint64_t j = (uint64_t)kSegWarps * (g - ubase) + lane;  // this lane's segment
+      const uint32_t cnt = j < S ? (uint32_t)min((uint64_t)kSegOut, M.n - kSegOut * j) : 0u;
+      // this unit's sign/mantissa bytes and the next unit's stream
+      for (uint32_t q = 0; q < 4u; ++q)
+        if (16u * q < cnt) seg_cp16(sm_a + 16u * (32u * q + lane), M.sm + kSegOut * j + 16u * q);
+      uint32_t lo_n = 0;
+      bool staged_n = true;
+      if (g + kSegWarps < s1) stage_in(an, En, stage_a + kSegStage * ((it + 1) & 1u), lo_n, staged_n);
+      seg_commit();
+      uint32_t an2 = 0, En2 = 0;
+      if (g + 2 * kSegWarps < s1) bounds(g + 2 * kSegWarps, an2, En2);
+      seg_wait_prev();  // this unit's stream
+      __syncwarp();
+
+      // ---- decode this lane's segment into its exponent row
+      const uint32_t st = stage_a + kSegStage * (it & 1u);
+      const uint32_t a_next = __shfl_down_sync(0xffffffffu, a, 1);  // every lane takes part
+      const uint32_t e = lane < 31u ? a_next : E;
+      const uint32_t lo_bits = 8u * lo;
+      const uint64_t gl_words = (alloc - lo) / 4;  // global words from lo (lo < alloc)
+      const uint32_t *gsrc = reinterpret_cast<const uint32_t *>(M.stream + lo);
+      auto word = [&](uint32_t k) -> uint32_t {
+        return bswap32(staged ? lds32(st + 4u * min(k, kSegStage / 4 - 1))
+                              : __ldg(gsrc + min((uint64_t)k, gl_words - 1)));
+      };
+      bool ok = table_ok && a >= lo_bits && a <= e && e <= M.total_bits &&
+                e - a <= (uint64_t)DF11_MAX_CODE_LEN * cnt;
+      if (cnt && ok)
+        ok = seg_decode_lane(a - lo_bits, e - lo_bits, cnt, table_short, tab, lut_a, row_a, 128u,
+                             word);
+      if (__ballot_sync(0xffffffffu, cnt && !ok) && lane == 0) set_status(P.status, DF11_ERR_CORRUPT);
+
+      // ---- merge: exponents + sign/mantissa -> BF16, 16 outputs at a time
+      seg_wait_all();  // this unit's sign/mantissa bytes (and the next unit's stream)
+      if (cnt && ok) {
+        uint16_t *o = M.out + kSegOut * j;
+#pragma unroll
+        for (uint32_t q = 0; q < 4u; ++q) {
+          if (16u * q < cnt) {
+            const uint4 sv = lds128(sm_a + 16u * (32u * q + lane));
+            const uint32_t e0 = lds32(row_a + 128u * (4u * q)), e1 = lds32(row_a + 128u * (4u * q + 1u)),
+                           e2 = lds32(row_a + 128u * (4u * q + 2u)),
+                           e3 = lds32(row_a + 128u * (4u * q + 3u));
+            uint4 r0, r1;
+            merge4(e0, sv.x, r0.x, r0.y);
+            merge4(e1, sv.y, r0.z, r0.w);
+            merge4(e2, sv.z, r1.x, r1.y);
+            merge4(e3, sv.w, r1.z, r1.w);
+            if (16u * q + 16u <= cnt) {
+              DF11_GLOBAL_CHECK(kSegOut * j + 16u * q + 16u <= M.n, continue)
+              reinterpret_cast<uint4 *>(o + 16u * q)[0] = r0;
+              reinterpret_cast<uint4 *>(o + 16u * q)[1] = r1;
+            } else {
+              const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+              for (uint32_t i = 0; i < 16u; ++i)
+                if (16u * q + i < cnt) o[16u * q + i] = (uint16_t)(wv[i >> 1] >> (16u * (i & 1u)));
+            }
+          }
+        }
+      }
+      __syncwarp();  // the stage and the sign/mantissa pieces are refilled next
+      a = an;
+      E = En;
+      lo = lo_n;
+      staged = staged_n;
+      an = an2;
+      En = En2;
+    }
+    seg_wait_all();
+  }
+}
+
+#undef DF11_SEG_APPEND
+#undef DF11_SEG_ADVANCE
+#undef DF11_LUT_ADDR
 
 // ============================================================ launch helpers
 
@@ -1987,6 +2295,10 @@ df11_status device_info(int *dev, int *sms, int *smem_optin = nullptr) {
           return DF11_ERR_CUDA;
     if (cudaFuncSetAttribute(decode_idx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              d.smem_optin) != cudaSuccess)
+      return DF11_ERR_CUDA;
+    if (d.smem_optin >= (int)kSegSmem &&
+        cudaFuncSetAttribute(decode_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSegSmem) != cudaSuccess)
       return DF11_ERR_CUDA;
     d.configured = true;
   }
@@ -2166,6 +2478,7 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
     uint32_t min_len = DF11_MAX_CODE_LEN;
     uint32_t unit_codes = 0;  // staging size: most codes in one unit of the batch
     bool indexed = io == nullptr;  // every matrix has a run index (plain decode only)
+    bool segmented = io == nullptr;  // every matrix has a segment index (plain decode only)
     for (uint32_t i = 0; i < k; ++i) {
       const df11_matrix &m = ms[first + i];
       if (m.n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
@@ -2173,9 +2486,11 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
       if (!m.stream || !m.gaps || !m.block_pos || !m.sign_mantissa || !m.tables)
         return DF11_ERR_INVALID_ARG;
       if (!aligned16(m.stream) || !aligned16(m.gaps) || !aligned16(m.sign_mantissa) ||
-          !aligned16(m.tables) || ((uintptr_t)m.block_pos & 3u) || !aligned16(m.run_index))
+          !aligned16(m.tables) || ((uintptr_t)m.block_pos & 3u) || !aligned16(m.run_index) ||
+          ((uintptr_t)m.seg_index & 3u))
         return DF11_ERR_INVALID_ARG;
       indexed = indexed && m.run_index != nullptr;
+      segmented = segmented && m.seg_index != nullptr && m.total_bits <= 0xFFFFFFFFull;
       if (io) {
         // the matrix is rows x cols; activations and sums 16-byte aligned
         const df11_matmul_io &q = io[first + i];
@@ -2206,6 +2521,8 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
       d.sm = m.sign_mantissa;
       d.tables = reinterpret_cast<const DecodeTables *>(m.tables);
       d.run_index = m.run_index;
+      d.seg = m.seg_index;
+      d.n_segs = (uint32_t)cdiv(m.n, kSegOut);
       d.out = io ? nullptr : d_outs[first + i];
       d.rows = io ? io[first + i].rows : 0u;
       d.cols = io ? io[first + i].cols : 1u;
@@ -2220,6 +2537,21 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
       ++P.count;
     }
     if (P.count == 0) continue;
+    if (segmented && smem_optin >= (int)kSegSmem) {
+      // the segment decoder: units of 32 segments, one CTA of 32 warps per SM
+      for (uint32_t i = 0; i < P.count; ++i)
+        P.unit_start[i + 1] = P.unit_start[i] + cdiv(P.m[i].n_segs, kSegWarps);
+      for (uint32_t i = P.count + 1; i <= DF11_MAX_BATCH; ++i) P.unit_start[i] = P.unit_start[P.count];
+      P.min_len = min_len;
+      P.stage_cap = 0;
+      P.batch = 0;
+      const uint64_t units = P.unit_start[P.count];
+      const uint64_t grid = std::min<uint64_t>(cdiv(units, kSegWarps), (uint64_t)sms);
+      decode_seg_kernel<<<(unsigned)grid, kSegThreads, kSegSmem, s>>>(P);
+      st = launch_status();
+      if (st != DF11_OK) return st;
+      continue;
+    }
     for (uint32_t i = P.count + 1; i <= DF11_MAX_BATCH; ++i) P.unit_start[i] = P.unit_start[P.count];
     P.stage_cap = (unit_codes + 15u) & ~15u;
     P.min_len = min_len;
@@ -2303,8 +2635,50 @@ extern "C" df11_status df11_build_run_index(const df11_matrix *m, uint16_t *d_ru
   P.min_len = m->min_len;
   P.status = d_status;
   const uint64_t grid = std::min<uint64_t>(B, (uint64_t)sms * 8);
-  run_index_kernel<<<(unsigned)grid, kRiThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      P, d_run_index);
+  run_index_kernel<false><<<(unsigned)grid, kRiThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      P, d_run_index, nullptr);
+  return launch_status();
+}
+
+extern "C" df11_status df11_build_segment_index(const df11_matrix *m, uint32_t *d_seg_index,
+                                                uint32_t *d_status, df11_stream_t stream) {
+  if (!m || !d_status) return DF11_ERR_INVALID_ARG;
+  if (m->n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
+  if (!d_seg_index || ((uintptr_t)d_seg_index & 3u)) return DF11_ERR_INVALID_ARG;
+  if (m->total_bits > 0xFFFFFFFFull) return DF11_ERR_TOO_LARGE;
+  if (m->n == 0) {
+    // one entry: total_bits (0)
+    return cudaMemsetAsync(d_seg_index, 0, 4, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DF11_OK
+               : DF11_ERR_CUDA;
+  }
+  if (!m->stream || !m->gaps || !m->block_pos || !m->tables || !aligned16(m->stream) ||
+      !aligned16(m->tables) || ((uintptr_t)m->block_pos & 3u))
+    return DF11_ERR_INVALID_ARG;
+  if (m->min_len < 1 || m->min_len > 8) return DF11_ERR_INVALID_ARG;
+  if (m->total_bits < m->n * (uint64_t)m->min_len || m->total_bits > m->n * 32ull)
+    return DF11_ERR_INVALID_ARG;
+  int dev, sms;
+  df11_status st = device_info(&dev, &sms);
+  if (st != DF11_OK) return st;
+  const uint64_t C = cdiv(m->total_bits, 64);
+  const uint64_t B = cdiv(C, DF11_BLOCK_CHUNKS);
+  DecParams P{};
+  DecMat &d = P.m[0];
+  d.stream = m->stream;
+  d.gaps = m->gaps;
+  d.pos = m->block_pos;
+  d.tables = reinterpret_cast<const DecodeTables *>(m->tables);
+  d.n = m->n;
+  d.total_bits = m->total_bits;
+  d.n_chunks = (uint32_t)C;
+  d.n_blocks = (uint32_t)B;
+  P.count = 1;
+  P.min_len = m->min_len;
+  P.status = d_status;
+  const uint64_t grid = std::min<uint64_t>(B, (uint64_t)sms * 8);
+  run_index_kernel<true><<<(unsigned)grid, kRiThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      P, nullptr, d_seg_index);
   return launch_status();
 }
 
@@ -2318,7 +2692,10 @@ extern "C" df11_status df11_test_decode_starved(const df11_matrix *m, uint16_t *
                                                 uint32_t *d_status, df11_stream_t stream) {
   if (!m || !d_out) return DF11_ERR_INVALID_ARG;
   uint16_t *outs[1] = {d_out};
-  return launch_decode(m, 1, outs, nullptr, 0, d_status, stream, 16u);
+  // the decoders with bulk-copy barriers (the segment decoder has none)
+  df11_matrix mm = *m;
+  mm.seg_index = nullptr;
+  return launch_decode(&mm, 1, outs, nullptr, 0, d_status, stream, 16u);
 }
 #endif
 
@@ -2387,4 +2764,349 @@ extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
   // written earlier in the same call
   return launch_encode(d_w, n, ecb, nullptr, total_bits, out, ws, d_status,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ============================================================ fused decode -> tensor-core GEMM
+//
+// y[j][r] += sum_c W[r][c] x[j][c] for up to 256 activation rows at a time,
+// with W decoded through its segment index straight into the B operand of
+// tcgen05.mma and never written to device memory.  A CTA owns 128 rows of W
+// (the MMA's N) and walks its columns in steps of 64: row r's columns
+// [64k, 64k + 64) are exactly segment r * cols / 64 + k of the segment index,
+// so decode lane t (four warps) decodes that segment and writes its 64 BF16
+// weights as row t of the step's B tile (K-major, 128-byte rows, 128-byte
+// swizzle).  The same lanes copy the step's activation tiles (cp.async,
+// zero-filled past the batch) as A.  A fifth warp issues, per step and per
+// 128-row M tile, four 128 x 128 x 16 MMAs accumulating in TMEM and commits
+// them to the stage's "empty" barrier; after the last step the decode warps
+// read the accumulators out of TMEM and add them to y.  Every wait is bounded.
+namespace {
+
+constexpr uint32_t kGemmN = 128;        // W rows per CTA (MMA N)
+constexpr uint32_t kGemmM = 128;        // activation rows per M tile (MMA M)
+constexpr uint32_t kGemmK = kSegOut;    // columns per step: one segment per row
+constexpr uint32_t kGemmStages = 2;
+constexpr uint32_t kGemmLanes = 128;    // decode lanes: one per W row of the tile
+constexpr uint32_t kGemmThreads = kGemmLanes + 32;
+constexpr uint32_t kGemmTile = kGemmN * kGemmK * 2;  // 16 KiB: a B tile, or one A tile
+constexpr uint32_t kGemmMaxMT = DF11_GEMM_MAX_BATCH / kGemmM;
+static_assert(kGemmN == kGemmM && kGemmK * 2 == 128, "one 128-byte swizzle row per tile row");
+
+struct GemmParams {
+  DecMat m[DF11_MAX_BATCH];
+  uint32_t tile_start[DF11_MAX_BATCH + 1];  // prefix sums of N tiles per matrix
+  uint32_t count;
+  uint32_t batch;  // activation rows of this launch (<= 128 * mt)
+  uint32_t mt;     // M tiles: 1 or 2
+  uint32_t min_len;
+  uint32_t *status;
+};
+
+__host__ __device__ constexpr uint32_t gemm_stage_bytes(uint32_t mt) { return (1 + mt) * kGemmTile; }
+__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t mt) {
+  // stages, tables, exponent rows, sign/mantissa pieces, barriers and the
+  // TMEM address, plus 1 KiB to align the stages to the swizzle atom
+  return kGemmStages * gemm_stage_bytes(mt) + kTablesSmem + 4 * kSegRowWords * kGemmLanes +
+         kGemmK * kGemmLanes + 64 + 1024;
+}
+
+// Shared-memory operand descriptor: K-major, 128-byte swizzle, rows of 128
+// bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu)  // start address
+         | ((uint64_t)1 << 16)               // leading byte offset (unused with swizzle)
+         | ((uint64_t)(1024 >> 4) << 32)     // stride byte offset: 8 rows
+         | ((uint64_t)1 << 46)               // descriptor version
+         | ((uint64_t)2 << 61);              // 128-byte swizzle
+}
+
+// Instruction descriptor: BF16 A and B (both K-major), FP32 accumulator,
+// M = 128, N = 128.
+constexpr uint32_t kGemmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kGemmN >> 3) << 17) |
+                                ((kGemmM >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kGemmIdesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void gemm_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp16_zfill(uint32_t dst, const void *src, uint32_t bytes) {
+  DF11_SMEM_CHECK(dst, 16, return)
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const __grid_constant__ GemmParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  const uint32_t MT = P.mt;
+  const uint32_t stage_bytes = gemm_stage_bytes(MT);
+  const uint32_t tab_off = kGemmStages * stage_bytes;
+  const uint32_t rows_off = tab_off + kTablesSmem;
+  const uint32_t smp_off = rows_off + 4 * kSegRowWords * kGemmLanes;
+  const uint32_t bar_off = smp_off + kGemmK * kGemmLanes;
+  const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem + tab_off);
+  const uint32_t lut_a = base + tab_off;
+  const uint32_t bar_full = base + bar_off;                  // per stage: decode lanes arrived
+  const uint32_t bar_empty = bar_full + 8 * kGemmStages;     // per stage: its MMAs completed
+  const uint32_t bar_done = bar_empty + 8 * kGemmStages;     // every MMA completed
+  uint32_t *slot = reinterpret_cast<uint32_t *>(smem + bar_off + 8 * (2 * kGemmStages + 1));
+  const uint32_t t = threadIdx.x, warp = t >> 5, lane = t & 31u;
+#ifdef DF11_CHECKED
+  if (t == 0) s_check_status = P.status;
+  __syncthreads();
+#endif
+
+  uint32_t mi = 0;
+  while (mi + 1 < P.count && blockIdx.x >= P.tile_start[mi + 1]) ++mi;
+  const DecMat &M = P.m[mi];
+  const uint32_t n0 = (blockIdx.x - P.tile_start[mi]) * kGemmN;
+  const uint32_t ksteps = M.cols / kGemmK;
+
+  {
+    const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
+    uint4 *dst = reinterpret_cast<uint4 *>(smem + tab_off);
+    for (uint32_t k = t; k < sizeof(DecodeTables) / 16; k += blockDim.x) dst[k] = __ldg(src + k);
+  }
+  if (t == 0) {
+    for (uint32_t s = 0; s < kGemmStages; ++s) {
+      mbar_init(bar_full + 8 * s, kGemmLanes);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_done, 1);
+    slot[1] = 0u;  // set when a bounded wait runs out
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 4) {
+    // kGemmM * MT columns of FP32 accumulators (a power of two >= 32)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     base + bar_off + 8 * (2 * kGemmStages + 1)),
+                 "r"(kGemmN * MT)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  bool tbad = false;
+  for (uint32_t k = t; k < (uint32_t)df11i::kLutSize; k += blockDim.x)
+    tbad |= lut_entry_bad(tab.lut[k].y, P.min_len);
+  tc_fence_before();
+  const bool table_ok = !__syncthreads_or(tbad);
+  tc_fence_after();
+  const bool table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(slot);
+  volatile uint32_t *gave_up = slot + 1;
+
+  if (warp < 4) {
+    // ---- decode lane t: row n0 + t of W, one segment per step
+    const uint32_t r = n0 + t;
+    const bool row_ok = r < M.rows;
+    const uint64_t seg0 = (uint64_t)r * ksteps;  // segment of (row r, step 0)
+    const uint32_t *sw = reinterpret_cast<const uint32_t *>(M.stream);
+    const uint64_t last_w = (2048ull * M.n_blocks + 16) / 4 - 1;
+    auto word = [&](uint32_t k) -> uint32_t { return bswap32(__ldg(sw + min((uint64_t)k, last_w))); };
+    const uint32_t row_a = base + rows_off + 4 * t;  // exponent word w: row_a + 512 w
+    const uint32_t smp = base + smp_off;
+    uint32_t a = row_ok ? __ldg(M.seg + seg0) : 0u;
+    bool bad = !table_ok;
+    for (uint32_t k = 0; k < ksteps; ++k) {
+      const uint32_t s = k % kGemmStages, use = k / kGemmStages;
+      // the stage is free once the MMAs of step k - kGemmStages completed
+      if (k >= kGemmStages && !mbar_wait(bar_empty + 8 * s, (use - 1) & 1u)) {
+        *gave_up = 1u;
+        break;
+      }
+      const uint32_t st = base + s * stage_bytes;
+      // the step's activation tiles: row m, 16-byte chunk c at chunk c ^ (m & 7)
+      for (uint32_t i = t; i < MT * kGemmM * 8; i += kGemmLanes) {
+        const uint32_t mm = i >> 3, c = i & 7u;
+        const bool in = mm < P.batch;
+        const uint16_t *src = in ? M.x + (uint64_t)mm * M.cols + kGemmK * k + 8 * c : M.x;
+        cp16_zfill(st + kGemmTile * (1 + mm / kGemmM) + (mm % kGemmM) * 128 + ((c ^ (mm & 7u)) << 4),
+                   src, in ? 16u : 0u);
+      }
+      // this row's 64 sign/mantissa bytes: piece q at smp + 16 (128 q + t)
+      if (row_ok)
+        for (uint32_t q = 0; q < 4u; ++q)
+          seg_cp16(smp + 16u * (kGemmLanes * q + t), M.sm + (seg0 + k) * kGemmK + 16u * q);
+      seg_commit();
+      const uint32_t e = row_ok ? __ldg(M.seg + seg0 + k + 1) : 0u;
+      bool ok = row_ok && table_ok && a <= e && e <= M.total_bits &&
+                e - a <= (uint32_t)DF11_MAX_CODE_LEN * kGemmK;
+      if (ok) ok = seg_decode_lane(a, e, kGemmK, table_short, tab, lut_a, row_a, 4u * kGemmLanes, word);
+      bad |= row_ok && !ok;
+      seg_wait_all();
+      // row t of the B tile: 16-byte chunk c at chunk c ^ (t & 7)
+      const uint32_t brow = st + 128u * t;
+#pragma unroll
+      for (uint32_t q = 0; q < 4u; ++q) {
+        uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0;
+        if (ok) {
+          const uint4 sv = lds128(smp + 16u * (kGemmLanes * q + t));
+          const uint32_t stride = 4u * kGemmLanes;
+          merge4(lds32(row_a + stride * (4u * q)), sv.x, r0.x, r0.y);
+          merge4(lds32(row_a + stride * (4u * q + 1u)), sv.y, r0.z, r0.w);
+          merge4(lds32(row_a + stride * (4u * q + 2u)), sv.z, r1.x, r1.y);
+          merge4(lds32(row_a + stride * (4u * q + 3u)), sv.w, r1.z, r1.w);
+        }
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(brow + (((2u * q) ^ (t & 7u)) << 4)),
+                     "r"(r0.x), "r"(r0.y), "r"(r0.z), "r"(r0.w)
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(brow + (((2u * q + 1u) ^ (t & 7u)) << 4)),
+                     "r"(r1.x), "r"(r1.y), "r"(r1.z), "r"(r1.w)
+                     : "memory");
+      }
+      // the tiles, written through the generic proxy, are read by the MMA
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      gemm_arrive(bar_full + 8 * s);
+      a = e;
+    }
+    if (bad) set_status(P.status, DF11_ERR_CORRUPT);
+  } else if (lane == 0) {
+    // ---- the MMA issuer
+    for (uint32_t k = 0; k < ksteps; ++k) {
+      const uint32_t s = k % kGemmStages, use = k / kGemmStages;
+      if (!mbar_wait(bar_full + 8 * s, use & 1u)) {
+        *gave_up = 1u;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t st = base + s * stage_bytes;
+      for (uint32_t mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (uint32_t kk = 0; kk < kGemmK / 16; ++kk)
+          umma_bf16(tmem + kGemmN * mt, umma_desc_sw128(st + kGemmTile * (1 + mt) + 32u * kk),
+                    umma_desc_sw128(st + 32u * kk), (k | kk) != 0u);
+      umma_commit(bar_empty + 8 * s);
+    }
+    umma_commit(bar_done);  // arrives once every MMA issued above has completed
+  }
+
+  // ---- epilogue: the accumulators (lane = activation row) added to y
+  const bool done = mbar_wait(bar_done, 0);
+  if (!done) *gave_up = 1u;
+  tc_fence_after();
+  __syncthreads();
+  const bool fail = *gave_up != 0u;
+  if (t == 0 && fail) set_status(P.status, DF11_ERR_TIMEOUT);
+  if (warp < 4 && !fail) {  // (fail is the same for every thread: read after the barrier)
+    for (uint32_t mt = 0; mt < MT; ++mt) {
+      const uint32_t j = kGemmM * mt + 32u * warp + lane;  // activation row
+#pragma unroll 1
+      for (uint32_t c = 0; c < kGemmN; c += 16) {
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+            "%11, %12, %13, %14, %15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+              "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+              "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(tmem + ((32u * warp) << 16) + kGemmN * mt + c));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (j < P.batch) {
+          float *yr = M.y + (uint64_t)j * M.rows + n0 + c;
+#pragma unroll
+          for (uint32_t i = 0; i < 16; ++i)
+            if (n0 + c + i < M.rows) yr[i] += __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGemmN * MT)
+                 : "memory");
+  }
+}
+
+}  // namespace
+
+extern "C" df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_matmul_io *io,
+                                              uint32_t count, uint32_t batch, uint32_t *d_status,
+                                              df11_stream_t stream) {
+  if (count == 0) return DF11_OK;
+  if (!ms || !io || !d_status || batch < 1) return DF11_ERR_INVALID_ARG;
+  int dev, sms, smem_optin;
+  df11_status st = device_info(&dev, &sms, &smem_optin);
+  if (st != DF11_OK) return st;
+  static bool configured[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!configured[dev]) {
+      if (smem_optin < (int)gemm_smem_bytes(kGemmMaxMT)) return DF11_ERR_INVALID_ARG;
+      if (cudaFuncSetAttribute(decode_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)gemm_smem_bytes(kGemmMaxMT)) != cudaSuccess)
+        return DF11_ERR_CUDA;
+      configured[dev] = true;
+    }
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // batches above DF11_GEMM_MAX_BATCH rows: one pass per 256 rows (W decoded again)
+  for (uint32_t j0 = 0; j0 < batch; j0 += DF11_GEMM_MAX_BATCH) {
+    const uint32_t nb = std::min<uint32_t>(DF11_GEMM_MAX_BATCH, batch - j0);
+    for (uint32_t first = 0; first < count; first += DF11_MAX_BATCH) {
+      const uint32_t k = std::min<uint32_t>(DF11_MAX_BATCH, count - first);
+      GemmParams P{};
+      P.status = d_status;
+      P.batch = nb;
+      P.mt = (nb + kGemmM - 1) / kGemmM;
+      P.min_len = DF11_MAX_CODE_LEN;
+      for (uint32_t i = 0; i < k; ++i) {
+        const df11_matrix &m = ms[first + i];
+        const df11_matmul_io &q = io[first + i];
+        if (m.n == 0) continue;
+        if (m.n > DF11_MAX_N || m.total_bits > 0xFFFFFFFFull) return DF11_ERR_TOO_LARGE;
+        if (!m.stream || !m.sign_mantissa || !m.tables || !m.seg_index || !aligned16(m.stream) ||
+            !aligned16(m.sign_mantissa) || !aligned16(m.tables) || ((uintptr_t)m.seg_index & 3u))
+          return DF11_ERR_INVALID_ARG;
+        if (m.min_len < 1 || m.min_len > 8 || m.total_bits < m.n * (uint64_t)m.min_len ||
+            m.total_bits > m.n * 32ull)
+          return DF11_ERR_INVALID_ARG;
+        if ((uint64_t)q.rows * q.cols != m.n || q.cols % kGemmK || !q.x || !q.y ||
+            !aligned16(q.x) || ((uintptr_t)q.y & 3u))
+          return DF11_ERR_INVALID_ARG;
+        DecMat &d = P.m[P.count];
+        d.stream = m.stream;
+        d.sm = m.sign_mantissa;
+        d.seg = m.seg_index;
+        d.tables = reinterpret_cast<const DecodeTables *>(m.tables);
+        d.n = m.n;
+        d.total_bits = m.total_bits;
+        d.n_blocks = (uint32_t)cdiv(cdiv(m.total_bits, 64), DF11_BLOCK_CHUNKS);
+        d.n_segs = (uint32_t)cdiv(m.n, kSegOut);
+        d.rows = q.rows;
+        d.cols = q.cols;
+        d.x = q.x + (uint64_t)j0 * q.cols;
+        d.y = q.y + (uint64_t)j0 * q.rows;
+        P.tile_start[P.count + 1] = P.tile_start[P.count] + (uint32_t)cdiv(q.rows, kGemmN);
+        P.min_len = std::min(P.min_len, m.min_len);
+        ++P.count;
+      }
+      if (P.count == 0) continue;
+      const uint32_t tiles = P.tile_start[P.count];
+      decode_gemm_tc_kernel<<<tiles, kGemmThreads, gemm_smem_bytes(P.mt), s>>>(P);
+      st = launch_status();
+      if (st != DF11_OK) return st;
+    }
+  }
+  return DF11_OK;
 }

@@ -5,8 +5,10 @@ margins (guard bands) hold a fixed byte pattern.  After df11_encode (and
 df11_encode_static_ws) the margins of every output and of the workspace and
 status words must still hold the pattern; df11_decode_block_batch must leave
 its inputs (stream, gaps, block positions, sign/mantissa plane, tables) and
-the margins of its outputs untouched.  The decoded words are compared with
-the input, and the encoded arrays with the oracle.
+the margins of its outputs untouched (with no index, the run index or the
+segment index; each index is built into a guarded buffer of its own).  The
+decoded words are compared with the input, and the encoded arrays with the
+oracle.
 
 Inputs: the cases whose sizes exercise the most paths -- codes longer than
 the decode table (cap 32), an odd number of blocks (a last work unit of one
@@ -143,8 +145,23 @@ def test_encode_and_decode_stay_inside_their_buffers(df11, name, gen, cap, stati
         want = oracle.run_index(x, enc.lengths, enc.total_bits)
         assert np.array_equal(ri.inner[: 2 * want.size].cpu().numpy().view(np.uint16), want)
     before["run_index"] = ri.full.clone()
-    for use_index in (False, True):
+    # the segment index, likewise
+    si = Guarded(max(16, sizes.seg_index_bytes), dev)
+    si_status = Guarded(16, dev, fill=0)
+    df11.check(df11.df11_build_segment_index(m, si.ptr, si_status.ptr, sh),
+               "df11_build_segment_index")
+    torch.cuda.synchronize()
+    assert int(si_status.inner.cpu().numpy().view(np.uint32)[0]) == 0, "segment index status"
+    assert si.margins_intact() and si_status.margins_intact(), \
+        "the segment index wrote outside its buffers"
+    for k, g in list(bufs.items()) + [("tables", tables), ("run_index", ri)]:
+        assert torch.equal(g.full, before[k]), f"the segment index modified its input {k}"
+    want = oracle.segment_index(x, enc.lengths, enc.total_bits)
+    assert np.array_equal(si.inner[: 4 * want.size].cpu().numpy().view(np.uint32), want)
+    before["seg_index"] = si.full.clone()
+    for use_index, use_seg in ((False, False), (True, False), (False, True)):
         m.run_index = ri.ptr if use_index else None
+        m.seg_index = si.ptr if use_seg else None
         out = Guarded(max(2 * n, 16), dev, fill=0x00)
         status = Guarded(16, dev, fill=0)
         df11.check(df11.df11_decode_block_batch([m], [out.ptr], status.ptr, sh),
@@ -153,7 +170,7 @@ def test_encode_and_decode_stay_inside_their_buffers(df11, name, gen, cap, stati
         assert int(status.inner.cpu().numpy().view(np.uint32)[0]) == 0, "decode status"
         assert out.margins_intact(), "decode wrote outside its output"
         assert status.margins_intact(), "decode wrote outside its status word"
-        for k, g in list(bufs.items()) + [("tables", tables), ("run_index", ri)]:
+        for k, g in list(bufs.items()) + [("tables", tables), ("run_index", ri), ("seg_index", si)]:
             assert torch.equal(g.full, before[k]), f"decode modified its input {k}"
         got = out.inner[: 2 * n].cpu().numpy().view(np.uint16)
         assert np.array_equal(got, x)

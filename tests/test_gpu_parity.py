@@ -49,6 +49,11 @@ def assert_encoded_equal(m, enc):
 
 CAPS = [11, 12, 32]
 
+# the three decoders: with the segment index (the default when a matrix has
+# one), with the run index, and with neither (per-unit prefix sums)
+DECODERS = {"segment": {}, "run": {"seg_index": False},
+            "plain": {"run_index": False, "seg_index": False}}
+
 
 def assert_run_index_equal(m, x, enc):
     if enc.n == 0:
@@ -57,6 +62,15 @@ def assert_run_index_equal(m, x, enc):
     want = oracle.run_index(x, enc.lengths, enc.total_bits)
     got = m.run_index[: want.size].cpu().numpy().view(np.uint16)
     assert np.array_equal(got, want), "run index differs"
+
+
+def assert_seg_index_equal(m, x, enc):
+    if enc.n == 0:
+        assert m.seg_index is None
+        return
+    want = oracle.segment_index(x, enc.lengths, enc.total_bits)
+    got = m.seg_index[: want.size].cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, want), "segment index differs"
 
 
 def full_check(codec, x: np.ndarray, cap: int, call_oracle_decode: bool = True):
@@ -68,16 +82,17 @@ def full_check(codec, x: np.ndarray, cap: int, call_oracle_decode: bool = True):
     m = codec.compress(w, cap=cap)
     assert_encoded_equal(m, enc)
     assert_run_index_equal(m, x, enc)
+    assert_seg_index_equal(m, x, enc)
     expected = oracle.decode(enc, chunked=True) if call_oracle_decode else x
-    out = codec.decompress(m)
-    assert np.array_equal(bits_of(out), expected), "decode (run index) of GPU-encoded data differs"
-    out = codec.decompress(m, run_index=False)
-    assert np.array_equal(bits_of(out), expected), "decode of GPU-encoded data differs"
+    for name, kw in DECODERS.items():
+        out = codec.decompress(m, **kw)
+        assert np.array_equal(bits_of(out), expected), f"decode ({name}) of GPU-encoded data differs"
     # decode of the oracle's own buffers (independent of the GPU encoder)
     cb = codec.codebook_from_lengths(enc.lengths, enc.codes)
     mo = codec.from_host_arrays(x.shape, enc.n, enc.total_bits, cb, enc.stream, enc.gaps_packed,
                                 enc.block_pos, enc.sign_mantissa, w.device)
     assert_run_index_equal(mo, x, enc)
+    assert_seg_index_equal(mo, x, enc)
     out2 = codec.decompress(mo)
     assert np.array_equal(bits_of(out2), expected), "decode of oracle-encoded data differs"
     return m, enc
@@ -160,19 +175,22 @@ def test_workload_block_batched(codec, wid, cap):
         m = codec.compress(to_dev(x), cap=cap)
         assert_encoded_equal(m, enc)
         assert_run_index_equal(m, x, enc)
+        assert_seg_index_equal(m, x, enc)
         mats.append(m)
         xs.append(x)
         del enc
-    for use_index in (True, False):
-        outs = codec.decompress_block(mats, run_index=use_index)
+    for name, kw in DECODERS.items():
+        outs = codec.decompress_block(mats, **kw)
         for x, o in zip(xs, outs):
-            assert np.array_equal(bits_of(o), x)
+            assert np.array_equal(bits_of(o), x), name
         del outs
 
 
 @pytest.mark.parametrize("use_index", [True, False])
 @pytest.mark.parametrize("cap", CAPS)
 def test_decode_reports_corrupt_positions_without_fault(codec, cap, use_index):
+    """Block positions are read by the run-index and plain decoders (the
+    segment decoder does not read them)."""
     x = workloads.random_bf16(2_000_000, seed=9)
     m = codec.compress(to_dev(x), cap=cap)
     pos = m.block_pos.clone()
@@ -180,22 +198,22 @@ def test_decode_reports_corrupt_positions_without_fault(codec, cap, use_index):
     for b in (3, 4):  # a position inside a decode unit and one between two units
         m.block_pos[b] += 5
         status.zero_()
-        codec.decompress(m, status=status, run_index=use_index)
+        codec.decompress(m, status=status, run_index=use_index, seg_index=False)
         assert int(status.item()) == 4  # DF11_ERR_CORRUPT
         m.block_pos.copy_(pos)
     m.block_pos[5] = int(m.n) + 100  # beyond the matrix: must not be dereferenced
     status.zero_()
-    codec.decompress(m, status=status, run_index=use_index)
+    codec.decompress(m, status=status, run_index=use_index, seg_index=False)
     assert int(status.item()) == 4
     m.block_pos.copy_(pos)
     m.stream[1000:1010] ^= 0x5A  # flipped stream bits change the counts
     status.zero_()
-    out = codec.decompress(m, status=status, run_index=use_index)
+    out = codec.decompress(m, status=status, run_index=use_index, seg_index=False)
     torch.cuda.synchronize()
     assert int(status.item()) in (0, 4)
     m.stream[1000:1010] ^= 0x5A
     status.zero_()
-    out = codec.decompress(m, status=status, run_index=use_index)
+    out = codec.decompress(m, status=status, run_index=use_index, seg_index=False)
     assert int(status.item()) == 0 and np.array_equal(bits_of(out), x)
 
 
@@ -210,9 +228,40 @@ def test_decode_reports_corrupt_run_index_without_fault(codec):
     for k, v in ((5, 1), (128, 3), (300, -7), (129, 30000), (255, 32767)):
         m.run_index[k] += v
         status.zero_()
-        codec.decompress(m, status=status)
+        codec.decompress(m, status=status, seg_index=False)
         assert int(status.item()) == 4, (k, v)
         m.run_index.copy_(ri)
+    status.zero_()
+    out = codec.decompress(m, status=status, seg_index=False)
+    assert int(status.item()) == 0 and np.array_equal(bits_of(out), x)
+
+
+@pytest.mark.parametrize("cap", CAPS)
+def test_decode_reports_corrupt_segment_index_without_fault(codec, cap):
+    """Segment-index entries that disagree with the stream (one bit off, far
+    off, past the stream, out of order) are reported as corrupt: the decode
+    of a segment must end exactly where the next one starts.  Stream bits
+    flipped under an intact index are reported or decode silently (the
+    format has no checksum), never fault; the decode of intact data after
+    them is exact."""
+    x = workloads.random_bf16(2_000_000, seed=11)
+    m = codec.compress(to_dev(x), cap=cap)
+    si = m.seg_index.clone()
+    S = (m.n + 63) // 64
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for k, v in ((5, 1), (31, -1), (32, 9), (1000, 100_000), (S - 1, 3), (S, 7),
+                 (700, 1 << 31), (701, -(1 << 20))):
+        m.seg_index[k] = int(si[k]) + v if 0 <= int(si[k]) + v < (1 << 31) else (1 << 31) - 1
+        status.zero_()
+        codec.decompress(m, status=status)
+        assert int(status.item()) == 4, (k, v)
+        m.seg_index.copy_(si)
+    m.stream[5000:5010] ^= 0x5A
+    status.zero_()
+    codec.decompress(m, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) in (0, 4)
+    m.stream[5000:5010] ^= 0x5A
     status.zero_()
     out = codec.decompress(m, status=status)
     assert int(status.item()) == 0 and np.array_equal(bits_of(out), x)
