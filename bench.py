@@ -38,7 +38,7 @@ import workloads  # noqa: E402
 METRIC = "DF11 decode output BF16 GB/s & % of HBM roofline (bit-exact); ratio"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0  # the fallback dense BF16 figure (burst)
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_seg_kernel_traffic.txt")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_idx_kernel_traffic.txt")
 KERNEL_SOURCE = os.path.join(ROOT, "lossless_bf16_weight_df11_b200", "csrc", "df11_kernels.cu")
 ORACLE_SAMPLE = ("q", "o", "k", "v", "gate")
 CAP = 11  # code-length cap of the benchmarked codebooks: DF11_TABLE_BITS, the decode table's reach
@@ -109,14 +109,14 @@ def measured_tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-DECODE_BEGIN = "// ============================================================ segment decoder"
-DECODE_END = "// ============================================================ launch helpers"
+DECODE_BEGIN = "// ============================================================ decode"
+DECODE_END = "// ============================================================ segment decoder"
 
 
 def kernel_hash() -> str:
-    """Fingerprint of the segment decoder's code (its section of
-    df11_kernels.cu without comments), so that a stored traffic figure is
-    used only for the kernel it was measured on."""
+    """Fingerprint of the indexed decoder's code (the decode section of
+    df11_kernels.cu, up to the segment decoder, without comments), so that a
+    stored traffic figure is used only for the kernel it was measured on."""
     with open(KERNEL_SOURCE, encoding="utf-8") as f:
         src = f.read()
     a, b = src.find(DECODE_BEGIN), src.find(DECODE_END)
@@ -311,7 +311,7 @@ def time_configs(torch, df11, codec, dev, steps, warmup, peak, peak_kind, skip_w
             b.record(stream)
         torch.cuda.synchronize()
         ms = statistics.median(a.elapsed_time(b) for a, b in evs)
-        algo = sum(m.seg_read_bytes for m in cms) + 2 * n
+        algo = sum(m.read_bytes + m.index_bytes for m in cms) + 2 * n
         lines[workloads.workload_name(wid)] = {
             "weights": n, "matrices": len(xs), "ms_per_launch": ms,
             "value": 2 * n / (ms / 1e3) / 1e9, "unit": "GB/s", "weights_per_s": n / (ms / 1e3),
@@ -428,9 +428,9 @@ def run_df11(args):
     seg_index_bytes = sum(4 * (-(-m.n // df11.SEGMENT) + 1) for m in cms)
     stored = sum(m.stored_bytes for m in cms)
     ratio = stored / (2 * n_total)
-    # the segment decoder's bytes: the stream, the sign/mantissa plane and the
-    # segment index read, the BF16 written
-    algo_bytes = seg_read + 2 * n_total
+    # the indexed decoder's bytes: the format's arrays and the run index read,
+    # the BF16 written
+    algo_bytes = read_bytes + index_bytes + 2 * n_total
 
     outs = [torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in xs]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -480,15 +480,15 @@ def run_df11(args):
     if int(status.item()) != 0:
         raise df11.DF11Error(int(status.item()), "decode (device)")
 
-    # ---- the same block through the two other decoders: with the run index
-    # (each thread's first output known, exponents placed directly) and with
-    # no index (per-unit prefix sums of the threads' counts); and the time to
-    # build each index (once, when a matrix is placed on the device)
+    # ---- the same block through the two other decoders: with the segment
+    # index (each lane decodes 64 codes from a known bit) and with no index
+    # (per-unit prefix sums of the threads' counts); and the time to build
+    # each index (once, when a matrix is placed on the device)
     other = None
     if args.cap32:
         other = {}
         for name, kw, kern, algo in (
-                ("run_index", (True, False), "decode_idx_kernel", read_bytes + index_bytes + 2 * n_total),
+                ("seg_index", (False, True), "decode_seg_kernel", seg_read + 2 * n_total),
                 ("no_index", (False, False), "decode_kernel", read_bytes + 2 * n_total)):
             abis_o = [m.abi(*kw) for m in cms]
 
@@ -569,7 +569,7 @@ def run_df11(args):
     if args.cap32:
         cms32 = [codec.compress(w, cap=32) for w in ws]
         abis32 = [m.abi() for m in cms32]
-        algo32 = sum(m.seg_read_bytes for m in cms32) + 2 * n_total
+        algo32 = sum(m.read_bytes + m.index_bytes for m in cms32) + 2 * n_total
 
         def step32():
             st = df11.df11_decode_block_batch(abis32, out_ptrs, status.data_ptr(), sh)
@@ -635,9 +635,9 @@ def run_df11(args):
     achieved = algo_bytes / (avg_launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": profiled_traffic(name),
-                "peak_kind": peak_kind, "kernel": "decode_seg_kernel",
+                "peak_kind": peak_kind, "kernel": "decode_idx_kernel",
                 "algorithmic_bytes_per_launch": algo_bytes,
-                "seg_index_bytes_per_launch": seg_index_bytes,
+                "run_index_bytes_per_launch": index_bytes,
                 "frac_of_8TBps": achieved / 8000.0,
                 "median_launch_ms": statistics.median(per_launch_ms)}
 
@@ -1003,7 +1003,7 @@ def end_to_end(torch, df11, codec, cms, xs, dev, steps, dist, world):
     host_parts, dev_parts = [], []
     h2d = 0
     for m in cms:
-        for buf in (m.stream, m.gaps, m.block_pos, m.sign_mantissa, m.tables, m.seg_index):
+        for buf in (m.stream, m.gaps, m.block_pos, m.sign_mantissa, m.tables, m.run_index):
             h = torch.empty(buf.shape, dtype=buf.dtype, pin_memory=True)
             h.copy_(buf)
             d = torch.empty_like(buf)
@@ -1018,11 +1018,11 @@ def end_to_end(torch, df11, codec, cms, xs, dev, steps, dist, world):
     abis = []
     k = 0
     for m in cms:
-        d_stream, d_gaps, d_pos, d_sm, d_tab, d_seg = dev_parts[k:k + 6]
+        d_stream, d_gaps, d_pos, d_sm, d_tab, d_ri = dev_parts[k:k + 6]
         k += 6
-        a = m.abi(False, True)
+        a = m.abi(True, False)
         a.stream, a.gaps, a.block_pos = d_stream.data_ptr(), d_gaps.data_ptr(), d_pos.data_ptr()
-        a.sign_mantissa, a.tables, a.seg_index = d_sm.data_ptr(), d_tab.data_ptr(), d_seg.data_ptr()
+        a.sign_mantissa, a.tables, a.run_index = d_sm.data_ptr(), d_tab.data_ptr(), d_ri.data_ptr()
         abis.append(a)
     stream = torch.cuda.Stream(device=dev)
     sh = int(stream.cuda_stream)

@@ -308,12 +308,12 @@ df11_status df11_decode(const df11_matrix *m, uint16_t *d_out, uint32_t *d_statu
  *   ms      host array of count matrices, each with its own tables.
  *   d_outs  host array of count device pointers (16-byte aligned).
  * One launch per DF11_MAX_BATCH matrices.  When every matrix of a launch has
- * a segment index (df11_matrix.seg_index; total_bits < 2^32), the launch
- * takes the segment decoder: each segment's decode must end exactly where the
- * next segment starts.  Otherwise, when every matrix has a run index
- * (df11_matrix.run_index), the launch takes the indexed decoder, and each
- * thread's decoded count is also checked against the index.  Without either
- * index every block's count is checked against its stored position.
+ * a run index (df11_matrix.run_index), the launch takes the indexed decoder,
+ * and each thread's decoded count is also checked against the index.
+ * Otherwise, when every matrix has a segment index (df11_matrix.seg_index;
+ * total_bits < 2^32), it takes the segment decoder: each segment's decode
+ * must end exactly where the next segment starts.  Without either index
+ * every block's count is checked against its stored position.
  */
 df11_status df11_decode_block_batch(const df11_matrix *ms, uint32_t count,
                                     uint16_t *const *d_outs, uint32_t *d_status,

@@ -34,6 +34,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <vector>
 #include <cstddef>
 #include <mutex>
 
@@ -742,7 +743,9 @@ __device__ __forceinline__ bool smem_ok(uint32_t a, uint32_t bytes) {
 // returns a value whose top four bits are set: read as a table entry's
 // control word it consumes 15 bits and decodes nothing, so every decode loop
 // still advances to its end.)
+#ifdef DF11_CHECKED
 constexpr uint32_t kCheckFailValue = 0xF0000000u;
+#endif
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   DF11_SMEM_CHECK(a, 4, return kCheckFailValue)
   uint32_t v;
@@ -1991,7 +1994,7 @@ __global__ void __launch_bounds__(kRiThreads) run_index_kernel(const __grid_cons
 constexpr uint32_t kSegWarps = 32;
 constexpr uint32_t kSegThreads = 32 * kSegWarps;
 constexpr uint32_t kSegUnit = 32 * kSegOut;          // outputs per warp unit
-constexpr uint32_t kSegRowWords = kSegOut / 4 + 1;   // exponent words per lane, + 1 spare
+constexpr uint32_t kSegRowWords = kSegOut / 4;       // exponent words per lane
 constexpr uint32_t kSegStage = 1024;                 // stream bytes per stage
 constexpr uint32_t kSegWarpBytes = 128 * kSegRowWords + kSegUnit + 2 * kSegStage;
 constexpr uint32_t kSegSmem = kTablesSmem + kSegWarps * kSegWarpBytes;
@@ -2033,15 +2036,16 @@ __device__ __forceinline__ void seg_wait_all() { asm volatile("cp.async.wait_gro
   }
 
 // One lane's segment: cnt (<= 64) codes from stream bit p (relative to the
-// words word(k) returns, byte-swapped to MSB-first), exponents into the
-// lane's row.  True when exactly cnt codes were decoded and the last one
-// ended at pend (where the next segment starts).
+// words word(k) returns, byte-swapped to MSB-first; hw, lw and nxt are words
+// p/32, p/32 + 1 and p/32 + 2), exponents into the lane's row.  True when
+// exactly cnt codes were decoded and the last one ended at pend (where the
+// next segment starts).
 template <class WordFn>
 __device__ __forceinline__ bool seg_decode_lane(uint32_t p, uint32_t pend, uint32_t cnt,
                                                 bool table_short, const DecodeTables &tab,
                                                 uint32_t lut_a, uint32_t row_a, uint32_t row_stride,
-                                                WordFn word) {
-  uint32_t hw = word(p >> 5), lw = word((p >> 5) + 1u), nxt = word((p >> 5) + 2u);
+                                                WordFn word, uint32_t hw, uint32_t lw,
+                                                uint32_t nxt) {
   uint32_t nb = 0, cur = 0;
   const uint32_t nb_end = 8u * cnt;
   if (table_short) {
@@ -2079,7 +2083,7 @@ __device__ __forceinline__ bool seg_decode_lane(uint32_t p, uint32_t pend, uint3
     const uint32_t pn = p + adv;
     DF11_SEG_ADVANCE(pn)
   }
-  sts32(row_a + (nb >> 5) * row_stride, cur);  // the word being filled
+  if (nb & 31u) sts32(row_a + (nb >> 5) * row_stride, cur);  // the word being filled
   return nb == nb_end && p == pend;
 }
 
@@ -2184,9 +2188,11 @@ __global__ void __launch_bounds__(kSegThreads, 1) decode_seg_kernel(const __grid
       };
       bool ok = table_ok && a >= lo_bits && a <= e && e <= M.total_bits &&
                 e - a <= (uint64_t)DF11_MAX_CODE_LEN * cnt;
-      if (cnt && ok)
-        ok = seg_decode_lane(a - lo_bits, e - lo_bits, cnt, table_short, tab, lut_a, row_a, 128u,
-                             word);
+      if (cnt && ok) {
+        const uint32_t p = a - lo_bits;
+        ok = seg_decode_lane(p, e - lo_bits, cnt, table_short, tab, lut_a, row_a, 128u, word,
+                             word(p >> 5), word((p >> 5) + 1u), word((p >> 5) + 2u));
+      }
       if (__ballot_sync(0xffffffffu, cnt && !ok) && lane == 0) set_status(P.status, DF11_ERR_CORRUPT);
 
       // ---- merge: exponents + sign/mantissa -> BF16, 16 outputs at a time
@@ -2537,7 +2543,8 @@ df11_status launch_decode(const df11_matrix *ms, uint32_t count, uint16_t *const
       ++P.count;
     }
     if (P.count == 0) continue;
-    if (segmented && smem_optin >= (int)kSegSmem) {
+    // with both indices the run index wins: its decoder is the faster one
+    if (segmented && !indexed && smem_optin >= (int)kSegSmem) {
       // the segment decoder: units of 32 segments, one CTA of 32 warps per SM
       for (uint32_t i = 0; i < P.count; ++i)
         P.unit_start[i + 1] = P.unit_start[i] + cdiv(P.m[i].n_segs, kSegWarps);
@@ -2770,27 +2777,33 @@ extern "C" df11_status df11_encode_static_ws(const uint16_t *d_w, uint64_t n,
 //
 // y[j][r] += sum_c W[r][c] x[j][c] for up to 256 activation rows at a time,
 // with W decoded through its segment index straight into the B operand of
-// tcgen05.mma and never written to device memory.  A CTA owns 128 rows of W
-// (the MMA's N) and walks its columns in steps of 64: row r's columns
-// [64k, 64k + 64) are exactly segment r * cols / 64 + k of the segment index,
-// so decode lane t (four warps) decodes that segment and writes its 64 BF16
-// weights as row t of the step's B tile (K-major, 128-byte rows, 128-byte
-// swizzle).  The same lanes copy the step's activation tiles (cp.async,
-// zero-filled past the batch) as A.  A fifth warp issues, per step and per
-// 128-row M tile, four 128 x 128 x 16 MMAs accumulating in TMEM and commits
-// them to the stage's "empty" barrier; after the last step the decode warps
-// read the accumulators out of TMEM and add them to y.  Every wait is bounded.
+// tcgen05.mma and never written to device memory.  A CTA (one per SM) owns
+// 256 rows of W (the MMA's N) and walks its columns in steps of 64: row r's
+// columns [64k, 64k + 64) are exactly segment r * cols / 64 + k of the
+// segment index, so decode lane t (eight warps) decodes that segment and
+// writes its 64 BF16 weights as row t of the step's B tile (K-major,
+// 128-byte rows, 128-byte swizzle).  Everything a step reads from global
+// memory is requested a step ahead with cp.async: the lane's 64 stream bytes
+// from its segment's start, its 64 sign/mantissa bytes, and the step's
+// activation tiles (zero-filled past the batch) as A.  A ninth warp issues,
+// per step and 128-row M tile, four 128 x 256 x 16 MMAs accumulating in TMEM
+// and commits them to the stage's "empty" barrier; after the last step the
+// decode warps read the accumulators out of TMEM and add them to y.  Every
+// wait is bounded.
 namespace {
 
-constexpr uint32_t kGemmN = 128;        // W rows per CTA (MMA N)
+constexpr uint32_t kGemmN = 256;        // W rows per CTA (MMA N)
 constexpr uint32_t kGemmM = 128;        // activation rows per M tile (MMA M)
 constexpr uint32_t kGemmK = kSegOut;    // columns per step: one segment per row
 constexpr uint32_t kGemmStages = 2;
-constexpr uint32_t kGemmLanes = 128;    // decode lanes: one per W row of the tile
+constexpr uint32_t kGemmLanes = kGemmN;  // decode lanes: one per W row of the tile
 constexpr uint32_t kGemmThreads = kGemmLanes + 32;
-constexpr uint32_t kGemmTile = kGemmN * kGemmK * 2;  // 16 KiB: a B tile, or one A tile
+constexpr uint32_t kGemmBTile = kGemmN * kGemmK * 2;  // 32 KiB
+constexpr uint32_t kGemmATile = kGemmM * kGemmK * 2;  // 16 KiB
+constexpr uint32_t kGemmWin = 64;       // stream bytes staged per lane and step
 constexpr uint32_t kGemmMaxMT = DF11_GEMM_MAX_BATCH / kGemmM;
-static_assert(kGemmN == kGemmM && kGemmK * 2 == 128, "one 128-byte swizzle row per tile row");
+static_assert(kGemmK * 2 == 128, "one 128-byte swizzle row per tile row");
+static_assert(kGemmN * kGemmMaxMT <= 512, "accumulators fit the 512 TMEM columns");
 
 struct GemmParams {
   DecMat m[DF11_MAX_BATCH];
@@ -2802,12 +2815,15 @@ struct GemmParams {
   uint32_t *status;
 };
 
-__host__ __device__ constexpr uint32_t gemm_stage_bytes(uint32_t mt) { return (1 + mt) * kGemmTile; }
+__host__ __device__ constexpr uint32_t gemm_stage_bytes(uint32_t mt) {
+  return kGemmBTile + mt * kGemmATile;
+}
+// stages, tables, exponent rows, two buffers each of sign/mantissa bytes and
+// of stream bytes, barriers and the TMEM address, plus 1 KiB to align the
+// stages to the swizzle atom
 __host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t mt) {
-  // stages, tables, exponent rows, sign/mantissa pieces, barriers and the
-  // TMEM address, plus 1 KiB to align the stages to the swizzle atom
   return kGemmStages * gemm_stage_bytes(mt) + kTablesSmem + 4 * kSegRowWords * kGemmLanes +
-         kGemmK * kGemmLanes + 64 + 1024;
+         2 * kGemmK * kGemmLanes + 2 * kGemmWin * kGemmLanes + 64 + 1024;
 }
 
 // Shared-memory operand descriptor: K-major, 128-byte swizzle, rows of 128
@@ -2821,7 +2837,7 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
 }
 
 // Instruction descriptor: BF16 A and B (both K-major), FP32 accumulator,
-// M = 128, N = 128.
+// M = 128, N = 256.
 constexpr uint32_t kGemmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kGemmN >> 3) << 17) |
                                 ((kGemmM >> 4) << 24);
 
@@ -2850,6 +2866,7 @@ __device__ __forceinline__ void cp16_zfill(uint32_t dst, const void *src, uint32
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
                : "memory");
 }
+__device__ __forceinline__ void cp_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -2861,7 +2878,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
   const uint32_t tab_off = kGemmStages * stage_bytes;
   const uint32_t rows_off = tab_off + kTablesSmem;
   const uint32_t smp_off = rows_off + 4 * kSegRowWords * kGemmLanes;
-  const uint32_t bar_off = smp_off + kGemmK * kGemmLanes;
+  const uint32_t win_off = smp_off + 2 * kGemmK * kGemmLanes;
+  const uint32_t bar_off = win_off + 2 * kGemmWin * kGemmLanes;
   const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem + tab_off);
   const uint32_t lut_a = base + tab_off;
   const uint32_t bar_full = base + bar_off;                  // per stage: decode lanes arrived
@@ -2869,6 +2887,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
   const uint32_t bar_done = bar_empty + 8 * kGemmStages;     // every MMA completed
   uint32_t *slot = reinterpret_cast<uint32_t *>(smem + bar_off + 8 * (2 * kGemmStages + 1));
   const uint32_t t = threadIdx.x, warp = t >> 5, lane = t & 31u;
+  constexpr uint32_t kMmaWarp = kGemmLanes / 32;
 #ifdef DF11_CHECKED
   if (t == 0) s_check_status = P.status;
   __syncthreads();
@@ -2879,6 +2898,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
   const DecMat &M = P.m[mi];
   const uint32_t n0 = (blockIdx.x - P.tile_start[mi]) * kGemmN;
   const uint32_t ksteps = M.cols / kGemmK;
+  const uint32_t ncols = kGemmN * MT;  // TMEM columns: a power of two
 
   {
     const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
@@ -2894,11 +2914,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
     slot[1] = 0u;  // set when a bounded wait runs out
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 4) {
-    // kGemmM * MT columns of FP32 accumulators (a power of two >= 32)
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      base + bar_off + 8 * (2 * kGemmStages + 1)),
-                 "r"(kGemmN * MT)
+                 "r"(ncols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -2913,17 +2932,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(slot);
   volatile uint32_t *gave_up = slot + 1;
 
-  if (warp < 4) {
+  if (warp < kMmaWarp) {
     // ---- decode lane t: row n0 + t of W, one segment per step
     const uint32_t r = n0 + t;
     const bool row_ok = r < M.rows;
     const uint64_t seg0 = (uint64_t)r * ksteps;  // segment of (row r, step 0)
-    const uint32_t *sw = reinterpret_cast<const uint32_t *>(M.stream);
-    const uint64_t last_w = (2048ull * M.n_blocks + 16) / 4 - 1;
-    auto word = [&](uint32_t k) -> uint32_t { return bswap32(__ldg(sw + min((uint64_t)k, last_w))); };
-    const uint32_t row_a = base + rows_off + 4 * t;  // exponent word w: row_a + 512 w
-    const uint32_t smp = base + smp_off;
+    const uint64_t alloc = 2048ull * M.n_blocks + 16;  // the stream's allocation (bytes)
+    const uint32_t row_a = base + rows_off + 4 * t;    // exponent word w: row_a + 1024 w
+    const uint32_t smp = base + smp_off;               // sign/mantissa: 2 buffers
+    const uint32_t win = base + win_off;               // stream bytes: 2 buffers
+    // step k's sign/mantissa bytes (piece q of lane t at 16 (256 q + t)) and
+    // the 64 stream bytes from its start a, 16-byte aligned, into buffers k & 1
+    auto fetch = [&](uint32_t k, uint32_t a) {
+      if (!row_ok || k >= ksteps) return;
+      const uint32_t b = k & 1u;
+      for (uint32_t q = 0; q < 4u; ++q)
+        seg_cp16(smp + kGemmK * kGemmLanes * b + 16u * (kGemmLanes * q + t),
+                 M.sm + (seg0 + k) * kGemmK + 16u * q);
+      const uint64_t lo = min((uint64_t)((a >> 3) & ~15u), alloc - kGemmWin);
+      for (uint32_t q = 0; q < kGemmWin / 16; ++q)
+        seg_cp16(win + kGemmWin * kGemmLanes * b + 16u * (kGemmLanes * q + t), M.stream + lo + 16u * q);
+    };
     uint32_t a = row_ok ? __ldg(M.seg + seg0) : 0u;
+    uint32_t e = row_ok ? __ldg(M.seg + seg0 + 1) : 0u;
+    fetch(0, a);
+    seg_commit();
     bool bad = !table_ok;
     for (uint32_t k = 0; k < ksteps; ++k) {
       const uint32_t s = k % kGemmStages, use = k / kGemmStages;
@@ -2938,27 +2971,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
         const uint32_t mm = i >> 3, c = i & 7u;
         const bool in = mm < P.batch;
         const uint16_t *src = in ? M.x + (uint64_t)mm * M.cols + kGemmK * k + 8 * c : M.x;
-        cp16_zfill(st + kGemmTile * (1 + mm / kGemmM) + (mm % kGemmM) * 128 + ((c ^ (mm & 7u)) << 4),
+        cp16_zfill(st + kGemmBTile + kGemmATile * (mm / kGemmM) + (mm % kGemmM) * 128 +
+                       ((c ^ (mm & 7u)) << 4),
                    src, in ? 16u : 0u);
       }
-      // this row's 64 sign/mantissa bytes: piece q at smp + 16 (128 q + t)
-      if (row_ok)
-        for (uint32_t q = 0; q < 4u; ++q)
-          seg_cp16(smp + 16u * (kGemmLanes * q + t), M.sm + (seg0 + k) * kGemmK + 16u * q);
+      seg_commit();    // this step's tiles
+      fetch(k + 1, e);  // the next step starts where this one ends
       seg_commit();
-      const uint32_t e = row_ok ? __ldg(M.seg + seg0 + k + 1) : 0u;
-      bool ok = row_ok && table_ok && a <= e && e <= M.total_bits &&
+      const uint32_t e_next = row_ok && k + 1 < ksteps ? __ldg(M.seg + seg0 + k + 2) : 0u;
+      cp_wait2();  // this step's stream and sign/mantissa bytes
+      // the staged words from lo; past them (a segment longer than the
+      // staged bytes allow), global memory
+      const uint32_t b = k & 1u;
+      const uint32_t lo = (uint32_t)min((uint64_t)((a >> 3) & ~15u), alloc - kGemmWin);
+      const uint32_t *gsrc = reinterpret_cast<const uint32_t *>(M.stream + lo);
+      // the lane's 16-byte pieces interleave with the other lanes': piece q
+      // of lane t at 16 (256 q + t) in the buffer
+      const uint32_t wbuf = win + kGemmWin * kGemmLanes * b + 16u * t;
+      auto word = [&](uint32_t j) -> uint32_t {
+        return bswap32(j < kGemmWin / 4 ? lds32(wbuf + 16u * kGemmLanes * (j >> 2) + 4u * (j & 3u))
+                                        : __ldg(gsrc + min((uint64_t)j, (alloc - lo) / 4 - 1)));
+      };
+      bool ok = row_ok && table_ok && a <= e && e <= M.total_bits && a >= 8u * lo &&
                 e - a <= (uint32_t)DF11_MAX_CODE_LEN * kGemmK;
-      if (ok) ok = seg_decode_lane(a, e, kGemmK, table_short, tab, lut_a, row_a, 4u * kGemmLanes, word);
+      if (ok) {
+        const uint32_t p = a - 8u * lo;
+        ok = seg_decode_lane(p, e - 8u * lo, kGemmK, table_short, tab, lut_a, row_a, 4u * kGemmLanes,
+                             word, word(p >> 5), word((p >> 5) + 1u), word((p >> 5) + 2u));
+      }
       bad |= row_ok && !ok;
-      seg_wait_all();
       // row t of the B tile: 16-byte chunk c at chunk c ^ (t & 7)
       const uint32_t brow = st + 128u * t;
+      const uint32_t smk = smp + kGemmK * kGemmLanes * b;
 #pragma unroll
       for (uint32_t q = 0; q < 4u; ++q) {
         uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0;
         if (ok) {
-          const uint4 sv = lds128(smp + 16u * (kGemmLanes * q + t));
+          const uint4 sv = lds128(smk + 16u * (kGemmLanes * q + t));
           const uint32_t stride = 4u * kGemmLanes;
           merge4(lds32(row_a + stride * (4u * q)), sv.x, r0.x, r0.y);
           merge4(lds32(row_a + stride * (4u * q + 1u)), sv.y, r0.z, r0.w);
@@ -2972,11 +3021,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
                      "r"(r1.x), "r"(r1.y), "r"(r1.z), "r"(r1.w)
                      : "memory");
       }
+      seg_wait_prev();  // this step's activation tiles (all but the next step's bytes)
       // the tiles, written through the generic proxy, are read by the MMA
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       gemm_arrive(bar_full + 8 * s);
       a = e;
+      e = e_next;
     }
+    seg_wait_all();
     if (bad) set_status(P.status, DF11_ERR_CORRUPT);
   } else if (lane == 0) {
     // ---- the MMA issuer
@@ -2991,25 +3043,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
       for (uint32_t mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (uint32_t kk = 0; kk < kGemmK / 16; ++kk)
-          umma_bf16(tmem + kGemmN * mt, umma_desc_sw128(st + kGemmTile * (1 + mt) + 32u * kk),
+          umma_bf16(tmem + kGemmN * mt,
+                    umma_desc_sw128(st + kGemmBTile + kGemmATile * mt + 32u * kk),
                     umma_desc_sw128(st + 32u * kk), (k | kk) != 0u);
       umma_commit(bar_empty + 8 * s);
     }
     umma_commit(bar_done);  // arrives once every MMA issued above has completed
   }
 
-  // ---- epilogue: the accumulators (lane = activation row) added to y
+  // ---- epilogue: the accumulators (TMEM lane = activation row) added to y.
+  // Warps w and w + 4 share lanes 32 (w % 4).. and split the 256 columns.
   const bool done = mbar_wait(bar_done, 0);
   if (!done) *gave_up = 1u;
   tc_fence_after();
   __syncthreads();
-  const bool fail = *gave_up != 0u;
+  const bool fail = *gave_up != 0u;  // the same for every thread: read after the barrier
   if (t == 0 && fail) set_status(P.status, DF11_ERR_TIMEOUT);
-  if (warp < 4 && !fail) {  // (fail is the same for every thread: read after the barrier)
+  if (warp < kMmaWarp && !fail) {
+    const uint32_t quarter = warp & 3u, half = warp >> 2;
     for (uint32_t mt = 0; mt < MT; ++mt) {
-      const uint32_t j = kGemmM * mt + 32u * warp + lane;  // activation row
+      const uint32_t j = kGemmM * mt + 32u * quarter + lane;  // activation row
 #pragma unroll 1
-      for (uint32_t c = 0; c < kGemmN; c += 16) {
+      for (uint32_t c = kGemmN / 2 * half; c < kGemmN / 2 * (half + 1); c += 16) {
         uint32_t v[16];
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -3017,7 +3072,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
               "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
               "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(tmem + ((32u * warp) << 16) + kGemmN * mt + c));
+            : "r"(tmem + ((32u * quarter) << 16) + kGemmN * mt + c));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
         if (j < P.batch) {
           float *yr = M.y + (uint64_t)j * M.rows + n0 + c;
@@ -3030,9 +3085,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGemmN * MT)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols)
                  : "memory");
   }
 }
@@ -3059,31 +3114,41 @@ extern "C" df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_
       configured[dev] = true;
     }
   }
+  // check every matrix, then order them by columns, longest first: a CTA's
+  // time grows with cols, so the long tiles start first
+  std::vector<uint32_t> order;
+  for (uint32_t i = 0; i < count; ++i) {
+    const df11_matrix &m = ms[i];
+    const df11_matmul_io &q = io[i];
+    if (m.n == 0) continue;
+    if (m.n > DF11_MAX_N || m.total_bits > 0xFFFFFFFFull) return DF11_ERR_TOO_LARGE;
+    if (!m.stream || !m.sign_mantissa || !m.tables || !m.seg_index || !aligned16(m.stream) ||
+        !aligned16(m.sign_mantissa) || !aligned16(m.tables) || ((uintptr_t)m.seg_index & 3u))
+      return DF11_ERR_INVALID_ARG;
+    if (m.min_len < 1 || m.min_len > 8 || m.total_bits < m.n * (uint64_t)m.min_len ||
+        m.total_bits > m.n * 32ull)
+      return DF11_ERR_INVALID_ARG;
+    if ((uint64_t)q.rows * q.cols != m.n || q.cols % kGemmK || !q.x || !q.y || !aligned16(q.x) ||
+        ((uintptr_t)q.y & 3u))
+      return DF11_ERR_INVALID_ARG;
+    order.push_back(i);
+  }
+  std::stable_sort(order.begin(), order.end(),
+                   [&](uint32_t x, uint32_t y) { return io[x].cols > io[y].cols; });
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // batches above DF11_GEMM_MAX_BATCH rows: one pass per 256 rows (W decoded again)
   for (uint32_t j0 = 0; j0 < batch; j0 += DF11_GEMM_MAX_BATCH) {
     const uint32_t nb = std::min<uint32_t>(DF11_GEMM_MAX_BATCH, batch - j0);
-    for (uint32_t first = 0; first < count; first += DF11_MAX_BATCH) {
-      const uint32_t k = std::min<uint32_t>(DF11_MAX_BATCH, count - first);
+    for (size_t first = 0; first < order.size(); first += DF11_MAX_BATCH) {
+      const size_t k = std::min<size_t>(DF11_MAX_BATCH, order.size() - first);
       GemmParams P{};
       P.status = d_status;
       P.batch = nb;
       P.mt = (nb + kGemmM - 1) / kGemmM;
       P.min_len = DF11_MAX_CODE_LEN;
-      for (uint32_t i = 0; i < k; ++i) {
-        const df11_matrix &m = ms[first + i];
-        const df11_matmul_io &q = io[first + i];
-        if (m.n == 0) continue;
-        if (m.n > DF11_MAX_N || m.total_bits > 0xFFFFFFFFull) return DF11_ERR_TOO_LARGE;
-        if (!m.stream || !m.sign_mantissa || !m.tables || !m.seg_index || !aligned16(m.stream) ||
-            !aligned16(m.sign_mantissa) || !aligned16(m.tables) || ((uintptr_t)m.seg_index & 3u))
-          return DF11_ERR_INVALID_ARG;
-        if (m.min_len < 1 || m.min_len > 8 || m.total_bits < m.n * (uint64_t)m.min_len ||
-            m.total_bits > m.n * 32ull)
-          return DF11_ERR_INVALID_ARG;
-        if ((uint64_t)q.rows * q.cols != m.n || q.cols % kGemmK || !q.x || !q.y ||
-            !aligned16(q.x) || ((uintptr_t)q.y & 3u))
-          return DF11_ERR_INVALID_ARG;
+      for (size_t i = 0; i < k; ++i) {
+        const df11_matrix &m = ms[order[first + i]];
+        const df11_matmul_io &q = io[order[first + i]];
         DecMat &d = P.m[P.count];
         d.stream = m.stream;
         d.sm = m.sign_mantissa;
@@ -3101,7 +3166,6 @@ extern "C" df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_
         P.min_len = std::min(P.min_len, m.min_len);
         ++P.count;
       }
-      if (P.count == 0) continue;
       const uint32_t tiles = P.tile_start[P.count];
       decode_gemm_tc_kernel<<<tiles, kGemmThreads, gemm_smem_bytes(P.mt), s>>>(P);
       st = launch_status();

@@ -49,9 +49,9 @@ def assert_encoded_equal(m, enc):
 
 CAPS = [11, 12, 32]
 
-# the three decoders: with the segment index (the default when a matrix has
-# one), with the run index, and with neither (per-unit prefix sums)
-DECODERS = {"segment": {}, "run": {"seg_index": False},
+# the three decoders: with the run index (the default when a matrix has one),
+# with the segment index alone, and with neither (per-unit prefix sums)
+DECODERS = {"run": {}, "segment": {"run_index": False},
             "plain": {"run_index": False, "seg_index": False}}
 
 
@@ -228,11 +228,11 @@ def test_decode_reports_corrupt_run_index_without_fault(codec):
     for k, v in ((5, 1), (128, 3), (300, -7), (129, 30000), (255, 32767)):
         m.run_index[k] += v
         status.zero_()
-        codec.decompress(m, status=status, seg_index=False)
+        codec.decompress(m, status=status)
         assert int(status.item()) == 4, (k, v)
         m.run_index.copy_(ri)
     status.zero_()
-    out = codec.decompress(m, status=status, seg_index=False)
+    out = codec.decompress(m, status=status)
     assert int(status.item()) == 0 and np.array_equal(bits_of(out), x)
 
 
@@ -253,17 +253,17 @@ def test_decode_reports_corrupt_segment_index_without_fault(codec, cap):
                  (700, 1 << 31), (701, -(1 << 20))):
         m.seg_index[k] = int(si[k]) + v if 0 <= int(si[k]) + v < (1 << 31) else (1 << 31) - 1
         status.zero_()
-        codec.decompress(m, status=status)
+        codec.decompress(m, status=status, run_index=False)
         assert int(status.item()) == 4, (k, v)
         m.seg_index.copy_(si)
     m.stream[5000:5010] ^= 0x5A
     status.zero_()
-    codec.decompress(m, status=status)
+    codec.decompress(m, status=status, run_index=False)
     torch.cuda.synchronize()
     assert int(status.item()) in (0, 4)
     m.stream[5000:5010] ^= 0x5A
     status.zero_()
-    out = codec.decompress(m, status=status)
+    out = codec.decompress(m, status=status, run_index=False)
     assert int(status.item()) == 0 and np.array_equal(bits_of(out), x)
 
 
