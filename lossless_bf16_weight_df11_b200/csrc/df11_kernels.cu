@@ -2801,13 +2801,14 @@ constexpr uint32_t kGemmThreads = kGemmLanes + 32;
 constexpr uint32_t kGemmBTile = kGemmN * kGemmK * 2;  // 32 KiB
 constexpr uint32_t kGemmATile = kGemmM * kGemmK * 2;  // 16 KiB
 constexpr uint32_t kGemmWin = 64;       // stream bytes staged per lane and step
+constexpr uint32_t kGemmChunk = 64;     // steps per work item: 4096 columns
 constexpr uint32_t kGemmMaxMT = DF11_GEMM_MAX_BATCH / kGemmM;
 static_assert(kGemmK * 2 == 128, "one 128-byte swizzle row per tile row");
 static_assert(kGemmN * kGemmMaxMT <= 512, "accumulators fit the 512 TMEM columns");
 
 struct GemmParams {
   DecMat m[DF11_MAX_BATCH];
-  uint32_t tile_start[DF11_MAX_BATCH + 1];  // prefix sums of N tiles per matrix
+  uint32_t item_start[DF11_MAX_BATCH + 1];  // prefix sums of work items per matrix
   uint32_t count;
   uint32_t batch;  // activation rows of this launch (<= 128 * mt)
   uint32_t mt;     // M tiles: 1 or 2
@@ -2825,6 +2826,7 @@ __host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t mt) {
   return kGemmStages * gemm_stage_bytes(mt) + kTablesSmem + 4 * kSegRowWords * kGemmLanes +
          2 * kGemmK * kGemmLanes + 2 * kGemmWin * kGemmLanes + 64 + 1024;
 }
+static_assert(8 * (2 * kGemmStages + 3) + 8 <= 64, "barriers and the TMEM address fit");
 
 // Shared-memory operand descriptor: K-major, 128-byte swizzle, rows of 128
 // bytes, 8-row groups 1024 bytes apart.
@@ -2882,209 +2884,240 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
   const uint32_t bar_off = win_off + 2 * kGemmWin * kGemmLanes;
   const DecodeTables &tab = *reinterpret_cast<const DecodeTables *>(smem + tab_off);
   const uint32_t lut_a = base + tab_off;
-  const uint32_t bar_full = base + bar_off;                  // per stage: decode lanes arrived
-  const uint32_t bar_empty = bar_full + 8 * kGemmStages;     // per stage: its MMAs completed
-  const uint32_t bar_done = bar_empty + 8 * kGemmStages;     // every MMA completed
-  uint32_t *slot = reinterpret_cast<uint32_t *>(smem + bar_off + 8 * (2 * kGemmStages + 1));
+  const uint32_t bar_full = base + bar_off;               // per stage: decode lanes arrived
+  const uint32_t bar_empty = bar_full + 8 * kGemmStages;  // per stage: its MMAs completed
+  const uint32_t bar_done = bar_empty + 8 * kGemmStages;  // an item's MMAs completed
+  const uint32_t bar_free = bar_done + 8;                 // an item's accumulators read out
+  const uint32_t bar_last = bar_free + 8;                 // every MMA completed
+  uint32_t *slot = reinterpret_cast<uint32_t *>(smem + bar_off + 8 * (2 * kGemmStages + 3));
   const uint32_t t = threadIdx.x, warp = t >> 5, lane = t & 31u;
   constexpr uint32_t kMmaWarp = kGemmLanes / 32;
 #ifdef DF11_CHECKED
   if (t == 0) s_check_status = P.status;
   __syncthreads();
 #endif
-
-  uint32_t mi = 0;
-  while (mi + 1 < P.count && blockIdx.x >= P.tile_start[mi + 1]) ++mi;
-  const DecMat &M = P.m[mi];
-  const uint32_t n0 = (blockIdx.x - P.tile_start[mi]) * kGemmN;
-  const uint32_t ksteps = M.cols / kGemmK;
   const uint32_t ncols = kGemmN * MT;  // TMEM columns: a power of two
-
-  {
-    const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
-    uint4 *dst = reinterpret_cast<uint4 *>(smem + tab_off);
-    for (uint32_t k = t; k < sizeof(DecodeTables) / 16; k += blockDim.x) dst[k] = __ldg(src + k);
-  }
   if (t == 0) {
     for (uint32_t s = 0; s < kGemmStages; ++s) {
       mbar_init(bar_full + 8 * s, kGemmLanes);
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_done, 1);
+    mbar_init(bar_free, kGemmLanes);
+    mbar_init(bar_last, 1);
     slot[1] = 0u;  // set when a bounded wait runs out
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     base + bar_off + 8 * (2 * kGemmStages + 1)),
+                     base + bar_off + 8 * (2 * kGemmStages + 3)),
                  "r"(ncols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  __syncthreads();
-  bool tbad = false;
-  for (uint32_t k = t; k < (uint32_t)df11i::kLutSize; k += blockDim.x)
-    tbad |= lut_entry_bad(tab.lut[k].y, P.min_len);
   tc_fence_before();
-  const bool table_ok = !__syncthreads_or(tbad);
+  __syncthreads();
   tc_fence_after();
-  const bool table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(slot);
   volatile uint32_t *gave_up = slot + 1;
 
-  if (warp < kMmaWarp) {
-    // ---- decode lane t: row n0 + t of W, one segment per step
-    const uint32_t r = n0 + t;
-    const bool row_ok = r < M.rows;
-    const uint64_t seg0 = (uint64_t)r * ksteps;  // segment of (row r, step 0)
-    const uint64_t alloc = 2048ull * M.n_blocks + 16;  // the stream's allocation (bytes)
-    const uint32_t row_a = base + rows_off + 4 * t;    // exponent word w: row_a + 1024 w
-    const uint32_t smp = base + smp_off;               // sign/mantissa: 2 buffers
-    const uint32_t win = base + win_off;               // stream bytes: 2 buffers
-    // step k's sign/mantissa bytes (piece q of lane t at 16 (256 q + t)) and
-    // the 64 stream bytes from its start a, 16-byte aligned, into buffers k & 1
-    auto fetch = [&](uint32_t k, uint32_t a) {
-      if (!row_ok || k >= ksteps) return;
-      const uint32_t b = k & 1u;
-      for (uint32_t q = 0; q < 4u; ++q)
-        seg_cp16(smp + kGemmK * kGemmLanes * b + 16u * (kGemmLanes * q + t),
-                 M.sm + (seg0 + k) * kGemmK + 16u * q);
-      const uint64_t lo = min((uint64_t)((a >> 3) & ~15u), alloc - kGemmWin);
-      for (uint32_t q = 0; q < kGemmWin / 16; ++q)
-        seg_cp16(win + kGemmWin * kGemmLanes * b + 16u * (kGemmLanes * q + t), M.stream + lo + 16u * q);
-    };
-    uint32_t a = row_ok ? __ldg(M.seg + seg0) : 0u;
-    uint32_t e = row_ok ? __ldg(M.seg + seg0 + 1) : 0u;
-    fetch(0, a);
-    seg_commit();
-    bool bad = !table_ok;
-    for (uint32_t k = 0; k < ksteps; ++k) {
-      const uint32_t s = k % kGemmStages, use = k / kGemmStages;
-      // the stage is free once the MMAs of step k - kGemmStages completed
-      if (k >= kGemmStages && !mbar_wait(bar_empty + 8 * s, (use - 1) & 1u)) {
-        *gave_up = 1u;
-        break;
-      }
-      const uint32_t st = base + s * stage_bytes;
-      // the step's activation tiles: row m, 16-byte chunk c at chunk c ^ (m & 7)
-      for (uint32_t i = t; i < MT * kGemmM * 8; i += kGemmLanes) {
-        const uint32_t mm = i >> 3, c = i & 7u;
-        const bool in = mm < P.batch;
-        const uint16_t *src = in ? M.x + (uint64_t)mm * M.cols + kGemmK * k + 8 * c : M.x;
-        cp16_zfill(st + kGemmBTile + kGemmATile * (mm / kGemmM) + (mm % kGemmM) * 128 +
-                       ((c ^ (mm & 7u)) << 4),
-                   src, in ? 16u : 0u);
-      }
-      seg_commit();    // this step's tiles
-      fetch(k + 1, e);  // the next step starts where this one ends
-      seg_commit();
-      const uint32_t e_next = row_ok && k + 1 < ksteps ? __ldg(M.seg + seg0 + k + 2) : 0u;
-      cp_wait2();  // this step's stream and sign/mantissa bytes
-      // the staged words from lo; past them (a segment longer than the
-      // staged bytes allow), global memory
-      const uint32_t b = k & 1u;
-      const uint32_t lo = (uint32_t)min((uint64_t)((a >> 3) & ~15u), alloc - kGemmWin);
-      const uint32_t *gsrc = reinterpret_cast<const uint32_t *>(M.stream + lo);
-      // the lane's 16-byte pieces interleave with the other lanes': piece q
-      // of lane t at 16 (256 q + t) in the buffer
-      const uint32_t wbuf = win + kGemmWin * kGemmLanes * b + 16u * t;
-      auto word = [&](uint32_t j) -> uint32_t {
-        return bswap32(j < kGemmWin / 4 ? lds32(wbuf + 16u * kGemmLanes * (j >> 2) + 4u * (j & 3u))
-                                        : __ldg(gsrc + min((uint64_t)j, (alloc - lo) / 4 - 1)));
-      };
-      bool ok = row_ok && table_ok && a <= e && e <= M.total_bits && a >= 8u * lo &&
-                e - a <= (uint32_t)DF11_MAX_CODE_LEN * kGemmK;
-      if (ok) {
-        const uint32_t p = a - 8u * lo;
-        ok = seg_decode_lane(p, e - 8u * lo, kGemmK, table_short, tab, lut_a, row_a, 4u * kGemmLanes,
-                             word, word(p >> 5), word((p >> 5) + 1u), word((p >> 5) + 2u));
-      }
-      bad |= row_ok && !ok;
-      // row t of the B tile: 16-byte chunk c at chunk c ^ (t & 7)
-      const uint32_t brow = st + 128u * t;
-      const uint32_t smk = smp + kGemmK * kGemmLanes * b;
-#pragma unroll
-      for (uint32_t q = 0; q < 4u; ++q) {
-        uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0;
-        if (ok) {
-          const uint4 sv = lds128(smk + 16u * (kGemmLanes * q + t));
-          const uint32_t stride = 4u * kGemmLanes;
-          merge4(lds32(row_a + stride * (4u * q)), sv.x, r0.x, r0.y);
-          merge4(lds32(row_a + stride * (4u * q + 1u)), sv.y, r0.z, r0.w);
-          merge4(lds32(row_a + stride * (4u * q + 2u)), sv.z, r1.x, r1.y);
-          merge4(lds32(row_a + stride * (4u * q + 3u)), sv.w, r1.z, r1.w);
-        }
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(brow + (((2u * q) ^ (t & 7u)) << 4)),
-                     "r"(r0.x), "r"(r0.y), "r"(r0.z), "r"(r0.w)
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(brow + (((2u * q + 1u) ^ (t & 7u)) << 4)),
-                     "r"(r1.x), "r"(r1.y), "r"(r1.z), "r"(r1.w)
-                     : "memory");
-      }
-      seg_wait_prev();  // this step's activation tiles (all but the next step's bytes)
-      // the tiles, written through the generic proxy, are read by the MMA
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      gemm_arrive(bar_full + 8 * s);
-      a = e;
-      e = e_next;
+  // this CTA's work items: a contiguous share of the launch's (matrix, tile
+  // of 256 rows, chunk of kGemmChunk steps) list
+  const uint32_t total = P.item_start[P.count];
+  const uint32_t i0 = (uint32_t)((uint64_t)blockIdx.x * total / gridDim.x);
+  const uint32_t i1 = (uint32_t)((uint64_t)(blockIdx.x + 1) * total / gridDim.x);
+  uint32_t gstep = 0;  // steps so far: stage gstep % 2, its use gstep / 2
+  uint32_t nitems = 0;
+  uint32_t mi = 0xFFFFFFFFu;
+  bool table_ok = false, table_short = true;
+  bool bad = false;
+  for (uint32_t item = i0; item < i1; ++item) {
+    uint32_t m = mi == 0xFFFFFFFFu ? 0 : mi;
+    while (m + 1 < P.count && item >= P.item_start[m + 1]) ++m;
+    const DecMat &M = P.m[m];
+    if (m != mi) {
+      // a new matrix: its tables (every thread is past the previous item's decode)
+      __syncthreads();
+      const uint4 *src = reinterpret_cast<const uint4 *>(M.tables);
+      uint4 *dst = reinterpret_cast<uint4 *>(smem + tab_off);
+      for (uint32_t k = t; k < sizeof(DecodeTables) / 16; k += blockDim.x) dst[k] = __ldg(src + k);
+      __syncthreads();
+      bool tbad = false;
+      for (uint32_t k = t; k < (uint32_t)df11i::kLutSize; k += blockDim.x)
+        tbad |= lut_entry_bad(tab.lut[k].y, P.min_len);
+      table_ok = !__syncthreads_or(tbad);
+      table_short = tab.max_len <= (uint32_t)df11i::kLutBits;
+      mi = m;
     }
-    seg_wait_all();
-    if (bad) set_status(P.status, DF11_ERR_CORRUPT);
-  } else if (lane == 0) {
-    // ---- the MMA issuer
-    for (uint32_t k = 0; k < ksteps; ++k) {
-      const uint32_t s = k % kGemmStages, use = k / kGemmStages;
-      if (!mbar_wait(bar_full + 8 * s, use & 1u)) {
-        *gave_up = 1u;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t st = base + s * stage_bytes;
-      for (uint32_t mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (uint32_t kk = 0; kk < kGemmK / 16; ++kk)
-          umma_bf16(tmem + kGemmN * mt,
-                    umma_desc_sw128(st + kGemmBTile + kGemmATile * mt + 32u * kk),
-                    umma_desc_sw128(st + 32u * kk), (k | kk) != 0u);
-      umma_commit(bar_empty + 8 * s);
-    }
-    umma_commit(bar_done);  // arrives once every MMA issued above has completed
-  }
+    const uint32_t ksteps = M.cols / kGemmK;
+    const uint32_t chunks = (ksteps + kGemmChunk - 1) / kGemmChunk;
+    const uint32_t local = item - P.item_start[m];
+    const uint32_t n0 = (local / chunks) * kGemmN;
+    const uint32_t k0 = (local % chunks) * kGemmChunk, k1 = min(k0 + kGemmChunk, ksteps);
 
-  // ---- epilogue: the accumulators (TMEM lane = activation row) added to y.
-  // Warps w and w + 4 share lanes 32 (w % 4).. and split the 256 columns.
-  const bool done = mbar_wait(bar_done, 0);
-  if (!done) *gave_up = 1u;
-  tc_fence_after();
-  __syncthreads();
-  const bool fail = *gave_up != 0u;  // the same for every thread: read after the barrier
-  if (t == 0 && fail) set_status(P.status, DF11_ERR_TIMEOUT);
-  if (warp < kMmaWarp && !fail) {
-    const uint32_t quarter = warp & 3u, half = warp >> 2;
-    for (uint32_t mt = 0; mt < MT; ++mt) {
-      const uint32_t j = kGemmM * mt + 32u * quarter + lane;  // activation row
-#pragma unroll 1
-      for (uint32_t c = kGemmN / 2 * half; c < kGemmN / 2 * (half + 1); c += 16) {
-        uint32_t v[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-            "%11, %12, %13, %14, %15}, [%16];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-              "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-              "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(tmem + ((32u * quarter) << 16) + kGemmN * mt + c));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (j < P.batch) {
-          float *yr = M.y + (uint64_t)j * M.rows + n0 + c;
+    if (warp < kMmaWarp) {
+      // ---- decode lane t: row n0 + t of W, one segment per step
+      const uint32_t r = n0 + t;
+      const bool row_ok = r < M.rows;
+      const uint64_t seg0 = (uint64_t)r * ksteps;  // segment of (row r, step 0)
+      const uint64_t alloc = 2048ull * M.n_blocks + 16;  // the stream's allocation (bytes)
+      const uint32_t row_a = base + rows_off + 4 * t;    // exponent word w: row_a + 1024 w
+      const uint32_t smp = base + smp_off;               // sign/mantissa: 2 buffers
+      const uint32_t win = base + win_off;               // stream bytes: 2 buffers
+      // step k's sign/mantissa bytes (piece q of lane t at 16 (256 q + t)) and
+      // the 64 stream bytes from its start a, 16-byte aligned, into buffers k & 1
+      auto fetch = [&](uint32_t k, uint32_t a) {
+        if (!row_ok || k >= k1) return;
+        const uint32_t bf = k & 1u;
+        for (uint32_t q = 0; q < 4u; ++q)
+          seg_cp16(smp + kGemmK * kGemmLanes * bf + 16u * (kGemmLanes * q + t),
+                   M.sm + (seg0 + k) * kGemmK + 16u * q);
+        const uint64_t lo = min((uint64_t)((a >> 3) & ~15u), alloc - kGemmWin);
+        for (uint32_t q = 0; q < kGemmWin / 16; ++q)
+          seg_cp16(win + kGemmWin * kGemmLanes * bf + 16u * (kGemmLanes * q + t),
+                   M.stream + lo + 16u * q);
+      };
+      uint32_t a = row_ok ? __ldg(M.seg + seg0 + k0) : 0u;
+      uint32_t e = row_ok ? __ldg(M.seg + seg0 + k0 + 1) : 0u;
+      fetch(k0, a);
+      seg_commit();
+      for (uint32_t k = k0; k < k1; ++k, ++gstep) {
+        const uint32_t s = gstep % kGemmStages, use = gstep / kGemmStages;
+        // the stage is free once the MMAs of its previous step completed
+        if (*gave_up || (gstep >= kGemmStages && !mbar_wait(bar_empty + 8 * s, (use - 1) & 1u))) {
+          *gave_up = 1u;  // (a bounded wait ran out: the CTA skips the rest of its
+          continue;       // work but keeps its loop structure, barriers included)
+        }
+        const uint32_t st = base + s * stage_bytes;
+        // the step's activation tiles: row m, 16-byte chunk c at chunk c ^ (m & 7)
+        for (uint32_t i = t; i < MT * kGemmM * 8; i += kGemmLanes) {
+          const uint32_t mm = i >> 3, c = i & 7u;
+          const bool in = mm < P.batch;
+          const uint16_t *src = in ? M.x + (uint64_t)mm * M.cols + kGemmK * k + 8 * c : M.x;
+          cp16_zfill(st + kGemmBTile + kGemmATile * (mm / kGemmM) + (mm % kGemmM) * 128 +
+                         ((c ^ (mm & 7u)) << 4),
+                     src, in ? 16u : 0u);
+        }
+        seg_commit();     // this step's tiles
+        fetch(k + 1, e);  // the next step starts where this one ends
+        seg_commit();
+        const uint32_t e_next = row_ok && k + 1 < k1 ? __ldg(M.seg + seg0 + k + 2) : 0u;
+        cp_wait2();  // this step's stream and sign/mantissa bytes
+        // the staged words from lo (the lane's 16-byte pieces interleave with
+        // the other lanes': piece q of lane t at 16 (256 q + t)); past them (a
+        // segment longer than the staged bytes allow), global memory
+        const uint32_t bf = k & 1u;
+        const uint32_t lo = (uint32_t)min((uint64_t)((a >> 3) & ~15u), alloc - kGemmWin);
+        const uint32_t *gsrc = reinterpret_cast<const uint32_t *>(M.stream + lo);
+        const uint32_t wbuf = win + kGemmWin * kGemmLanes * bf + 16u * t;
+        auto word = [&](uint32_t j) -> uint32_t {
+          return bswap32(j < kGemmWin / 4 ? lds32(wbuf + 16u * kGemmLanes * (j >> 2) + 4u * (j & 3u))
+                                          : __ldg(gsrc + min((uint64_t)j, (alloc - lo) / 4 - 1)));
+        };
+        bool ok = row_ok && table_ok && a <= e && e <= M.total_bits && a >= 8u * lo &&
+                  e - a <= (uint32_t)DF11_MAX_CODE_LEN * kGemmK;
+        if (ok) {
+          const uint32_t p = a - 8u * lo;
+          ok = seg_decode_lane(p, e - 8u * lo, kGemmK, table_short, tab, lut_a, row_a,
+                               4u * kGemmLanes, word, word(p >> 5), word((p >> 5) + 1u),
+                               word((p >> 5) + 2u));
+        }
+        bad |= row_ok && !ok;
+        // row t of the B tile: 16-byte chunk c at chunk c ^ (t & 7)
+        const uint32_t brow = st + 128u * t;
+        const uint32_t smk = smp + kGemmK * kGemmLanes * bf;
 #pragma unroll
-          for (uint32_t i = 0; i < 16; ++i)
-            if (n0 + c + i < M.rows) yr[i] += __uint_as_float(v[i]);
+        for (uint32_t q = 0; q < 4u; ++q) {
+          uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = r0;
+          if (ok) {
+            const uint4 sv = lds128(smk + 16u * (kGemmLanes * q + t));
+            const uint32_t stride = 4u * kGemmLanes;
+            merge4(lds32(row_a + stride * (4u * q)), sv.x, r0.x, r0.y);
+            merge4(lds32(row_a + stride * (4u * q + 1u)), sv.y, r0.z, r0.w);
+            merge4(lds32(row_a + stride * (4u * q + 2u)), sv.z, r1.x, r1.y);
+            merge4(lds32(row_a + stride * (4u * q + 3u)), sv.w, r1.z, r1.w);
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(brow + (((2u * q) ^ (t & 7u)) << 4)),
+                       "r"(r0.x), "r"(r0.y), "r"(r0.z), "r"(r0.w)
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(brow + (((2u * q + 1u) ^ (t & 7u)) << 4)),
+                       "r"(r1.x), "r"(r1.y), "r"(r1.z), "r"(r1.w)
+                       : "memory");
+        }
+        seg_wait_prev();  // this step's activation tiles (all but the next step's bytes)
+        // the tiles, written through the generic proxy, are read by the MMA
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        gemm_arrive(bar_full + 8 * s);
+        a = e;
+        e = e_next;
+      }
+      seg_wait_all();
+      // ---- the item's accumulators (TMEM lane = activation row) added to y.
+      // Warps w and w + 4 share lanes 32 (w % 4).. and split the 256 columns;
+      // other items add to the same sums, hence the atomic adds.
+      if (*gave_up || !mbar_wait(bar_done, nitems & 1u)) *gave_up = 1u;
+      tc_fence_after();
+      const uint32_t quarter = warp & 3u, half = warp >> 2;
+      // (the TMEM loads need the whole warp: it skips them together)
+      const bool skip = __any_sync(0xffffffffu, *gave_up != 0u);
+      for (uint32_t mt = 0; mt < (skip ? 0u : MT); ++mt) {
+        const uint32_t j = kGemmM * mt + 32u * quarter + lane;  // activation row
+#pragma unroll 1
+        for (uint32_t c = kGemmN / 2 * half; c < kGemmN / 2 * (half + 1); c += 16) {
+          uint32_t v[16];
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+              "%11, %12, %13, %14, %15}, [%16];"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+                "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+              : "r"(tmem + ((32u * quarter) << 16) + kGemmN * mt + c));
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          if (j < P.batch) {
+            float *yr = M.y + (uint64_t)j * M.rows + n0 + c;
+#pragma unroll
+            for (uint32_t i = 0; i < 16; ++i)
+              if (n0 + c + i < M.rows) atomicAdd(yr + i, __uint_as_float(v[i]));
+          }
         }
       }
+      tc_fence_before();
+      gemm_arrive(bar_free);  // the next item's MMAs may overwrite the accumulators
+    } else if (lane == 0) {
+      // ---- the MMA issuer: the item's steps into the accumulators, once the
+      // previous item's were read out
+      if (*gave_up || (nitems > 0 && !mbar_wait(bar_free, (nitems - 1) & 1u))) *gave_up = 1u;
+      tc_fence_after();
+      for (uint32_t k = k0; k < k1; ++k, ++gstep) {
+        const uint32_t s = gstep % kGemmStages, use = gstep / kGemmStages;
+        if (*gave_up || !mbar_wait(bar_full + 8 * s, use & 1u)) {
+          *gave_up = 1u;
+          continue;
+        }
+        tc_fence_after();
+        const uint32_t st = base + s * stage_bytes;
+        for (uint32_t mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (uint32_t kk = 0; kk < kGemmK / 16; ++kk)
+            umma_bf16(tmem + kGemmN * mt,
+                      umma_desc_sw128(st + kGemmBTile + kGemmATile * mt + 32u * kk),
+                      umma_desc_sw128(st + 32u * kk), (k != k0) || (kk != 0u));
+        umma_commit(bar_empty + 8 * s);
+      }
+      umma_commit(bar_done);  // arrives once the item's MMAs have completed
+    } else {
+      // lanes 1..31 of the MMA warp follow the loop (for the table barriers)
+      gstep += k1 - k0;
     }
+    ++nitems;
   }
+  if (bad) set_status(P.status, DF11_ERR_CORRUPT);
+  // every MMA this CTA issued has completed before the accumulators go
+  if (warp == kMmaWarp && lane == 0) umma_commit(bar_last);
+  if (!mbar_wait(bar_last, 0)) *gave_up = 1u;
   tc_fence_before();
   __syncthreads();
+  if (t == 0 && *gave_up) set_status(P.status, DF11_ERR_TIMEOUT);
   if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols)
@@ -3114,8 +3147,7 @@ extern "C" df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_
       configured[dev] = true;
     }
   }
-  // check every matrix, then order them by columns, longest first: a CTA's
-  // time grows with cols, so the long tiles start first
+  // check every matrix (the work items are then listed longest matrix first)
   std::vector<uint32_t> order;
   for (uint32_t i = 0; i < count; ++i) {
     const df11_matrix &m = ms[i];
@@ -3162,12 +3194,16 @@ extern "C" df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_
         d.cols = q.cols;
         d.x = q.x + (uint64_t)j0 * q.cols;
         d.y = q.y + (uint64_t)j0 * q.rows;
-        P.tile_start[P.count + 1] = P.tile_start[P.count] + (uint32_t)cdiv(q.rows, kGemmN);
+        P.item_start[P.count + 1] =
+            P.item_start[P.count] +
+            (uint32_t)(cdiv(q.rows, kGemmN) * cdiv(q.cols / kGemmK, kGemmChunk));
         P.min_len = std::min(P.min_len, m.min_len);
         ++P.count;
       }
-      const uint32_t tiles = P.tile_start[P.count];
-      decode_gemm_tc_kernel<<<tiles, kGemmThreads, gemm_smem_bytes(P.mt), s>>>(P);
+      // one persistent CTA per SM, each with a contiguous share of the items
+      const uint32_t items = P.item_start[P.count];
+      const uint32_t grid = std::min<uint32_t>(items, (uint32_t)sms);
+      decode_gemm_tc_kernel<<<grid, kGemmThreads, gemm_smem_bytes(P.mt), s>>>(P);
       st = launch_status();
       if (st != DF11_OK) return st;
     }
