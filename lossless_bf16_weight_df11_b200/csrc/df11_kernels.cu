@@ -714,15 +714,18 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
 // status word, so an indexing error shows as a status, not a fault.  The
 // product build compiles the checks away.
 #ifdef DF11_CHECKED
+// Set by each checked kernel before its first checked access: the status word
+// and the shared-space address of its own dynamic shared memory (an extern
+// shared array declared outside the kernel was found not to start there).
 __shared__ uint32_t *s_check_status;
-extern __shared__ __align__(128) uint8_t df11_dyn_smem[];
+__shared__ uint32_t s_dyn_base;
 __device__ __forceinline__ void check_failed() {
   if (s_check_status) atomicCAS(s_check_status, 0u, (uint32_t)DF11_ERR_BOUNDS);
 }
 __device__ __forceinline__ bool smem_ok(uint32_t a, uint32_t bytes) {
   uint32_t size;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(size));
-  const uint32_t lo = smem_addr(df11_dyn_smem);
+  const uint32_t lo = s_dyn_base;
   const bool ok = a >= lo && a - lo <= size && bytes <= size - (a - lo) && (a & (bytes - 1)) == 0;
   if (!ok) check_failed();
   return ok;
@@ -1149,7 +1152,10 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_kernel(const __grid_
   const uint64_t g1 = (uint64_t)(blockIdx.x + 1) * total / gridDim.x;
   if (g0 >= g1) return;  // the same for every thread of the CTA
 #ifdef DF11_CHECKED
-  if (threadIdx.x == 0) s_check_status = P.status;
+  if (threadIdx.x == 0) {
+    s_check_status = P.status;
+    s_dyn_base = smem_addr(smem);
+  }
   __syncthreads();
 #endif
 
@@ -1573,7 +1579,10 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_idx_kernel(const __g
   const uint64_t g1 = (uint64_t)(blockIdx.x + 1) * total / gridDim.x;
   if (g0 >= g1) return;  // the same for every thread of the CTA
 #ifdef DF11_CHECKED
-  if (threadIdx.x == 0) s_check_status = P.status;
+  if (threadIdx.x == 0) {
+    s_check_status = P.status;
+    s_dyn_base = smem_addr(smem);
+  }
   __syncthreads();
 #endif
 
@@ -2104,7 +2113,10 @@ __global__ void __launch_bounds__(kSegThreads, 1) decode_seg_kernel(const __grid
   const uint64_t g1 = (uint64_t)(blockIdx.x + 1) * total / gridDim.x;
   if (g0 >= g1) return;  // the same for every thread of the CTA
 #ifdef DF11_CHECKED
-  if (threadIdx.x == 0) s_check_status = P.status;
+  if (threadIdx.x == 0) {
+    s_check_status = P.status;
+    s_dyn_base = smem_addr(smem);
+  }
   __syncthreads();
 #endif
   uint32_t m = 0;
@@ -2820,11 +2832,12 @@ __host__ __device__ constexpr uint32_t gemm_stage_bytes(uint32_t mt) {
   return kGemmBTile + mt * kGemmATile;
 }
 // stages, tables, exponent rows, two buffers each of sign/mantissa bytes and
-// of stream bytes, barriers and the TMEM address, plus 1 KiB to align the
-// stages to the swizzle atom
+// of stream bytes, barriers and the TMEM address (the stages start the
+// dynamic shared memory, which the kernel declares 1024-byte aligned: the
+// swizzle atom)
 __host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t mt) {
   return kGemmStages * gemm_stage_bytes(mt) + kTablesSmem + 4 * kSegRowWords * kGemmLanes +
-         2 * kGemmK * kGemmLanes + 2 * kGemmWin * kGemmLanes + 64 + 1024;
+         2 * kGemmK * kGemmLanes + 2 * kGemmWin * kGemmLanes + 64;
 }
 static_assert(8 * (2 * kGemmStages + 3) + 8 <= 64, "barriers and the TMEM address fit");
 
@@ -2873,8 +2886,12 @@ __device__ __forceinline__ void cp_wait2() { asm volatile("cp.async.wait_group 2
 __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t *smem = smem_raw + (base - raw);
+  if (raw & 1023u) {  // the declared alignment was not honoured: nothing is done
+    if (threadIdx.x == 0) set_status(P.status, DF11_ERR_CUDA);
+    return;
+  }
+  const uint32_t base = raw;
+  uint8_t *smem = smem_raw;
   const uint32_t MT = P.mt;
   const uint32_t stage_bytes = gemm_stage_bytes(MT);
   const uint32_t tab_off = kGemmStages * stage_bytes;
@@ -2893,7 +2910,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_tc_kernel(const _
   const uint32_t t = threadIdx.x, warp = t >> 5, lane = t & 31u;
   constexpr uint32_t kMmaWarp = kGemmLanes / 32;
 #ifdef DF11_CHECKED
-  if (t == 0) s_check_status = P.status;
+  if (t == 0) {
+    s_check_status = P.status;
+    s_dyn_base = raw;
+  }
   __syncthreads();
 #endif
   const uint32_t ncols = kGemmN * MT;  // TMEM columns: a power of two
@@ -3132,21 +3152,30 @@ extern "C" df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_
                                               df11_stream_t stream) {
   if (count == 0) return DF11_OK;
   if (!ms || !io || !d_status || batch < 1) return DF11_ERR_INVALID_ARG;
-  int dev, sms, smem_optin;
-  df11_status st = device_info(&dev, &sms, &smem_optin);
+  int dev, sms;
+  df11_status st = device_info(&dev, &sms);
   if (st != DF11_OK) return st;
-  static bool configured[64] = {};
+  // the dynamic shared memory this kernel may take: the device's per-CTA
+  // limit less the kernel's own static shared variables
+  static int avail[64] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
-    if (!configured[dev]) {
-      if (smem_optin < (int)gemm_smem_bytes(kGemmMaxMT)) return DF11_ERR_INVALID_ARG;
-      if (cudaFuncSetAttribute(decode_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)gemm_smem_bytes(kGemmMaxMT)) != cudaSuccess)
+    if (!avail[dev]) {
+      int optin = 0;
+      cudaFuncAttributes fa;
+      if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, decode_gemm_tc_kernel) != cudaSuccess)
         return DF11_ERR_CUDA;
-      configured[dev] = true;
+      const int a = optin - (int)fa.sharedSizeBytes;
+      if (cudaFuncSetAttribute(decode_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               std::min(a, (int)gemm_smem_bytes(kGemmMaxMT))) != cudaSuccess)
+        return DF11_ERR_CUDA;
+      avail[dev] = a;
     }
   }
+  if (avail[dev] < (int)gemm_smem_bytes(std::min<uint32_t>(kGemmMaxMT, (batch + kGemmM - 1) / kGemmM)))
+    return DF11_ERR_INVALID_ARG;
   // check every matrix (the work items are then listed longest matrix first)
   std::vector<uint32_t> order;
   for (uint32_t i = 0; i < count; ++i) {
