@@ -417,18 +417,19 @@ __global__ void __launch_bounds__(df11i::kEncThreads) enc_pack_kernel(
     }
     if (n_blocks > 0 && (s64 >> 14) < n_blocks - 1) block_pos[n_blocks - 1] = (uint32_t)n;
   }
-  // sign/mantissa plane ([Format]: kept verbatim, one byte per value)
+  // sign/mantissa plane ([Format]: kept verbatim, one byte per value).  Two
+  // values per 32-bit word: the sign (bit 15 of a value) moved down to bit 7,
+  // the mantissa (bits 6..0) kept, both values at once; then the two low
+  // bytes of two such words packed into one word of four plane bytes
   if (i0 + 16 <= n) {
     uint32_t pk[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      uint32_t x = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t wv = v[4 * q + j];
-        x |= (((wv >> 8) & 0x80u) | (wv & 0x7Fu)) << (8 * j);
-      }
-      pk[q] = x;
+      const uint32_t w0 = (uint32_t)v[4 * q] | ((uint32_t)v[4 * q + 1] << 16);
+      const uint32_t w1 = (uint32_t)v[4 * q + 2] | ((uint32_t)v[4 * q + 3] << 16);
+      const uint32_t t0 = (w0 & 0x007F007Fu) | ((w0 >> 8) & 0x00800080u);
+      const uint32_t t1 = (w1 & 0x007F007Fu) | ((w1 >> 8) & 0x00800080u);
+      pk[q] = __byte_perm(t0, t1, 0x6420);
     }
     *reinterpret_cast<uint4 *>(sign_mantissa + i0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   } else {
