@@ -514,6 +514,62 @@ df11_status df11_read(const void *buf, uint64_t buf_bytes, df11_host_matrix *out
  */
 df11_status df11_codebook_from_lengths(const uint8_t len[256], uint32_t cap, df11_codebook *out);
 
+/*
+ * df11_decode_host_scratch_bytes -- host.  Device scratch that
+ * df11_decode_host_batch needs for these matrices: every matrix's decode
+ * tables, plus three slots each as large as the largest piece needs (its
+ * device arrays, run index and BF16 output; pieces as df11_decode_host_batch
+ * cuts them).  Reads each matrix's code lengths and a few of its block
+ * positions.  0 if a matrix's (n, total_bits) pair is invalid
+ * (df11_sizes_from_bits) or the call would reject its metadata.
+ */
+uint64_t df11_decode_host_scratch_bytes(const df11_host_matrix *ms, uint32_t count);
+
+/*
+ * df11_decode_host_batch -- decode matrices held in HOST memory into HOST
+ * memory: the [Kernel] decode with its host-to-device and device-to-host
+ * copies, pipelined.  Every matrix is cut into pieces of whole decode units:
+ * the call's first piece is 256 blocks of 256 chunks long at most, every
+ * later one twice the one before, up to 4096 blocks (about 26 M values for
+ * exponent codes of 2.6 bits); a cut is moved on by a unit where the codes
+ * running over it would leave the piece fewer than codebook.min_len bits per
+ * value.  Per piece: its stored arrays are copied
+ * into a slot of d_scratch, its block positions are made relative to its
+ * first value, its run index is built (df11_build_run_index), it is decoded
+ * (df11_decode), and its BF16 bit patterns are copied to their place in
+ * h_outs[i].  Each matrix's decode tables are built on the device from its
+ * code lengths.  The copies in, the kernels and the copies out run on three
+ * streams the call creates and releases, so both copy directions and the
+ * kernels overlap from piece to piece.  The work starts after what is already
+ * queued on `stream`, and `stream` waits for all of it: a synchronize of
+ * `stream` makes every h_outs[i] ready.
+ *
+ *   ms        count host matrices (df11_host_matrix, as df11_read gives; the
+ *             code lengths rebuild each codebook, df11_codebook_from_lengths)
+ *   h_outs    count host buffers of n uint16 each.  Page-locked host memory
+ *             (cudaHostAlloc) for ms' arrays and h_outs lets the copies run
+ *             asynchronously at full PCIe speed; pageable memory works, with
+ *             copies that the driver stages through its own buffers
+ *   d_scratch device memory, 256-byte aligned, of at least
+ *             df11_decode_host_scratch_bytes(ms, count) bytes; the call owns
+ *             it until `stream` has passed the call
+ *   d_status  device status word, as df11_decode
+ *
+ * The host checks every matrix first, and queues nothing when it fails:
+ * DF11_ERR_INVALID_ARG for a null pointer, code lengths that do not form a
+ * code or whose shortest code is longer than 8 bits, a max_block_codes above
+ * what the shortest code allows, or too little scratch; DF11_ERR_TOO_LARGE
+ * for n above DF11_MAX_N; DF11_ERR_CORRUPT when block_pos[0] is not 0,
+ * block_pos[n_blocks] is not n, or the positions at a cut leave a piece an
+ * impossible size.  DF11_ERR_CUDA if a stream, event, copy or launch fails
+ * once queuing started (what was queued still finishes before `stream` goes
+ * on).  Other data errors go to d_status, as in df11_decode.
+ */
+df11_status df11_decode_host_batch(const df11_host_matrix *ms, uint32_t count,
+                                   uint16_t *const *h_outs, void *d_scratch,
+                                   uint64_t scratch_bytes, uint32_t *d_status,
+                                   df11_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

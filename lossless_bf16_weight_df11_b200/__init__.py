@@ -144,6 +144,10 @@ def _declare(lib):
                                       ctypes.POINTER(ctypes.c_uint64)]),
         "df11_read": (ctypes.c_int, [_vp, _u64, ctypes.POINTER(df11_host_matrix)]),
         "df11_codebook_from_lengths": (ctypes.c_int, [_vp, _u32, ctypes.POINTER(df11_codebook)]),
+        "df11_decode_host_scratch_bytes": (_u64, [ctypes.POINTER(df11_host_matrix), _u32]),
+        "df11_decode_host_batch": (ctypes.c_int, [ctypes.POINTER(df11_host_matrix), _u32,
+                                                  ctypes.POINTER(ctypes.c_void_p), _vp, _u64,
+                                                  _vp, _vp]),
         "df11_build_codebook_device": (ctypes.c_int, [_vp, _u32, _vp, _vp, _vp, _vp, _vp]),
         "df11_encode_device_codebook": (ctypes.c_int, [_vp, _u64, _vp, _u64,
                                                        ctypes.POINTER(df11_encoded), _vp,
@@ -309,6 +313,23 @@ def df11_read(buf: int, buf_bytes: int):
     out = df11_host_matrix()
     st = load().df11_read(buf, buf_bytes, ctypes.byref(out))
     return st, out
+
+
+def df11_decode_host_scratch_bytes(ms) -> int:
+    """Device scratch df11_decode_host_batch needs for these host matrices
+    (0 for an invalid one); see include/df11.h."""
+    arr = (df11_host_matrix * len(ms))(*ms)
+    return int(load().df11_decode_host_scratch_bytes(arr, len(ms)))
+
+
+def df11_decode_host_batch(ms, h_outs, d_scratch: int, scratch_bytes: int, d_status: int,
+                           stream: int = 0) -> int:
+    """Decode host matrices into host buffers (addresses h_outs), copies and
+    kernels pipelined over the device scratch; see include/df11.h."""
+    arr = (df11_host_matrix * len(ms))(*ms)
+    outs = (ctypes.c_void_p * len(h_outs))(*h_outs)
+    return load().df11_decode_host_batch(arr, len(ms), outs, d_scratch, scratch_bytes, d_status,
+                                         stream)
 
 
 def df11_codebook_from_lengths(lengths: int, cap: int = MAX_CODE_LEN):

@@ -22,7 +22,8 @@ from . import (CODEBOOK_BYTES, MAX_CODE_LEN, SEGMENT, TABLE_BITS, DF11Error, che
                df11_build_codebook, df11_build_segment_index,
                df11_build_codebook_device, df11_build_tables, df11_codebook,
                df11_codebook_from_lengths, df11_decode, df11_decode_block_batch,
-               df11_decode_matmul_batch, df11_decode_gemm_batch, df11_encode, df11_encode_device_codebook, df11_encoded,
+               df11_decode_matmul_batch, df11_decode_gemm_batch, df11_decode_host_batch,
+               df11_decode_host_scratch_bytes, df11_encode, df11_encode_device_codebook, df11_encoded,
                df11_build_run_index, df11_encoded_sizes, df11_file_bytes, df11_histogram,
                df11_host_matrix, df11_matmul_io,
                df11_matrix, df11_read, df11_sizes, df11_sizes_from_bits, df11_tables_bytes,
@@ -348,8 +349,8 @@ def compress_block_device(ws, cap: int = DEFAULT_CAP, stream=None,
 
 def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
                stream=None, run_index: bool = True, seg_index: bool = True) -> torch.Tensor:
-    """Decode one matrix: with its segment index when it has one, else with
-    its run index; seg_index / run_index False leave the index out."""
+    """Decode one matrix: with its run index when it has one, else with its
+    segment index; run_index / seg_index False leave the index out."""
     dev = m.stream.device
     if out is None:
         out = torch.empty(m.shape, dtype=torch.bfloat16, device=dev)
@@ -368,9 +369,9 @@ def decompress(m: DF11Matrix, out: torch.Tensor | None = None, status: torch.Ten
 
 def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=None,
                      run_index: bool = True, seg_index: bool = True):
-    """Decode every matrix of a block in one launch (the segment decoder when
-    every matrix has a segment index, else the indexed decoder when every
-    matrix has a run index; seg_index / run_index False leave them out)."""
+    """Decode every matrix of a block in one launch (the indexed decoder when
+    every matrix has a run index, else the segment decoder when every matrix
+    has a segment index; run_index / seg_index False leave them out)."""
     dev = ms[0].stream.device
     if outs is None:
         outs = [torch.empty(m.shape, dtype=torch.bfloat16, device=dev) for m in ms]
@@ -386,6 +387,74 @@ def decompress_block(ms, outs=None, status: torch.Tensor | None = None, stream=N
         s = int(status.item())
         if s:
             raise DF11Error(s, "df11_decode_block_batch (device)")
+    return outs
+
+
+@dataclass
+class HostMatrix:
+    """A compressed matrix whose stored arrays sit in page-locked host memory:
+    the input of decompress_host (df11_decode_host_batch)."""
+    shape: tuple
+    n: int
+    total_bits: int
+    cap: int
+    max_block_codes: int
+    arrays: dict            # stream, gaps, block_pos, sign_mantissa, lengths: pinned uint8
+
+    @classmethod
+    def from_matrix(cls, m: DF11Matrix) -> "HostMatrix":
+        arrays = {}
+        for k, v in m.host_arrays().items():
+            t = torch.empty(v.nbytes, dtype=torch.uint8, pin_memory=True)
+            t.copy_(torch.from_numpy(np.ascontiguousarray(v).view(np.uint8)))
+            arrays[k] = t
+        return cls(tuple(m.shape), m.n, m.total_bits, int(m.codebook.cap),
+                   int(m.max_block_codes), arrays)
+
+    @property
+    def h2d_bytes(self) -> int:
+        """Bytes one decode copies to the device (the four stored arrays)."""
+        return sum(self.arrays[k].numel() for k in ("stream", "gaps", "block_pos",
+                                                    "sign_mantissa"))
+
+    def abi(self) -> df11_host_matrix:
+        hm = df11_host_matrix(n=self.n, total_bits=self.total_bits, cap=self.cap,
+                              max_block_codes=self.max_block_codes, ndim=0)
+        for k in ("lengths", "gaps", "block_pos", "stream", "sign_mantissa"):
+            setattr(hm, k, self.arrays[k].data_ptr())
+        return hm
+
+
+def host_scratch(hms, device) -> torch.Tensor:
+    """Device scratch for decompress_host over these matrices."""
+    size = df11_decode_host_scratch_bytes([h.abi() for h in hms])
+    if size == 0 and hms:
+        raise DF11Error(1, "df11_decode_host_scratch_bytes")
+    return torch.empty(max(size, 256), dtype=torch.uint8, device=device)
+
+
+def decompress_host(hms, outs=None, scratch: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None, stream=None, device="cuda"):
+    """Decode host-resident matrices into page-locked host BF16 tensors:
+    copies in, run index, decode and copies out pipelined by the library.
+    With a caller's status the call returns with the work queued on stream;
+    without one it waits and raises on a device-reported error."""
+    if outs is None:
+        outs = [torch.empty(h.shape, dtype=torch.bfloat16, pin_memory=True) for h in hms]
+    if scratch is None:
+        scratch = host_scratch(hms, device)
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(1, dtype=torch.int32, device=scratch.device)
+    with torch.cuda.device(scratch.device):
+        check(df11_decode_host_batch([h.abi() for h in hms], [o.data_ptr() for o in outs],
+                                     scratch.data_ptr(), scratch.numel(), status.data_ptr(),
+                                     _stream_handle(stream)), "df11_decode_host_batch")
+    if own_status:
+        (stream if stream is not None else torch.cuda.current_stream(scratch.device)).synchronize()
+        s = int(status.item())
+        if s:
+            raise DF11Error(s, "df11_decode_host_batch (device)")
     return outs
 
 

@@ -3240,3 +3240,274 @@ extern "C" df11_status df11_decode_gemm_batch(const df11_matrix *ms, const df11_
   }
   return DF11_OK;
 }
+
+// ============================================================ decode from host memory, pipelined
+//
+// Matrices held in host memory, decoded into host memory.  Each matrix is cut
+// into pieces of whole decode units (kPieceBlocks blocks), and every piece is
+// a matrix of its own to the kernels: its stored arrays are copied in, its
+// block positions are made relative to its first output, its run index is
+// built, it is decoded, and its BF16 words are copied out to their place in
+// the matrix.  Pieces take turns in kHostSlots slots of the caller's device
+// scratch, and three streams of the call's own carry the copies in, the
+// kernels and the copies out, so that both copy directions and the kernels
+// overlap from one piece to the next.
+namespace {
+
+constexpr uint64_t kHostAlign = 256;
+constexpr uint32_t kHostSlots = 3;
+#ifndef DF11_PIECE_BLOCKS
+#define DF11_PIECE_BLOCKS 4096  // about 26 M values at 2.6 code bits per value
+#endif
+#ifndef DF11_FIRST_PIECE_BLOCKS
+#define DF11_FIRST_PIECE_BLOCKS 256
+#endif
+constexpr uint64_t kPieceBlocks = DF11_PIECE_BLOCKS;
+constexpr uint64_t kFirstPieceBlocks = DF11_FIRST_PIECE_BLOCKS;
+static_assert(kPieceBlocks % kUnitBlocks == 0 && kFirstPieceBlocks % kUnitBlocks == 0 &&
+                  kFirstPieceBlocks <= kPieceBlocks,
+              "pieces are whole decode units");
+constexpr uint64_t kBlockBits = 64ull * DF11_BLOCK_CHUNKS;
+
+inline uint64_t up_to(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// The decode tables of a codebook, built on the device from the codebook
+// itself (a kernel parameter), so the call queues no pageable copy.
+__global__ void __launch_bounds__(kCbThreads) tables_kernel(const __grid_constant__ df11_codebook cb,
+                                                            DecodeTables *__restrict__ t_out) {
+  __shared__ df11cb::TableAux aux;
+  const int t = threadIdx.x;
+  uint32_t *tz = reinterpret_cast<uint32_t *>(t_out);
+  for (uint32_t i = t; i < sizeof(DecodeTables) / 4; i += kCbThreads) tz[i] = 0u;
+  __syncthreads();
+  if (t == 0) df11cb::table_lengths(&cb, t_out, aux);  // checked on the host already
+  __syncthreads();
+  df11cb::table_value(&cb, t_out, t);
+  __syncthreads();
+  for (uint32_t v = t; v < (uint32_t)df11i::kLutSize; v += kCbThreads)
+    t_out->lut[v] = df11cb::lut_entry_for(*t_out, aux, cb.max_len, v);
+}
+
+// Block positions of a piece, made relative to its first output.
+__global__ void rebase_pos_kernel(uint32_t *__restrict__ pos, uint32_t count, uint32_t base) {
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x)
+    pos[i] -= base;
+}
+
+// A piece: blocks [b0, b1) of matrix `mat`, outputs [p0, p1), code bits from
+// the piece's first chunk to its end.
+struct Piece {
+  uint32_t mat;
+  uint64_t b0, b1, p0, p1, bits;
+};
+
+// One piece's arrays in a slot (offsets from the slot).
+struct HostSlot {
+  uint64_t stream, gaps, pos, sm, run_index, out, bytes;
+};
+HostSlot host_slot(const df11_sizes &z) {
+  HostSlot s{};
+  uint64_t o = 0;
+  s.stream = o, o = up_to(o + z.stream_alloc, kHostAlign);
+  s.gaps = o, o = up_to(o + z.gaps_alloc, kHostAlign);
+  s.pos = o, o = up_to(o + z.block_pos_alloc, kHostAlign);
+  s.sm = o, o = up_to(o + z.sign_mantissa_alloc, kHostAlign);
+  s.run_index = o, o = up_to(o + std::max<uint64_t>(16, z.run_index_bytes), kHostAlign);
+  s.out = o, o = up_to(o + 2 * z.n, kHostAlign);
+  s.bytes = o;
+  return s;
+}
+
+uint32_t shortest_code(const uint8_t *len) {
+  uint32_t m = 0;
+  for (int s = 0; s < 256; ++s)
+    if (len[s] && (!m || len[s] < m)) m = len[s];
+  return m;
+}
+
+// Cuts every matrix into pieces and sizes the scratch: the decode tables of
+// every matrix, then kHostSlots slots as large as the largest piece needs.
+// The call's first piece is short (kFirstPieceBlocks), so the first copy out
+// starts early; each piece after it may be twice as long as the one before,
+// up to kPieceBlocks, so the copy in of the next piece still ends before the
+// copy out of the current one.  Few long pieces suit the PCIe link: copies
+// in and out running at once lose bandwidth with every extra pair.  A cut falls between two decode units, and only where the positions stored
+// there are in order and leave the piece at least min_len bits per value
+// (codes running over the cut can shorten a piece by a few bits; such a cut
+// moves on by a unit).  A last piece of one block would hold no code start
+// and joins the piece before it.
+df11_status plan_pieces(const df11_host_matrix *ms, uint32_t count, std::vector<Piece> *pieces,
+                        uint64_t *tables_bytes, uint64_t *slot_bytes) {
+  *tables_bytes = up_to((uint64_t)count * up_to(sizeof(DecodeTables), 16), kHostAlign);
+  *slot_bytes = 0;
+  uint64_t limit = kFirstPieceBlocks;  // doubles with every piece up to kPieceBlocks
+  for (uint32_t i = 0; i < count; ++i) {
+    const df11_host_matrix &h = ms[i];
+    df11_sizes z;
+    df11_status st = df11_sizes_from_bits(h.n, h.total_bits, &z);
+    if (st != DF11_OK) return st;
+    if (!h.n) continue;
+    if (!h.lengths || !h.block_pos || !h.gaps || !h.stream || !h.sign_mantissa)
+      return DF11_ERR_INVALID_ARG;
+    // the decoder's conditions on a matrix (a complete code over at most 256
+    // values has a code of at most 8 bits)
+    const uint32_t ml = shortest_code(h.lengths);
+    if (ml < 1 || ml > 8) return DF11_ERR_INVALID_ARG;
+    if (h.max_block_codes > (64 + ml - 1) / ml * DF11_BLOCK_CHUNKS) return DF11_ERR_INVALID_ARG;
+    const uint64_t B = z.n_blocks;
+    if (h.block_pos[0] != 0 || h.block_pos[B] != h.n) return DF11_ERR_CORRUPT;
+    auto settle = [B](uint64_t b) { return B - b < kUnitBlocks ? B : b; };  // no 1-block tail
+    for (uint64_t b0 = 0; b0 < B;) {
+      auto fits = [&](uint64_t b1) {
+        const uint64_t p1 = h.block_pos[b1], p0 = h.block_pos[b0];
+        return p1 >= p0 && p1 <= h.n && (p1 - p0) * ml <= (b1 - b0) * kBlockBits;
+      };
+      uint64_t b1 = settle(std::min(B, b0 + limit));
+      limit = std::min(2 * limit, kPieceBlocks);
+      while (b1 < B && !fits(b1)) b1 = settle(b1 + kUnitBlocks);
+      Piece pc{i, b0, b1, h.block_pos[b0], h.block_pos[b1],
+               (b1 == B ? h.total_bits : b1 * kBlockBits) - b0 * kBlockBits};
+      if (pc.p1 < pc.p0 || (pc.p1 - pc.p0) * ml > pc.bits) return DF11_ERR_CORRUPT;
+      df11_sizes pz;
+      if (df11_sizes_from_bits(pc.p1 - pc.p0, pc.bits, &pz) != DF11_OK) return DF11_ERR_CORRUPT;
+      *slot_bytes = std::max(*slot_bytes, host_slot(pz).bytes);
+      if (pieces) pieces->push_back(pc);
+      b0 = b1;
+    }
+  }
+  return DF11_OK;
+}
+
+}  // namespace
+
+extern "C" uint64_t df11_decode_host_scratch_bytes(const df11_host_matrix *ms, uint32_t count) {
+  if (!ms && count) return 0;
+  uint64_t tb, sb;
+  if (plan_pieces(ms, count, nullptr, &tb, &sb) != DF11_OK) return 0;
+  return tb + kHostSlots * sb;
+}
+
+extern "C" df11_status df11_decode_host_batch(const df11_host_matrix *ms, uint32_t count,
+                                              uint16_t *const *h_outs, void *d_scratch,
+                                              uint64_t scratch_bytes, uint32_t *d_status,
+                                              df11_stream_t stream) {
+  if (count == 0) return DF11_OK;
+  if (!ms || !h_outs || !d_scratch || !d_status || ((uintptr_t)d_scratch % kHostAlign))
+    return DF11_ERR_INVALID_ARG;
+  // host side first: every matrix's codebook (checked), its pieces, the sizes
+  std::vector<df11_codebook> cbs(count);
+  for (uint32_t i = 0; i < count; ++i) {
+    const df11_host_matrix &h = ms[i];
+    if (h.n > DF11_MAX_N) return DF11_ERR_TOO_LARGE;
+    if (!h.n) continue;
+    if (!h.lengths || !h_outs[i]) return DF11_ERR_INVALID_ARG;
+    const uint32_t cap = h.cap >= 1 && h.cap <= DF11_MAX_CODE_LEN ? h.cap : DF11_MAX_CODE_LEN;
+    df11_status st = df11_codebook_from_lengths(h.lengths, cap, &cbs[i]);
+    if (st != DF11_OK) return st;
+  }
+  std::vector<Piece> pieces;
+  uint64_t tb, sb;
+  df11_status st = plan_pieces(ms, count, &pieces, &tb, &sb);
+  if (st != DF11_OK) return st;
+  if (scratch_bytes < tb + kHostSlots * sb) return DF11_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_info(&dev, &sms)) != DF11_OK) return st;  // a usable device
+
+  uint8_t *base = static_cast<uint8_t *>(d_scratch);
+  const uint64_t tstride = up_to(sizeof(DecodeTables), 16);
+  cudaStream_t caller = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t cs = nullptr, xs = nullptr, ds = nullptr;
+  std::vector<cudaEvent_t> ev;  // every event made here, released at the end
+  auto event = [&](cudaEvent_t *e) {
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    ev.push_back(*e);
+    return true;
+  };
+  cudaEvent_t start = nullptr, slot_free[kHostSlots] = {};
+  bool ok = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&xs, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&ds, cudaStreamNonBlocking) == cudaSuccess && event(&start);
+  // everything starts after the work already queued on the caller's stream
+  ok = ok && cudaEventRecord(start, caller) == cudaSuccess &&
+       cudaStreamWaitEvent(cs, start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(xs, start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(ds, start, 0) == cudaSuccess;
+  // every matrix's decode tables, on the kernel stream
+  for (uint32_t i = 0; ok && i < count; ++i) {
+    if (!ms[i].n) continue;
+    tables_kernel<<<1, kCbThreads, 0, xs>>>(cbs[i], reinterpret_cast<DecodeTables *>(base + i * tstride));
+    ok = cudaGetLastError() == cudaSuccess;
+  }
+  for (size_t k = 0; ok && k < pieces.size(); ++k) {
+    const Piece &pc = pieces[k];
+    const df11_host_matrix &h = ms[pc.mat];
+    df11_sizes hz, z;
+    df11_sizes_from_bits(h.n, h.total_bits, &hz);
+    df11_sizes_from_bits(pc.p1 - pc.p0, pc.bits, &z);
+    const HostSlot L = host_slot(z);
+    const uint32_t slot = (uint32_t)(k % kHostSlots);
+    uint8_t *sp = base + tb + slot * sb;
+    // copy in, once the slot's previous piece has been copied out: the
+    // piece's stream plus the next 16 bytes (read past its last run), its
+    // gaps, positions and sign/mantissa bytes
+    const uint64_t s_off = pc.b0 * (kBlockBits / 8), g_off = pc.b0 * (DF11_GAP_BITS * DF11_BLOCK_CHUNKS / 8);
+    const uint64_t s_len = std::min<uint64_t>(z.stream_bytes + 16, hz.stream_bytes - s_off);
+    const uint64_t g_len = std::min<uint64_t>(z.gaps_bytes + 1, hz.gaps_bytes - g_off);
+    const uint64_t n = pc.p1 - pc.p0;
+    cudaEvent_t in_done, dec_done, freed;
+    ok = event(&in_done) && event(&dec_done) && event(&freed);
+    if (ok && slot_free[slot]) ok = cudaStreamWaitEvent(cs, slot_free[slot], 0) == cudaSuccess;
+    ok = ok &&
+         cudaMemcpyAsync(sp + L.stream, h.stream + s_off, s_len, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+         cudaMemcpyAsync(sp + L.gaps, h.gaps + g_off, g_len, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+         cudaMemcpyAsync(sp + L.pos, h.block_pos + pc.b0, 4 * (pc.b1 - pc.b0 + 1), cudaMemcpyHostToDevice,
+                         cs) == cudaSuccess &&
+         cudaMemcpyAsync(sp + L.sm, h.sign_mantissa + pc.p0, n, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+         cudaEventRecord(in_done, cs) == cudaSuccess;
+    // positions relative to the piece, its run index, its decode
+    df11_matrix m{};
+    m.n = n;
+    m.total_bits = pc.bits;
+    m.stream = sp + L.stream;
+    m.gaps = sp + L.gaps;
+    m.block_pos = reinterpret_cast<const uint32_t *>(sp + L.pos);
+    m.sign_mantissa = sp + L.sm;
+    m.tables = base + pc.mat * tstride;
+    m.min_len = cbs[pc.mat].min_len;
+    m.max_block_codes = h.max_block_codes;
+    uint16_t *d_out = reinterpret_cast<uint16_t *>(sp + L.out);
+    ok = ok && cudaStreamWaitEvent(xs, in_done, 0) == cudaSuccess;
+    if (ok && pc.p0) {
+      const uint32_t cnt = (uint32_t)(pc.b1 - pc.b0 + 1);
+      rebase_pos_kernel<<<(cnt + 255) / 256, 256, 0, xs>>>(reinterpret_cast<uint32_t *>(sp + L.pos), cnt,
+                                                            (uint32_t)pc.p0);
+      ok = cudaGetLastError() == cudaSuccess;
+    }
+    ok = ok && df11_build_run_index(&m, reinterpret_cast<uint16_t *>(sp + L.run_index), d_status,
+                                    reinterpret_cast<df11_stream_t>(xs)) == DF11_OK;
+    m.run_index = reinterpret_cast<const uint16_t *>(sp + L.run_index);
+    ok = ok && launch_decode(&m, 1, &d_out, nullptr, 0, d_status, reinterpret_cast<df11_stream_t>(xs)) == DF11_OK;
+    ok = ok && cudaEventRecord(dec_done, xs) == cudaSuccess;
+    // copy out to the piece's place; the slot is free after it
+    ok = ok && cudaStreamWaitEvent(ds, dec_done, 0) == cudaSuccess &&
+         cudaMemcpyAsync(h_outs[pc.mat] + pc.p0, d_out, 2 * n, cudaMemcpyDeviceToHost, ds) == cudaSuccess &&
+         cudaEventRecord(freed, ds) == cudaSuccess;
+    if (ok) slot_free[slot] = freed;
+  }
+  // the caller's stream waits for all three streams (after a failure too,
+  // for whatever was queued before it uses the scratch)
+  for (cudaStream_t q : {cs, xs, ds}) {
+    cudaEvent_t done;
+    if (!q || !event(&done) || cudaEventRecord(done, q) != cudaSuccess ||
+        cudaStreamWaitEvent(caller, done, 0) != cudaSuccess)
+      ok = false;
+  }
+  // streams and events are released by CUDA once their work completes
+  for (cudaEvent_t e : ev) cudaEventDestroy(e);
+  if (cs) cudaStreamDestroy(cs);
+  if (xs) cudaStreamDestroy(xs);
+  if (ds) cudaStreamDestroy(ds);
+  if (ok) return DF11_OK;
+  cudaGetLastError();
+  return DF11_ERR_CUDA;
+}
