@@ -958,6 +958,52 @@ __device__ __forceinline__ void merge_unit(const Pending &q, uint32_t lin_a, uin
   // starts at byte P0 & 15 >= base8 - (P0 & ~15))
 }
 
+// The same merge with the whole 8-output groups claimed by warps, 32 groups
+// at a time, from a shared counter (*ctr, zero before the first claim): a
+// warp that finished its decoding early merges more of the unit, so the
+// group barrier after the merge waits less for the slowest decoder.
+__device__ __forceinline__ void merge_unit_claimed(const Pending &q, uint32_t lin_a, uint32_t sm_a,
+                                                   int t, uint32_t *ctr) {
+  const uint32_t base8 = q.P0 & ~7u;
+  const uint32_t off8 = base8 - (q.P0 & ~15u);
+  const uint32_t lin8 = lin_a + off8, smb = sm_a + off8;
+  const uint32_t head = q.P0 & 7u;
+  const uint32_t span8 = q.P1 - base8;
+  const uint32_t full0 = head ? 1u : 0u;
+  const uint32_t full1 = span8 >> 3;
+  uint4 *out4 = reinterpret_cast<uint4 *>(q.out + base8);
+  const uint32_t lane = (uint32_t)t & 31u;
+  while (true) {
+    uint32_t c = 0;
+    if (lane == 0) c = atomicAdd(ctr, 32u);
+    c = __shfl_sync(0xffffffffu, c, 0);
+    if (full0 + c >= full1) break;  // (the same for the whole warp)
+    const uint32_t k = full0 + c + lane;
+    if (k < full1) {
+      uint4 r;
+      merge_group8(lin8, smb, k, r);
+      DF11_GLOBAL_CHECK(base8 + 8 * k + 8 <= q.n, continue)
+      out4[k] = r;
+    }
+  }
+  const bool last_edge = (span8 & 7u) != 0 && !(head && full1 == 0);
+  if ((t == 0 && head) || (t == 1 && last_edge)) {
+    const uint32_t k = t == 0 ? 0u : full1;
+    const uint32_t lo = t == 0 ? head : 0u;
+    const uint32_t hi = min(8u, span8 - 8 * k);
+    uint4 r;
+    merge_group8(lin8, smb, k, r);
+    const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
+    uint16_t *o = q.out + base8 + 8 * k;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if ((uint32_t)j >= lo && (uint32_t)j < hi) {
+        DF11_GLOBAL_CHECK(base8 + 8 * k + j < q.n, continue)
+        o[j] = (uint16_t)(wv[j >> 1] >> (16 * (j & 1)));
+      }
+  }
+}
+
 // Fused matmul merge: the unit's decoded weights are multiplied with the
 // activations instead of being stored.  Lane l of warp w takes 8-weight
 // groups w*32 + l, + 256, ... (flat index base8 + 8k, masked to the unit's
@@ -1602,6 +1648,7 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_idx_kernel(const __g
   while (m + 1 < P.count && g0 >= P.unit_start[m + 1]) ++m;
   for (; m < P.count && P.unit_start[m] < g1; ++m) {
     if (__syncthreads_or(timed_out)) return;
+    if (t == 0) meta[4] = meta[12] = 0u;  // the two merge counters (used after a group barrier)
     const uint64_t s0 = max(g0, P.unit_start[m]), s1 = min(g1, P.unit_start[m + 1]);
     if (s0 >= s1) continue;
     const DecMat &M = P.m[m];
@@ -1788,8 +1835,10 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_idx_kernel(const __g
       }
       // ---- the previous unit's merge (its row is the other one)
       if (have_prev) {
-        if (!mbar_wait(bar_sm, (it - 1) & 1)) tmo = true;
-        else if (prev.ok) merge_unit(prev, gbase + (s ? GL.lin0 : GL.lin1), sm_a, t);
+        // (warp-uniform: the claimed merge shuffles across the whole warp)
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_sm, (it - 1) & 1))) tmo = true;
+        else if (prev.ok)
+          merge_unit_claimed(prev, gbase + (s ? GL.lin0 : GL.lin1), sm_a, t, meta + (s ^ 1u) * 8 + 4);
       }
       // ---- [B] the group's flags
       const uint32_t wf = (__ballot_sync(0xffffffffu, bad) ? 1u : 0u) |
@@ -1797,6 +1846,7 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_idx_kernel(const __g
       uint32_t *wfl = wflags + 8 * s;
       if (lane == 0) wfl[warp] = wf;
       group_sync(bar_id);
+      if (t == 0) meta[(s ^ 1u) * 8 + 4] = 0u;  // the merge counter of the unit just merged
       const uint32_t flagbits = __reduce_or_sync(0xffffffffu, lane < kT / 32 ? wfl[lane] : 0u);
       if (flagbits & 2u) {
         if (t == 0) {
@@ -1825,12 +1875,14 @@ __global__ void __launch_bounds__(kT *kMaxGroups, 1) decode_idx_kernel(const __g
     }
     if (!timed_out && have_prev) {
       group_sync(bar_id);
-      const bool got = mbar_wait(bar_sm, (it - 1) & 1);
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar_sm, (it - 1) & 1));
       if (!got) {
         if (lane == 0) set_status(P.status, DF11_ERR_TIMEOUT);
         timed_out = true;
       }
-      if (got && prev.ok) merge_unit(prev, gbase + (((it - 1) & 1) ? GL.lin1 : GL.lin0), sm_a, t);
+      if (got && prev.ok)
+        merge_unit_claimed(prev, gbase + (((it - 1) & 1) ? GL.lin1 : GL.lin0), sm_a, t,
+                           meta + ((it - 1) & 1u) * 8 + 4);
     }
   }
 }
