@@ -930,11 +930,19 @@ __device__ __forceinline__ void merge_unit(const Pending &q, uint32_t lin_a, uin
   const uint32_t full0 = head ? 1u : 0u;
   const uint32_t full1 = span8 >> 3;
   uint4 *out4 = reinterpret_cast<uint4 *>(q.out + base8);
-  for (uint32_t k = full0 + t; k < full1; k += kT) {
-    uint4 r;
-    merge_group8(lin8, smb, k, r);
-    DF11_GLOBAL_CHECK(base8 + 8 * k + 8 <= q.n, continue)
-    out4[k] = r;
+  // four independent groups per thread and pass: their shared-memory reads
+  // overlap
+  for (uint32_t k0 = full0 + t; k0 < full1; k0 += 4 * kT) {
+#pragma unroll
+    for (uint32_t j = 0; j < 4; ++j) {
+      const uint32_t k = k0 + j * kT;
+      if (k < full1) {
+        uint4 r;
+        merge_group8(lin8, smb, k, r);
+        DF11_GLOBAL_CHECK(base8 + 8 * k + 8 <= q.n, continue)
+        out4[k] = r;
+      }
+    }
   }
   // ragged first group (thread 0) and last group (thread 1, unless it is the
   // first one); element j of group k is output base8 + 8k + j
@@ -958,10 +966,15 @@ __device__ __forceinline__ void merge_unit(const Pending &q, uint32_t lin_a, uin
   // starts at byte P0 & 15 >= base8 - (P0 & ~15))
 }
 
-// The same merge with the whole 8-output groups claimed by warps, 32 groups
-// at a time, from a shared counter (*ctr, zero before the first claim): a
-// warp that finished its decoding early merges more of the unit, so the
-// group barrier after the merge waits less for the slowest decoder.
+// The same merge with the whole 8-output groups claimed by warps,
+// kMergeClaim groups at a time (four per lane), from a shared counter (*ctr,
+// zero before the first claim): a warp that finished its decoding early
+// merges more of the unit, so the group barrier after the merge waits less
+// for the slowest decoder, and each lane's four groups are independent work.
+// (Measured on a Llama-3-70B-shaped block of 855 M weights: claims of 32 /
+// 64 / 96 / 128 / 160 / 256 groups gave 0.662 / 0.627 / 0.635 / 0.608 /
+// 0.608 / 0.628 ms per launch.)
+constexpr uint32_t kMergeClaim = 128;
 __device__ __forceinline__ void merge_unit_claimed(const Pending &q, uint32_t lin_a, uint32_t sm_a,
                                                    int t, uint32_t *ctr) {
   const uint32_t base8 = q.P0 & ~7u;
@@ -975,15 +988,20 @@ __device__ __forceinline__ void merge_unit_claimed(const Pending &q, uint32_t li
   const uint32_t lane = (uint32_t)t & 31u;
   while (true) {
     uint32_t c = 0;
-    if (lane == 0) c = atomicAdd(ctr, 32u);
+    if (lane == 0) c = atomicAdd(ctr, kMergeClaim);
     c = __shfl_sync(0xffffffffu, c, 0);
     if (full0 + c >= full1) break;  // (the same for the whole warp)
-    const uint32_t k = full0 + c + lane;
-    if (k < full1) {
-      uint4 r;
-      merge_group8(lin8, smb, k, r);
-      DF11_GLOBAL_CHECK(base8 + 8 * k + 8 <= q.n, continue)
-      out4[k] = r;
+    // kMergeClaim / 32 independent groups per lane: their shared-memory
+    // reads overlap
+#pragma unroll
+    for (uint32_t j = 0; j < kMergeClaim; j += 32) {
+      const uint32_t k = full0 + c + j + lane;
+      if (k < full1) {
+        uint4 r;
+        merge_group8(lin8, smb, k, r);
+        DF11_GLOBAL_CHECK(base8 + 8 * k + 8 <= q.n, continue)
+        out4[k] = r;
+      }
     }
   }
   const bool last_edge = (span8 & 7u) != 0 && !(head && full1 == 0);
